@@ -1,0 +1,382 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Every check here computes the expected value another way than the oracle
+does: hand-worked formula values, brute force, textbook library routines
+(numpy.linalg.norm, torch SDPA, torch autograd), finite differences and
+adjoint identities.  CPU only.
+"""
+
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lighthouse_oracle as lo
+from oracle import gap_repair
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- sizes
+
+def test_gathered_length_and_entry_count_golden():
+    with open(os.path.join(GOLDEN, "gathered_lengths.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        N, p, L, k = c["N"], c["p"], c["L"], c["k"]
+        assert lo.pyramid_entry_count(N, p, L) == c["entries"], c["name"]
+        assert lo.gathered_length(N, p, L, k) == c["S"], c["name"]
+        # the page formula itself, where every level has at least k candidates
+        if all(k <= N // p ** (l + 1) for l in range(L - 1)):
+            assert c["S"] == c["S_formula"] == N // p ** (L - 1) + (L - 1) * p * k
+
+
+@pytest.mark.parametrize("N,p,L,k", [(64, 2, 3, 5), (256, 4, 3, 7), (512, 2, 5, 9), (96, 2, 4, 100)])
+def test_sequence_length_matches_formula(N, p, L, k):
+    r = rng(1)
+    Q, K, V = (r.standard_normal((N, 4)) for _ in range(3))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=16)
+    assert len(sv["seq_level"]) == lo.gathered_length(N, p, L, k)
+    # levels: the top level whole, each other level p*min(k, M) entries
+    counts = np.bincount(sv["seq_level"], minlength=L)
+    assert counts[L - 1] == N // p ** (L - 1)
+    for l in range(L - 1):
+        assert counts[l] == p * min(k, N // p ** (l + 1))
+
+
+# ---------------------------------------------------------------- pooling
+
+def test_pool_equals_block_means_by_loops():
+    r = rng(2)
+    N, d, p, L = 48, 3, 2, 4
+    X = r.standard_normal((N, d))
+    levels = lo.pyramid_pool(X, p, L)
+    for l in range(L):
+        b = p ** l
+        assert levels[l].shape == (N // b, d)
+        for i in range(N // b):
+            for c in range(d):
+                want = sum(X[t, c] for t in range(i * b, (i + 1) * b)) / b
+                assert abs(levels[l][i, c] - want) < 1e-13
+
+
+def test_pool_equals_reshape_mean_p4():
+    r = rng(3)
+    X = r.standard_normal((256, 5))
+    levels = lo.pyramid_pool(X, 4, 4)
+    for l in range(4):
+        np.testing.assert_allclose(levels[l], X.reshape(256 // 4 ** l, 4 ** l, 5).mean(axis=1), rtol=0, atol=1e-14)
+
+
+def test_entry_count_is_sum_of_level_sizes():
+    X = np.zeros((1024, 2))
+    for p, L in [(2, 1), (2, 6), (4, 5), (8, 3)]:
+        lv = lo.pyramid_pool(X, p, L)
+        assert sum(x.shape[0] for x in lv) == lo.pyramid_entry_count(1024, p, L)
+        # O(N): bounded by N * p / (p - 1)
+        assert lo.pyramid_entry_count(1024, p, L) <= 1024 * p / (p - 1)
+
+
+# ---------------------------------------------------------------- scores
+
+@pytest.mark.parametrize("scorer", ["qk_sum", "k", "q"])
+def test_scores_vs_linalg_norm(scorer):
+    r = rng(4)
+    Q, K = r.standard_normal((40, 7)), r.standard_normal((40, 7))
+    nq, nk = np.linalg.norm(Q, axis=1), np.linalg.norm(K, axis=1)
+    want = {"qk_sum": nq + nk, "k": nk, "q": nq}[scorer]
+    np.testing.assert_allclose(lo.level0_scores(Q, K, scorer), want, rtol=1e-15)
+
+
+def test_score_pyramid_is_block_max_of_level0():
+    r = rng(5)
+    s0 = r.random(128)
+    sp = lo.score_pyramid(s0, 2, 5)
+    for l in range(5):
+        b = 2 ** l
+        for i in range(128 // b):
+            assert sp[l][i] == max(s0[i * b:(i + 1) * b])
+
+
+# ---------------------------------------------------------------- top-k
+
+def brute_topk(scores, k, T):
+    """Exhaustive: in every chunk (numpy.array_split), the q-subset with the
+    largest score sum, ties broken by the lexicographically smallest set."""
+    M = len(scores)
+    C = max(1, M // T)
+    kp = min(k, M)
+    out = []
+    for c, chunk in enumerate(np.array_split(np.arange(M), C)):
+        q = kp // C + (1 if c < kp % C else 0)
+        best = None
+        for sub in itertools.combinations(chunk.tolist(), q):
+            key = (-sum(scores[m] for m in sub), sub)
+            if best is None or key < best:
+                best = key
+        out.extend(best[1])
+    return np.array(sorted(out), dtype=np.int64)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_stratified_topk_bruteforce(seed):
+    r = rng(100 + seed)
+    M = int(r.integers(1, 13))
+    k = int(r.integers(1, 6))
+    T = int(r.integers(1, 8))
+    scores = r.integers(0, 4, M).astype(np.float64)  # many exact ties
+    got = lo.stratified_topk(scores, k, T)
+    np.testing.assert_array_equal(got, brute_topk(scores, k, T))
+
+
+def test_topk_single_chunk_is_stable_argsort():
+    r = rng(6)
+    s = r.integers(0, 5, 500).astype(np.float64)
+    got = lo.stratified_topk(s, 37, T=10_000)
+    want = np.sort(np.argsort(-s, kind="stable")[:37])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_selection_invariants():
+    r = rng(7)
+    N, p, L, k = 1024, 2, 5, 13
+    Q, K = r.standard_normal((N, 8)), r.standard_normal((N, 8))
+    sel, _ = lo.select(Q, K, p, L, k, T=64)
+    ent = lo.selected_entries(sel, N, p, L)
+    np.testing.assert_array_equal(ent[L - 1], np.arange(N // p ** (L - 1)))  # top level whole
+    for l in range(L - 1):
+        e = ent[l]
+        assert len(e) == p * min(k, N // p ** (l + 1))
+        assert np.all(np.diff(e) > 0)  # sorted, no duplicates
+        groups = e.reshape(-1, p)  # complete sibling groups
+        assert np.all(groups % p == np.arange(p)) and np.all(groups[:, 0] // p == sel[l])
+
+
+# ---------------------------------------------------------------- gather order
+
+def test_causal_order_invariants():
+    r = rng(8)
+    N, p, L, k = 512, 4, 4, 6
+    Q, K, V = (r.standard_normal((N, 4)) for _ in range(3))
+    _, sv = lo.forward_head(Q, K, V, p, L, k, T=32)
+    lv, ix = sv["seq_level"], sv["seq_index"]
+    last = (ix + 1) * p ** lv - 1
+    # keys (e, -l) strictly increasing: a valid causal order with no duplicate
+    keys = list(zip(last.tolist(), (-lv).tolist()))
+    assert all(a < b for a, b in zip(keys, keys[1:]))
+    # slot_of inverts the sequence map, and -1 marks the rest
+    for s, (l, i) in enumerate(zip(lv, ix)):
+        assert sv["slot_of"][l][i] == s
+    assert sum(int((t >= 0).sum()) for t in sv["slot_of"]) == len(lv)
+
+
+# ---------------------------------------------------------------- attention
+
+def torch_causal(Qs, Ks, Vs):
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x))[None, None] for x in (Qs, Ks, Vs))
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)[0, 0].numpy()
+
+
+def test_L1_is_dense_causal_attention():
+    r = rng(9)
+    Q, K, V = (r.standard_normal((300, 16)) for _ in range(3))
+    Y, sv = lo.forward_head(Q, K, V, p=2, L=1, k=5)
+    assert len(sv["seq_level"]) == 300
+    np.testing.assert_allclose(Y, torch_causal(Q, K, V), rtol=0, atol=1e-12)
+
+
+def test_attention_lse_and_rows_sum_to_one():
+    r = rng(10)
+    Qs, Ks = r.standard_normal((700, 8)), r.standard_normal((700, 8))
+    O, lse = lo.causal_attention(Qs, Ks, np.ones((700, 3)))
+    np.testing.assert_allclose(O, 1.0, rtol=0, atol=1e-13)
+    want = [np.log(np.sum(np.exp(Qs[t] @ Ks[:t + 1].T / np.sqrt(8)))) for t in range(0, 700, 37)]
+    np.testing.assert_allclose(lse[::37], want, rtol=1e-13)
+
+
+def position_formula(Os, slot_of, N, p, L):
+    """Y_j = sum_l [entry (l, floor((j+1)/p^l) - 1) kept] * Os[slot], by loops."""
+    Y = np.zeros((N, Os.shape[1]))
+    for j in range(N):
+        for l in range(L):
+            i = (j + 1) // p ** l - 1
+            if 0 <= i < len(slot_of[l]) and slot_of[l][i] >= 0:
+                Y[j] += Os[slot_of[l][i]]
+    return Y
+
+
+def test_full_budget_equals_dense_attention_over_sorted_pyramid():
+    r = rng(11)
+    N, p, L, d = 64, 2, 4, 8
+    Q, K, V = (r.standard_normal((N, d)) for _ in range(3))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k=10 ** 6)
+    # independent construction: every pyramid entry, sorted with Python's sort
+    pyr = [lo.pyramid_pool(X, p, L) for X in (Q, K, V)]
+    entries = sorted(((i + 1) * p ** l - 1, -l, l, i) for l in range(L) for i in range(N // p ** l))
+    assert len(entries) == lo.pyramid_entry_count(N, p, L)
+    seq = [[pyr[t][l][i] for (_, _, l, i) in entries] for t in range(3)]
+    Os = torch_causal(np.array(seq[0]), np.array(seq[1]), np.array(seq[2]))
+    slot_of = [np.full(N // p ** l, -1) for l in range(L)]
+    for s, (_, _, l, i) in enumerate(entries):
+        slot_of[l][i] = s
+    np.testing.assert_allclose(Y, position_formula(Os, slot_of, N, p, L), rtol=0, atol=1e-12)
+
+
+def test_scatter_matches_position_formula_with_partial_selection():
+    r = rng(12)
+    N, p, L, k = 96, 2, 4, 3
+    Q, K, V = (r.standard_normal((N, 5)) for _ in range(3))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=8)
+    np.testing.assert_allclose(Y, position_formula(sv["Os"], sv["slot_of"], N, p, L), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- causality
+
+def test_causality_value_perturbation():
+    r = rng(13)
+    N, p, L, k = 128, 2, 4, 4
+    Q, K, V = (r.standard_normal((N, 6)) for _ in range(3))
+    Y0, _ = lo.forward_head(Q, K, V, p, L, k, T=16)
+    for j in (0, 5, 31, 64, 126):
+        V2 = V.copy()
+        V2[j + 1] += 10.0
+        Y1, _ = lo.forward_head(Q, K, V2, p, L, k, T=16)
+        np.testing.assert_array_equal(Y1[:j + 1], Y0[:j + 1])
+        assert np.abs(Y1[j + 1:] - Y0[j + 1:]).max() > 0
+
+
+def test_causality_query_key_perturbation_with_frozen_selection():
+    r = rng(14)
+    N, p, L, k = 128, 4, 3, 3
+    Q, K, V = (r.standard_normal((N, 6)) for _ in range(3))
+    Y0, sv = lo.forward_head(Q, K, V, p, L, k, T=16)
+    for j in (2, 40, 100):
+        Q2, K2 = Q.copy(), K.copy()
+        Q2[j + 1] *= 3.0
+        K2[j + 1] -= 1.0
+        Y1, _ = lo.forward_head(Q2, K2, V, p, L, k, T=16, sel=sv["sel"])
+        np.testing.assert_array_equal(Y1[:j + 1], Y0[:j + 1])
+
+
+# ---------------------------------------------------------------- backward
+
+def test_finite_differences():
+    r = rng(15)
+    N, d, p, L, k = 32, 8, 2, 3, 2
+    Q, K, V, G = (r.standard_normal((N, d)) for _ in range(4))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k)
+    dQ, dK, dV, _ = lo.backward_head(G, sv)
+    h = 1e-6
+    for X, dX, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
+        num = np.zeros_like(X)
+        for t in range(N):
+            for c in range(d):
+                args_p = [Q.copy(), K.copy(), V.copy()]
+                args_m = [Q.copy(), K.copy(), V.copy()]
+                args_p[which][t, c] += h
+                args_m[which][t, c] -= h
+                Yp, svp = lo.forward_head(*args_p, p, L, k)
+                Ym, svm = lo.forward_head(*args_m, p, L, k)
+                for a, b in zip(svp["sel"] + svm["sel"], sv["sel"] + sv["sel"]):
+                    np.testing.assert_array_equal(a, b)  # selection unchanged at +-h
+                num[t, c] = (np.sum(Yp * G) - np.sum(Ym * G)) / (2 * h)
+        rel = np.abs(num - dX).max() / np.abs(dX).max()
+        assert rel < 1e-6, (which, rel)
+
+
+def test_gradient_of_token_covered_only_by_the_top_level():
+    # Top-k passes no gradient: a token whose only kept entry is its top-level
+    # parent gets exactly 1/p^(L-1) of that slot's gradient (pool adjoint).
+    r = rng(16)
+    N, d, p, L, k = 64, 4, 2, 2, 1
+    Q, K, V, G = (r.standard_normal((N, d)) for _ in range(4))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=64)
+    dQ, dK, dV, ex = lo.backward_head(G, sv)
+    kept0 = set(sv["seq_index"][sv["seq_level"] == 0].tolist())
+    assert len(kept0) == p * k
+    for t in range(N):
+        parent = sv["slot_of"][1][t // p]
+        assert parent >= 0
+        if t not in kept0:
+            np.testing.assert_allclose(dQ[t], ex["dQs"][parent] / p, rtol=1e-14, atol=0)
+            np.testing.assert_allclose(dV[t], ex["dVs"][parent] / p, rtol=1e-14, atol=0)
+
+
+def _adjoint_check(fwd, adj, x, y):
+    lhs = np.sum(fwd(x) * y)
+    rhs = np.sum(x * adj(y))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+
+
+def test_adjoint_identities():
+    r = rng(17)
+    N, d, p, L, k = 64, 3, 2, 4, 3
+    Q, K, V = (r.standard_normal((N, d)) for _ in range(3))
+    _, sv = lo.forward_head(Q, K, V, p, L, k, T=8)
+    sl, si = sv["seq_level"], sv["seq_index"]
+    S = len(sl)
+    # scatter_back and scatter_adjoint
+    _adjoint_check(lambda o: lo.scatter_back(o, sl, si, N, p, L),
+                   lambda y: lo.scatter_adjoint(y, sl, si, N, p),
+                   r.standard_normal((S, d)), r.standard_normal((N, d)))
+    # pool+gather and its adjoint
+    _adjoint_check(lambda x: lo.gather(lo.pyramid_pool(x, p, L), sl, si),
+                   lambda g: lo.pyramid_pool_adjoint(lo.gather_adjoint(g, sl, si, N, p, L), p),
+                   r.standard_normal((N, d)), r.standard_normal((S, d)))
+
+
+def test_backward_matches_torch_autograd():
+    """The hand-derived adjoints against torch autograd of an independently
+    written differentiable forward (same frozen sequence order)."""
+    r = rng(18)
+    N, d, p, L, k = 256, 16, 4, 3, 5
+    Q, K, V, G = (r.standard_normal((N, d)) for _ in range(4))
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=32)
+    dQ, dK, dV, _ = lo.backward_head(G, sv)
+    lv = torch.from_numpy(sv["seq_level"])
+    ix = torch.from_numpy(sv["seq_index"])
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+
+    def seq(X):
+        rows = []
+        for l, i in zip(lv.tolist(), ix.tolist()):
+            b = p ** l
+            rows.append(X[i * b:(i + 1) * b].mean(0))
+        return torch.stack(rows)
+
+    O = torch.nn.functional.scaled_dot_product_attention(seq(tq)[None], seq(tk)[None], seq(tv)[None], is_causal=True)[0]
+    Yt = torch.zeros(N, d, dtype=torch.float64)
+    for s, (l, i) in enumerate(zip(lv.tolist(), ix.tolist())):
+        a, b = (i + 1) * p ** l - 1, min(N, (i + 2) * p ** l - 1)
+        Yt = Yt.index_add(0, torch.arange(a, b), O[s].expand(b - a, d))
+    np.testing.assert_allclose(Yt.detach().numpy(), Y, rtol=0, atol=1e-12)
+    (Yt * torch.from_numpy(G)).sum().backward()
+    for got, want in ((dQ, tq.grad), (dK, tk.grad), (dV, tv.grad)):
+        np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------- gap repair
+
+def test_gap_repair_removes_near_ties():
+    from hierarchical_sparse_attention_pyramid_b200 import synth
+    w = synth.WORKLOADS["tiny_4k_fp32"]
+    h = synth.head_inputs(w, 0)
+    Q, K, n = gap_repair.repair_head(h["q"], h["k"], w.p, w.L, w.k, w.chunk, w.scorer)
+    assert gap_repair.near_ties(Q.double().numpy(), K.double().numpy(), w.p, w.L, w.k, w.chunk, w.scorer) == []
+    assert n < 0.01 * w.N
+    # a planted exact tie at the selection boundary: level-1 candidate scores
+    # (max over pairs of |K|) are 8, 6, 6, 2 and k=2 puts the boundary
+    # between the two 6s; the lower index wins, so token 5 is pushed down
+    Kt = torch.tensor([8, 1, 6, 1, 1, 6, 2, 1], dtype=torch.float32)[:, None]
+    Qt = torch.zeros_like(Kt)
+    assert gap_repair.near_ties(Qt.double().numpy(), Kt.double().numpy(), 2, 2, 2, 2048, "k") == [5]
+    Q2, K2, n2 = gap_repair.repair_head(Qt, Kt, 2, 2, 2, 2048, "k")
+    assert n2 == 1 and float(K2[5, 0]) == np.float32(6 * 0.98)
+    assert gap_repair.near_ties(Q2.double().numpy(), K2.double().numpy(), 2, 2, 2, 2048, "k") == []
