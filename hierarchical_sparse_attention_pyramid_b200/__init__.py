@@ -1,5 +1,10 @@
 """B200-native Lighthouse attention layer (hierarchical sparse attention pyramid).
 
 The compute path is the CUDA library ``liblh.so`` (C ABI, ``include/lh.h``);
-this package only marshals torch tensors into its calls.
+this package only marshals torch tensors into its calls.  ``synth`` draws the
+seeded synthetic inputs.
 """
+
+from .api import (Buffers, Layer, LighthouseAttentionFn, attn_bwd, attn_fwd, backward, check_error, forward,  # noqa: F401
+                  gather, lighthouse_attention, plan, pool_adjoint, pyramid_pool, scatter_back,
+                  scatter_back_adjoint, score_topk)

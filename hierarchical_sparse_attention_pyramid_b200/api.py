@@ -1,0 +1,244 @@
+"""torch front end of liblh: marshals CUDA tensors into the C ABI calls.
+
+Every function allocates its outputs with torch (device memory) and passes
+raw pointers and the current CUDA stream to liblh; all arithmetic runs in the
+library's kernels.  Shapes follow include/lh.h: Q, K, V, Y and their
+gradients are [B, H, N, d]; the gathered sequence tensors are [B*H, S, d].
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import LhConfig, LhPlanInfo, call
+
+_TORCH_DTYPE = {"bf16": torch.bfloat16, "fp32": torch.float32}
+
+
+@dataclass(frozen=True)
+class Layer:
+    """Shape and method parameters of one Lighthouse attention layer."""
+    B: int
+    H: int
+    N: int
+    d: int
+    L: int
+    p: int
+    k: int
+    chunk: int = 2048
+    dtype: str = "bf16"
+    scorer: str = "qk_sum"
+
+    def cfg(self) -> LhConfig:
+        return LhConfig(self.B, self.H, self.N, self.d, self.L, self.p, self.k, self.chunk,
+                        _lib.DTYPES[self.dtype], _lib.SCORERS[self.scorer])
+
+    @property
+    def torch_dtype(self):
+        return _TORCH_DTYPE[self.dtype]
+
+    @property
+    def BH(self):
+        return self.B * self.H
+
+    @staticmethod
+    def of(w) -> "Layer":
+        """From a synth.Workload (or anything with the same fields)."""
+        return Layer(w.B, w.H, w.N, w.d, w.L, w.p, w.k, w.chunk, w.dtype, w.scorer)
+
+
+def plan(layer: Layer) -> LhPlanInfo:
+    info = LhPlanInfo()
+    call("lh_plan", ctypes.byref(layer.cfg()), ctypes.byref(info))
+    return info
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("liblh takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("liblh takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.zeros(max(nbytes, _lib.ERR_WORD_BYTES), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ stages
+
+def pyramid_pool(layer: Layer, q, k, v):
+    """-> pyr_q, pyr_k, pyr_v [BH, upper_entries, d] (levels >= 1), norms [2, BH, N] fp32."""
+    info = plan(layer)
+    dev = q.device
+    shp = (layer.BH, max(info.upper_entries, 1), layer.d)
+    pq, pk, pv = (_empty(shp, layer.torch_dtype, dev) for _ in range(3))
+    norms = _empty((2, layer.BH, layer.N), torch.float32, dev)
+    call("lh_pyramid_pool", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(norms), _stream())
+    return pq, pk, pv, norms
+
+
+def score_topk(layer: Layer, norms, ws=None):
+    """-> sel [BH, sel_per_head] int32 (per level l at sel_off[l], ascending parents at level l+1)."""
+    info = plan(layer)
+    dev = norms.device
+    sel = torch.zeros((layer.BH, max(info.sel_per_head, 1)), dtype=torch.int32, device=dev)
+    ws = _ws(info.topk_ws_bytes, dev) if ws is None else ws
+    call("lh_score_topk", ctypes.byref(layer.cfg()), _p(norms), _p(ws), _p(sel), _stream())
+    return sel
+
+
+def gather(layer: Layer, q, k, v, pq, pk, pv, sel):
+    """-> qs, ks, vs [BH, S, d] bf16, seq_map [BH, S] int32, slot_of [BH, pyr_entries] int32."""
+    info = plan(layer)
+    dev = q.device
+    S = info.S
+    qs, ks, vs = (_empty((layer.BH, S, layer.d), torch.bfloat16, dev) for _ in range(3))
+    seq_map = _empty((layer.BH, S), torch.int32, dev)
+    slot_of = _empty((layer.BH, info.pyr_entries), torch.int32, dev)
+    call("lh_gather", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(sel),
+         _p(qs), _p(ks), _p(vs), _p(seq_map), _p(slot_of), _stream())
+    return qs, ks, vs, seq_map, slot_of
+
+
+def attn_fwd(layer: Layer, qs, ks, vs, ws=None):
+    """Causal attention over the sequence -> os [BH, S, d] bf16, lse [BH, S] fp32."""
+    BH, S, d = qs.shape
+    os_ = _empty((BH, S, d), torch.bfloat16, qs.device)
+    lse = _empty((BH, S), torch.float32, qs.device)
+    ws = _ws(0, qs.device) if ws is None else ws
+    call("lh_attn_fwd", ctypes.byref(layer.cfg()), ctypes.c_int64(S), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse),
+         _p(ws), _stream())
+    return os_, lse
+
+
+def attn_bwd(layer: Layer, qs, ks, vs, lse, dos, delta, ws=None):
+    """-> dqs, dks, dvs [BH, S, d] fp32."""
+    BH, S, d = qs.shape
+    dqs, dks, dvs = (_empty((BH, S, d), torch.float32, qs.device) for _ in range(3))
+    ws = _ws(0, qs.device) if ws is None else ws
+    call("lh_attn_bwd", ctypes.byref(layer.cfg()), ctypes.c_int64(S), _p(qs), _p(ks), _p(vs), _p(lse), _p(dos),
+         _p(delta), _p(dqs), _p(dks), _p(dvs), _p(ws), _stream())
+    return dqs, dks, dvs
+
+
+def scatter_back(layer: Layer, os_, slot_of):
+    y = _empty((layer.B, layer.H, layer.N, layer.d), layer.torch_dtype, os_.device)
+    call("lh_scatter_back", ctypes.byref(layer.cfg()), _p(os_), _p(slot_of), _p(y), _stream())
+    return y
+
+
+def scatter_back_adjoint(layer: Layer, dy, seq_map, os_):
+    BH, S, d = os_.shape
+    dos = _empty((BH, S, d), torch.bfloat16, dy.device)
+    delta = _empty((BH, S), torch.float32, dy.device)
+    call("lh_scatter_back_adjoint", ctypes.byref(layer.cfg()), _p(dy), _p(seq_map), _p(os_), _p(dos), _p(delta),
+         _stream())
+    return dos, delta
+
+
+def pool_adjoint(layer: Layer, dqs, dks, dvs, slot_of):
+    shp = (layer.B, layer.H, layer.N, layer.d)
+    dq, dk, dv = (_empty(shp, layer.torch_dtype, dqs.device) for _ in range(3))
+    call("lh_pool_adjoint", ctypes.byref(layer.cfg()), _p(dqs), _p(dks), _p(dvs), _p(slot_of), _p(dq), _p(dk),
+         _p(dv), _stream())
+    return dq, dk, dv
+
+
+# ------------------------------------------------------------------ whole layer
+
+class Buffers:
+    """Saved context and scratch of one layer shape, reusable across steps."""
+
+    def __init__(self, layer: Layer, device):
+        self.layer = layer
+        self.info = plan(layer)
+        self.ctx = torch.empty(self.info.ctx_bytes, dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(self.info.ws_bytes, dtype=torch.uint8, device=device)
+
+    def ctx_views(self) -> dict:
+        """Typed views of what lh_forward saved (for inspection and tests)."""
+        I, Lr = self.info, self.layer
+        S, BH, d = I.S, Lr.BH, Lr.d
+
+        def view(off, n, dtype, shape):
+            esz = torch.empty((), dtype=dtype).element_size()
+            return self.ctx[off:off + n * esz].view(dtype).view(shape)
+
+        return dict(
+            sel=view(I.ctx_off_sel, BH * I.sel_per_head, torch.int32, (BH, I.sel_per_head)),
+            seq_map=view(I.ctx_off_seq_map, BH * S, torch.int32, (BH, S)),
+            slot_of=view(I.ctx_off_slot_of, BH * I.pyr_entries, torch.int32, (BH, I.pyr_entries)),
+            qs=view(I.ctx_off_qs, BH * S * d, torch.bfloat16, (BH, S, d)),
+            ks=view(I.ctx_off_ks, BH * S * d, torch.bfloat16, (BH, S, d)),
+            vs=view(I.ctx_off_vs, BH * S * d, torch.bfloat16, (BH, S, d)),
+            os=view(I.ctx_off_os, BH * S * d, torch.bfloat16, (BH, S, d)),
+            lse=view(I.ctx_off_lse, BH * S, torch.float32, (BH, S)),
+        )
+
+
+def forward(layer: Layer, q, k, v, bufs: Buffers | None = None, y=None):
+    """Whole forward -> (y, bufs).  bufs holds the saved context for backward."""
+    bufs = Buffers(layer, q.device) if bufs is None else bufs
+    y = _empty((layer.B, layer.H, layer.N, layer.d), layer.torch_dtype, q.device) if y is None else y
+    call("lh_forward", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(y), _p(bufs.ctx),
+         ctypes.c_size_t(bufs.info.ctx_bytes), _p(bufs.ws), ctypes.c_size_t(bufs.info.ws_bytes), _stream())
+    return y, bufs
+
+
+def backward(layer: Layer, dy, bufs: Buffers, grads=None):
+    """Whole backward from the saved context -> (dq, dk, dv)."""
+    shp = (layer.B, layer.H, layer.N, layer.d)
+    if grads is None:
+        grads = tuple(_empty(shp, layer.torch_dtype, dy.device) for _ in range(3))
+    dq, dk, dv = grads
+    call("lh_backward", ctypes.byref(layer.cfg()), _p(dy), _p(bufs.ctx), ctypes.c_size_t(bufs.info.ctx_bytes),
+         _p(dq), _p(dk), _p(dv), _p(bufs.ws), ctypes.c_size_t(bufs.info.ws_bytes), _stream())
+    return dq, dk, dv
+
+
+def check_error(bufs_or_ws) -> None:
+    """Synchronise and raise if a kernel reported a timeout or a bad index."""
+    ws = bufs_or_ws.ws if isinstance(bufs_or_ws, Buffers) else bufs_or_ws
+    call("lh_check_error", _p(ws), _stream())
+
+
+class LighthouseAttentionFn(torch.autograd.Function):
+    """Autograd wrapper: forward saves liblh's context, backward consumes it.
+    The top-k selection is not differentiable; gradients reach Q, K, V only
+    through the pooled values."""
+
+    @staticmethod
+    def forward(fn_ctx, q, k, v, layer: Layer):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        y, bufs = forward(layer, q, k, v)
+        fn_ctx.layer = layer
+        fn_ctx.bufs = bufs
+        return y
+
+    @staticmethod
+    def backward(fn_ctx, dy):
+        dq, dk, dv = backward(fn_ctx.layer, dy.contiguous(), fn_ctx.bufs)
+        return dq, dk, dv, None
+
+
+def lighthouse_attention(q, k, v, L: int, p: int, k_budget: int, chunk: int = 2048, scorer: str = "qk_sum"):
+    """One Lighthouse attention layer over causal q, k, v of shape [B, H, N, d]."""
+    B, H, N, d = q.shape
+    dtype = {torch.bfloat16: "bf16", torch.float32: "fp32"}[q.dtype]
+    layer = Layer(B, H, N, d, L, p, k_budget, chunk, dtype, scorer)
+    return LighthouseAttentionFn.apply(q, k, v, layer)

@@ -1,0 +1,378 @@
+// C ABI of liblh: argument checks, planning of the buffers, and the stage and
+// whole-layer entry points declared in include/lh.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "lh_common.cuh"
+
+namespace lh {
+
+static thread_local char g_msg[512] = "";
+
+void set_error_message(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+lh_status fail(lh_status s, const char* what) {
+  set_error_message("%s", what);
+  return s;
+}
+
+lh_status cuda_fail(cudaError_t e, const char* where) {
+  set_error_message("%s: %s", where, cudaGetErrorString(e));
+  return LH_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ilog2(int64_t x) {
+  int r = 0;
+  while (((int64_t)1 << r) < x) ++r;
+  return r;
+}
+
+// fill the plan (sizes and offsets) of a validated configuration
+lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
+  if (!cfg || !info) return fail(LH_ERR_INVALID_ARG, "lh_plan: NULL argument");
+  memset(info, 0, sizeof(*info));
+  const int64_t B = cfg->B, H = cfg->H, N = cfg->N;
+  const int d = cfg->d, L = cfg->L, p = cfg->p, k = cfg->k;
+  const int chunk = cfg->chunk == 0 ? 2048 : cfg->chunk;
+  if (B < 1 || H < 1 || N < 1 || L < 1 || p < 1 || k < 1 || chunk < 1)
+    return fail(LH_ERR_INVALID_ARG, "lh_plan: sizes must be positive");
+  if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return fail(LH_ERR_INVALID_ARG, "lh_plan: bad dtype");
+  if (cfg->scorer < LH_SCORE_QK_SUM || cfg->scorer > LH_SCORE_Q) return fail(LH_ERR_INVALID_ARG, "lh_plan: bad scorer");
+  if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_plan: d must be 64 or 128");
+  if (p < 2 || (p & (p - 1)) != 0) return fail(LH_ERR_UNSUPPORTED, "lh_plan: p must be a power of two >= 2");
+  if (L > 8) return fail(LH_ERR_UNSUPPORTED, "lh_plan: L must be <= 8");
+  if (chunk > 4096) return fail(LH_ERR_UNSUPPORTED, "lh_plan: chunk must be <= 4096");
+  if (N >= ((int64_t)1 << 28)) return fail(LH_ERR_UNSUPPORTED, "lh_plan: N must be < 2^28");
+  if (B * H > (int64_t)65535 * 65535 || H > 65535) return fail(LH_ERR_UNSUPPORTED, "lh_plan: too many heads");
+  const int log2p = ilog2(p);
+  if ((int64_t)(L - 1) * log2p >= 28) return fail(LH_ERR_UNSUPPORTED, "lh_plan: p^(L-1) too large");
+  const int64_t ptop = (int64_t)1 << ((L - 1) * log2p);
+  if (N % ptop != 0) return fail(LH_ERR_UNSUPPORTED, "lh_plan: N must be divisible by p^(L-1)");
+
+  const int64_t BH = B * H;
+  int64_t pyr = 0, upper = 0, selsum = 0;
+  for (int l = 0; l < L; ++l) {
+    info->level_len[l] = N >> (l * log2p);
+    info->level_off[l] = pyr;
+    pyr += info->level_len[l];
+    if (l >= 1) {
+      info->upper_off[l] = upper;
+      upper += info->level_len[l];
+    }
+  }
+  int64_t S = info->level_len[L - 1];
+  for (int l = 0; l + 1 < L; ++l) {
+    const int64_t M = info->level_len[l + 1];
+    info->kprime[l] = (int32_t)(k < M ? k : M);
+    info->sel_off[l] = selsum;
+    selsum += info->kprime[l];
+    S += (int64_t)p * info->kprime[l];
+  }
+  if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_plan: S too large");
+  info->S = S;
+  info->pyr_entries = pyr;
+  info->upper_entries = upper;
+  info->sel_per_head = selsum;
+
+  const size_t e = cfg->dtype == LH_BF16 ? 2 : 4;
+  info->pyr_bytes = (size_t)BH * upper * d * e;
+  info->norms_bytes = (size_t)2 * BH * N * 4;
+  info->topk_ws_bytes = LH_ERR_WORD_BYTES + align_up((size_t)BH * upper * 4);
+  info->sel_bytes = (size_t)BH * selsum * 4;
+  info->seq_bytes = (size_t)BH * S * d * 2;
+  info->seq_map_bytes = (size_t)BH * S * 4;
+  info->slot_of_bytes = (size_t)BH * pyr * 4;
+  info->lse_bytes = (size_t)BH * S * 4;
+  info->grad_seq_bytes = (size_t)BH * S * d * 4;
+  info->attn_bwd_ws_bytes = LH_ERR_WORD_BYTES;
+
+  size_t off = 0;
+  auto take = [&](size_t n) { const size_t o = off; off = align_up(off + n); return o; };
+  info->ctx_off_sel = take(info->sel_bytes > 0 ? info->sel_bytes : 4);
+  info->ctx_off_seq_map = take(info->seq_map_bytes);
+  info->ctx_off_slot_of = take(info->slot_of_bytes);
+  info->ctx_off_qs = take(info->seq_bytes);
+  info->ctx_off_ks = take(info->seq_bytes);
+  info->ctx_off_vs = take(info->seq_bytes);
+  info->ctx_off_os = take(info->seq_bytes);
+  info->ctx_off_lse = take(info->lse_bytes);
+  info->ctx_bytes = off;
+
+  // forward scratch
+  off = LH_ERR_WORD_BYTES;
+  info->ws_off_pyr_q = take(info->pyr_bytes);
+  info->ws_off_pyr_k = take(info->pyr_bytes);
+  info->ws_off_pyr_v = take(info->pyr_bytes);
+  info->ws_off_norms = take(info->norms_bytes);
+  info->ws_off_topk = take(info->topk_ws_bytes);
+  const size_t fwd = off;
+  // backward scratch (overlaps the forward's)
+  off = LH_ERR_WORD_BYTES;
+  info->ws_off_dos = take(info->seq_bytes);
+  info->ws_off_delta = take(info->lse_bytes);
+  info->ws_off_dqs = take(info->grad_seq_bytes);
+  info->ws_off_dks = take(info->grad_seq_bytes);
+  info->ws_off_dvs = take(info->grad_seq_bytes);
+  const size_t bwd = off;
+  info->ws_bytes = fwd > bwd ? fwd : bwd;
+
+  if (D) {
+    D->BH = BH; D->N = N; D->S = S;
+    D->d = d; D->L = L; D->p = p; D->log2p = log2p; D->chunk = chunk;
+    D->dtype = cfg->dtype; D->scorer = cfg->scorer;
+    for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+      D->level_len[l] = info->level_len[l];
+      D->level_off[l] = info->level_off[l];
+      D->upper_off[l] = info->upper_off[l];
+      D->kprime[l] = info->kprime[l];
+      D->sel_off[l] = info->sel_off[l];
+    }
+    D->upper_entries = upper;
+    D->pyr_entries = pyr;
+    D->sel_per_head = selsum;
+  }
+  return LH_OK;
+}
+
+#define LH_CHECK_PTR(p)                                                           \
+  do {                                                                            \
+    if (!(p) || !aligned16(p)) return fail(LH_ERR_INVALID_ARG, #p " is NULL or not 16-byte aligned"); \
+  } while (0)
+
+#define LH_CUDA(call, where)                       \
+  do {                                             \
+    const cudaError_t e_ = (call);                 \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+int* err_word(void* ws) { return static_cast<int*>(ws); }
+
+}  // namespace
+}  // namespace lh
+
+using namespace lh;
+
+extern "C" {
+
+lh_status lh_plan(const lh_config* cfg, lh_plan_info* info) { return plan_impl(cfg, info, nullptr); }
+
+lh_status lh_pyramid_pool(const lh_config* cfg, const void* q, const void* k, const void* v, void* pyr_q,
+                          void* pyr_k, void* pyr_v, float* norms, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v); LH_CHECK_PTR(norms);
+  if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); }
+  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, (cudaStream_t)stream), "lh_pyramid_pool");
+  return LH_OK;
+}
+
+lh_status lh_score_topk(const lh_config* cfg, const float* norms, void* ws, int32_t* sel, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  if (D.L == 1) return LH_OK;
+  LH_CHECK_PTR(norms); LH_CHECK_PTR(ws); LH_CHECK_PTR(sel);
+  float* spyr = reinterpret_cast<float*>(static_cast<char*>(ws) + LH_ERR_WORD_BYTES);
+  LH_CUDA(launch_score_topk(D, norms, spyr, sel, err_word(ws), (cudaStream_t)stream), "lh_score_topk");
+  return LH_OK;
+}
+
+lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const void* v, const void* pyr_q,
+                    const void* pyr_k, const void* pyr_v, const int32_t* sel, void* qs, void* ks, void* vs,
+                    int32_t* seq_map, int32_t* slot_of, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v);
+  if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); LH_CHECK_PTR(sel); }
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(slot_of);
+  LH_CUDA(launch_gather(D, q, k, v, pyr_q, pyr_k, pyr_v, sel, qs, ks, vs, seq_map, slot_of, nullptr,
+                        (cudaStream_t)stream),
+          "lh_gather");
+  return LH_OK;
+}
+
+lh_status lh_attn_fwd(const lh_config* cfg, int64_t S, const void* qs, const void* ks, const void* vs, void* os,
+                      float* lse, void* ws, lh_stream_t stream) {
+  if (!cfg) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd: NULL cfg");
+  if (cfg->B < 1 || cfg->H < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd: sizes must be positive");
+  if (cfg->d != 64 && cfg->d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd: d must be 64 or 128");
+  if (cfg->H > 65535 || cfg->B * cfg->H > 65535) return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd: B*H must be <= 65535");
+  if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd: S too large");
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(os); LH_CHECK_PTR(lse); LH_CHECK_PTR(ws);
+  LH_CUDA(launch_attn_fwd(cfg->B * cfg->H, S, cfg->d, qs, ks, vs, os, lse, err_word(ws), (cudaStream_t)stream),
+          "lh_attn_fwd");
+  return LH_OK;
+}
+
+lh_status lh_attn_bwd(const lh_config* cfg, int64_t S, const void* qs, const void* ks, const void* vs,
+                      const float* lse, const void* dos, const float* delta, float* dqs, float* dks, float* dvs,
+                      void* ws, lh_stream_t stream) {
+  if (!cfg) return fail(LH_ERR_INVALID_ARG, "lh_attn_bwd: NULL cfg");
+  if (cfg->B < 1 || cfg->H < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "lh_attn_bwd: sizes must be positive");
+  if (cfg->d != 64 && cfg->d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd: d must be 64 or 128");
+  if (cfg->H > 65535 || cfg->B * cfg->H > 65535) return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd: B*H must be <= 65535");
+  if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd: S too large");
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(lse); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
+  LH_CHECK_PTR(dqs); LH_CHECK_PTR(dks); LH_CHECK_PTR(dvs); LH_CHECK_PTR(ws);
+  const int64_t BH = cfg->B * cfg->H;
+  LH_CUDA(cudaMemsetAsync(dqs, 0, (size_t)BH * S * cfg->d * sizeof(float), (cudaStream_t)stream), "lh_attn_bwd");
+  LH_CUDA(launch_attn_bwd(BH, S, cfg->d, qs, ks, vs, lse, dos, delta, dqs, dks, dvs, err_word(ws),
+                          (cudaStream_t)stream),
+          "lh_attn_bwd");
+  return LH_OK;
+}
+
+lh_status lh_scatter_back(const lh_config* cfg, const void* os, const int32_t* slot_of, void* y,
+                          lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(os); LH_CHECK_PTR(slot_of); LH_CHECK_PTR(y);
+  LH_CUDA(launch_scatter_back(D, os, slot_of, y, (cudaStream_t)stream), "lh_scatter_back");
+  return LH_OK;
+}
+
+lh_status lh_scatter_back_adjoint(const lh_config* cfg, const void* dy, const int32_t* seq_map, const void* os,
+                                  void* dos, float* delta, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(dy); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(os); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
+  LH_CUDA(launch_scatter_adjoint(D, dy, seq_map, os, dos, delta, nullptr, (cudaStream_t)stream),
+          "lh_scatter_back_adjoint");
+  return LH_OK;
+}
+
+lh_status lh_pool_adjoint(const lh_config* cfg, const float* dqs, const float* dks, const float* dvs,
+                          const int32_t* slot_of, void* dq, void* dk, void* dv, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(dqs); LH_CHECK_PTR(dks); LH_CHECK_PTR(dvs); LH_CHECK_PTR(slot_of);
+  LH_CHECK_PTR(dq); LH_CHECK_PTR(dk); LH_CHECK_PTR(dv);
+  LH_CUDA(launch_pool_adjoint(D, dqs, dks, dvs, slot_of, dq, dk, dv, (cudaStream_t)stream), "lh_pool_adjoint");
+  return LH_OK;
+}
+
+lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const void* v, void* y, void* ctx,
+                     size_t ctx_bytes, void* ws, size_t ws_bytes, lh_stream_t stream) {
+  lh_plan_info I;
+  Dims D;
+  lh_status s = plan_impl(cfg, &I, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v); LH_CHECK_PTR(y); LH_CHECK_PTR(ctx); LH_CHECK_PTR(ws);
+  if (ctx_bytes < I.ctx_bytes || ws_bytes < I.ws_bytes) return fail(LH_ERR_WORKSPACE, "lh_forward: ctx or ws too small");
+  const cudaStream_t st = (cudaStream_t)stream;
+  char* c = static_cast<char*>(ctx);
+  char* w = static_cast<char*>(ws);
+  int* errw = err_word(ws);
+  LH_CUDA(cudaMemsetAsync(errw, 0, sizeof(int), st), "lh_forward");
+  void* pq = w + I.ws_off_pyr_q;
+  void* pk = w + I.ws_off_pyr_k;
+  void* pv = w + I.ws_off_pyr_v;
+  float* norms = reinterpret_cast<float*>(w + I.ws_off_norms);
+  float* spyr = reinterpret_cast<float*>(w + I.ws_off_topk + LH_ERR_WORD_BYTES);
+  int32_t* sel = reinterpret_cast<int32_t*>(c + I.ctx_off_sel);
+  int32_t* seq_map = reinterpret_cast<int32_t*>(c + I.ctx_off_seq_map);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(c + I.ctx_off_slot_of);
+  void* qs = c + I.ctx_off_qs;
+  void* ks = c + I.ctx_off_ks;
+  void* vs = c + I.ctx_off_vs;
+  void* os = c + I.ctx_off_os;
+  float* lse = reinterpret_cast<float*>(c + I.ctx_off_lse);
+  LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st), "lh_forward: pool");
+  LH_CUDA(launch_score_topk(D, norms, spyr, sel, errw, st), "lh_forward: score_topk");
+  LH_CUDA(launch_gather(D, q, k, v, pq, pk, pv, sel, qs, ks, vs, seq_map, slot_of, errw, st), "lh_forward: gather");
+  LH_CUDA(launch_attn_fwd(D.BH, D.S, D.d, qs, ks, vs, os, lse, errw, st), "lh_forward: attn_fwd");
+  LH_CUDA(launch_scatter_back(D, os, slot_of, y, st), "lh_forward: scatter_back");
+  return LH_OK;
+}
+
+lh_status lh_backward(const lh_config* cfg, const void* dy, const void* ctx, size_t ctx_bytes, void* dq,
+                      void* dk, void* dv, void* ws, size_t ws_bytes, lh_stream_t stream) {
+  lh_plan_info I;
+  Dims D;
+  lh_status s = plan_impl(cfg, &I, &D);
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(dy); LH_CHECK_PTR(ctx); LH_CHECK_PTR(dq); LH_CHECK_PTR(dk); LH_CHECK_PTR(dv); LH_CHECK_PTR(ws);
+  if (ctx_bytes < I.ctx_bytes || ws_bytes < I.ws_bytes) return fail(LH_ERR_WORKSPACE, "lh_backward: ctx or ws too small");
+  const cudaStream_t st = (cudaStream_t)stream;
+  const char* c = static_cast<const char*>(ctx);
+  char* w = static_cast<char*>(ws);
+  int* errw = err_word(ws);
+  LH_CUDA(cudaMemsetAsync(errw, 0, sizeof(int), st), "lh_backward");
+  const int32_t* seq_map = reinterpret_cast<const int32_t*>(c + I.ctx_off_seq_map);
+  const int32_t* slot_of = reinterpret_cast<const int32_t*>(c + I.ctx_off_slot_of);
+  const void* qs = c + I.ctx_off_qs;
+  const void* ks = c + I.ctx_off_ks;
+  const void* vs = c + I.ctx_off_vs;
+  const void* os = c + I.ctx_off_os;
+  const float* lse = reinterpret_cast<const float*>(c + I.ctx_off_lse);
+  void* dos = w + I.ws_off_dos;
+  float* delta = reinterpret_cast<float*>(w + I.ws_off_delta);
+  float* dqs = reinterpret_cast<float*>(w + I.ws_off_dqs);
+  float* dks = reinterpret_cast<float*>(w + I.ws_off_dks);
+  float* dvs = reinterpret_cast<float*>(w + I.ws_off_dvs);
+  LH_CUDA(launch_scatter_adjoint(D, dy, seq_map, os, dos, delta, errw, st), "lh_backward: scatter_adjoint");
+  LH_CUDA(cudaMemsetAsync(dqs, 0, I.grad_seq_bytes, st), "lh_backward");
+  LH_CUDA(launch_attn_bwd(D.BH, D.S, D.d, qs, ks, vs, lse, dos, delta, dqs, dks, dvs, errw, st),
+          "lh_backward: attn_bwd");
+  LH_CUDA(launch_pool_adjoint(D, dqs, dks, dvs, slot_of, dq, dk, dv, st), "lh_backward: pool_adjoint");
+  return LH_OK;
+}
+
+lh_status lh_check_error(void* ws, lh_stream_t stream) {
+  if (!ws) return fail(LH_ERR_INVALID_ARG, "lh_check_error: NULL ws");
+  const cudaStream_t st = (cudaStream_t)stream;
+  LH_CUDA(cudaStreamSynchronize(st), "lh_check_error");
+  int word = 0;
+  LH_CUDA(cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost), "lh_check_error");
+  LH_CUDA(cudaMemset(ws, 0, sizeof(int)), "lh_check_error");
+  if (word & ERRW_TIMEOUT) return fail(LH_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (word & ERRW_BOUNDS) return fail(LH_ERR_DEVICE, "a device-side index check failed");
+  return LH_OK;
+}
+
+lh_status lh_clear_error(void* ws, lh_stream_t stream) {
+  if (!ws) return fail(LH_ERR_INVALID_ARG, "lh_clear_error: NULL ws");
+  LH_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream), "lh_clear_error");
+  return LH_OK;
+}
+
+const char* lh_status_string(lh_status status) {
+  switch (status) {
+    case LH_OK: return "ok";
+    case LH_ERR_INVALID_ARG: return "invalid argument";
+    case LH_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LH_ERR_WORKSPACE: return "workspace too small";
+    case LH_ERR_CUDA: return "CUDA error";
+    case LH_ERR_TIMEOUT: return "device wait timed out";
+    case LH_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* lh_last_error_message(void) { return g_msg; }
+
+}  // extern "C"

@@ -1,0 +1,126 @@
+// Shared device helpers and internal launch declarations of liblh.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "lh.h"
+
+namespace lh {
+
+// ---------------------------------------------------------------------------
+// derived shape of one call, computed on the host from lh_config + lh_plan
+// ---------------------------------------------------------------------------
+struct Dims {
+  int64_t BH, N, S;
+  int d, L, p, log2p, chunk;
+  int dtype;   // LH_BF16 / LH_FP32
+  int scorer;  // lh_scorer
+  int64_t level_len[LH_MAX_LEVELS];
+  int64_t level_off[LH_MAX_LEVELS];  // into slot_of rows
+  int64_t upper_off[LH_MAX_LEVELS];  // into pyramid rows (levels >= 1)
+  int64_t upper_entries, pyr_entries;
+  int32_t kprime[LH_MAX_LEVELS];
+  int64_t sel_off[LH_MAX_LEVELS];
+  int64_t sel_per_head;
+};
+
+// error word bits (first int32 of ws)
+enum : int { ERRW_TIMEOUT = 1, ERRW_BOUNDS = 2 };
+
+__device__ __forceinline__ void report_error(int* errw, int bits) {
+  if (errw) atomicOr(errw, bits);
+}
+
+// ---------------------------------------------------------------------------
+// element conversion
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// raw vector of B bytes (4, 8 or 16)
+template <int B> struct RawVec;
+template <> struct RawVec<4> { using type = uint32_t; };
+template <> struct RawVec<8> { using type = uint2; };
+template <> struct RawVec<16> { using type = uint4; };
+
+// load VE elements (VE * sizeof(T) bytes, naturally aligned) as floats
+template <typename T, int VE>
+__device__ __forceinline__ void load_vec(const T* src, float (&x)[VE]) {
+  using V = typename RawVec<sizeof(T) * VE>::type;
+  V u = __ldg(reinterpret_cast<const V*>(src));
+  const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+  for (int i = 0; i < VE; ++i) x[i] = Elem<T>::to_f(e[i]);
+}
+
+// same, through L1/L2 with the default cache policy (data written earlier in the stream)
+template <typename T, int VE>
+__device__ __forceinline__ void load_vec_rw(const T* src, float (&x)[VE]) {
+  using V = typename RawVec<sizeof(T) * VE>::type;
+  V u = *reinterpret_cast<const V*>(src);
+  const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+  for (int i = 0; i < VE; ++i) x[i] = Elem<T>::to_f(e[i]);
+}
+
+template <typename T, int VE>
+__device__ __forceinline__ void store_vec(T* dst, const float (&x)[VE]) {
+  using V = typename RawVec<sizeof(T) * VE>::type;
+  V u;
+  T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+  for (int i = 0; i < VE; ++i) e[i] = Elem<T>::from_f(x[i]);
+  *reinterpret_cast<V*>(dst) = u;
+}
+
+// fp32 vector of VE floats (VE in {2, 4, 8}) from 16-byte-aligned-or-smaller chunks
+template <int VE>
+__device__ __forceinline__ void load_f32(const float* src, float (&x)[VE]) {
+  if constexpr (VE == 8) {
+    float4 a = *reinterpret_cast<const float4*>(src);
+    float4 b = *reinterpret_cast<const float4*>(src + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else if constexpr (VE == 4) {
+    float4 a = *reinterpret_cast<const float4*>(src);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else {
+    static_assert(VE == 2, "2, 4 or 8 floats");
+    float2 a = *reinterpret_cast<const float2*>(src);
+    x[0] = a.x; x[1] = a.y;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers (host side, one per stage); all return cudaGetLastError()
+// ---------------------------------------------------------------------------
+cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void* v, void* pq, void* pk, void* pv,
+                        float* norms, cudaStream_t st);
+cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, int32_t* sel, int* errw,
+                              cudaStream_t st);
+cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
+                          const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st);
+cudaError_t launch_scatter_back(const Dims& D, const void* os, const int32_t* slot_of, void* y, cudaStream_t st);
+cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const void* os,
+                                   void* dos, float* delta, int* errw, cudaStream_t st);
+cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dks, const float* dvs,
+                                const int32_t* slot_of, void* dq, void* dk, void* dv, cudaStream_t st);
+cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, void* os,
+                            float* lse, int* errw, cudaStream_t st);
+cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
+                            const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
+                            float* dvs, int* errw, cudaStream_t st);
+
+// message of the last failure on this thread (set by the API layer)
+void set_error_message(const char* fmt, ...);
+
+}  // namespace lh

@@ -1,0 +1,359 @@
+// Stage 3 (gather into the causally ordered sequence), stage 5 (scatter-back)
+// and the scatter-back adjoint.
+//
+// Kept triples are sorted into causal order and form one contiguous sequence
+// of length S (techllm post "Lighthouse Attention: long-context pretraining",
+// How it works (3)).  Each output returns to its shifted range R(l,i) over the
+// original positions and every position sums what it receives (aitrends.kr
+// summary, Technical details (4); techllm post, How it works (4)).
+//
+// Entry (l, i) covers tokens [i p^l, (i+1) p^l); its key is
+// (e = (i+1) p^l - 1, -l) and its range is R(l,i) = [e, e + p^l).  The slot of
+// an entry is the number of kept entries with a smaller key, counted level by
+// level with binary searches over the sorted parent lists, so no sort runs.
+#include "lh_common.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr unsigned kFull = 0xffffffffu;
+
+struct GatherArgs {
+  const void* x0[3];   // q, k, v (level 0)
+  const void* pyr[3];  // pyramid levels >= 1
+  const int32_t* sel;
+  __nv_bfloat16* out[3];
+  int32_t* seq_map;
+  int32_t* slot_of;
+  int* errw;
+  int64_t BH, N, S, upper_entries, pyr_entries, sel_per_head;
+  int64_t level_len[LH_MAX_LEVELS];
+  int64_t level_off[LH_MAX_LEVELS];
+  int64_t upper_off[LH_MAX_LEVELS];
+  int64_t sel_off[LH_MAX_LEVELS];
+  int64_t cnt_off[LH_MAX_LEVELS + 1];  // first sequence entry id of each level's kept list
+  int32_t kprime[LH_MAX_LEVELS];
+  int L, log2p;
+};
+
+// kept entries of level lv with index < X
+__device__ __forceinline__ int64_t kept_below(const GatherArgs& a, const int32_t* sel_h, int lv, int64_t X) {
+  if (X <= 0) return 0;
+  if (lv == a.L - 1) return min(X, a.level_len[lv]);
+  const int32_t* s = sel_h + a.sel_off[lv];
+  const int n = a.kprime[lv];
+  const int64_t m = X >> a.log2p, r = X & ((1 << a.log2p) - 1);
+  int lo = 0, hi = n;  // lower_bound of m
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)s[mid] < m) lo = mid + 1;
+    else hi = mid;
+  }
+  int64_t cnt = (int64_t)lo << a.log2p;
+  if (r > 0 && lo < n && (int64_t)s[lo] == m) cnt += r;
+  return cnt;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) gather_kernel(GatherArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t bh = wid / a.S;
+  if (bh >= a.BH) return;
+  const int64_t id = wid % a.S;
+  const int32_t* sel_h = a.sel + bh * a.sel_per_head;
+  int l = 0;
+  while (l + 1 < a.L && id >= a.cnt_off[l + 1]) ++l;
+  const int64_t j = id - a.cnt_off[l];
+  int64_t i;
+  if (l < a.L - 1) i = ((int64_t)sel_h[a.sel_off[l] + (j >> a.log2p)] << a.log2p) + (j & ((1 << a.log2p) - 1));
+  else i = j;
+  const int64_t e = ((i + 1) << (l * a.log2p)) - 1;
+  // one level per lane: kept entries whose key is below (e, -l)
+  int64_t part = 0;
+  if (lane < a.L) {
+    const int lv = lane;
+    if (lv == l) part = j;
+    else if (lv > l) part = kept_below(a, sel_h, lv, (e + 1) >> (lv * a.log2p));
+    else part = kept_below(a, sel_h, lv, e >> (lv * a.log2p));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(kFull, part, o);
+  const int64_t slot = part;
+  if (slot < 0 || slot >= a.S || i < 0 || i >= a.level_len[l]) {
+    if (lane == 0) report_error(a.errw, ERRW_BOUNDS);
+    return;
+  }
+  if (lane == 0) {
+    a.seq_map[bh * a.S + slot] = (int32_t)(((int64_t)l << 28) | i);
+    a.slot_of[bh * a.pyr_entries + a.level_off[l] + i] = (int32_t)slot;
+  }
+  // copy the three rows, 8 elements per lane step, converting to bf16
+  constexpr int CH = D / 8;
+  for (int c = lane; c < 3 * CH; c += 32) {
+    const int t = c / CH, off = (c % CH) * 8;
+    const T* src = (l == 0) ? static_cast<const T*>(a.x0[t]) + (bh * a.N + i) * D
+                            : static_cast<const T*>(a.pyr[t]) + (bh * a.upper_entries + a.upper_off[l] + i) * D;
+    __nv_bfloat16* dst = a.out[t] + (bh * a.S + slot) * D + off;
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src + off);
+    } else {
+      float x[8];
+      load_f32<4>(reinterpret_cast<const float*>(src) + off, *reinterpret_cast<float(*)[4]>(x));
+      load_f32<4>(reinterpret_cast<const float*>(src) + off + 4, *reinterpret_cast<float(*)[4]>(x + 4));
+      store_vec<__nv_bfloat16, 8>(dst, x);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// scatter-back: Y_j = sum_l [kept] Os[slot(l, ((j+1) >> l log2p) - 1)]
+// one row per warp instruction; levels >= 1 are cached between their boundaries
+// ---------------------------------------------------------------------------
+struct ScatterArgs {
+  const __nv_bfloat16* os;
+  const int32_t* slot_of;
+  void* y;
+  int64_t BH, N, S, pyr_entries;
+  int64_t level_off[LH_MAX_LEVELS];
+  int64_t tasks_per_head;
+  int task_rows, log2p;
+};
+
+template <typename T, int D, int NL>
+__global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a) {
+  constexpr int VE = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t bh = wid / a.tasks_per_head;
+  if (bh >= a.BH) return;
+  const int64_t row0 = (wid % a.tasks_per_head) * a.task_rows;
+  const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
+  const int log2p = a.log2p;
+  const int32_t* so = a.slot_of + bh * a.pyr_entries;
+  const __nv_bfloat16* os = a.os + bh * a.S * D + lane * VE;
+  T* out = static_cast<T*>(a.y) + (bh * a.N + row0) * D + lane * VE;
+
+  float up[NL + 1][VE];
+  float upper[VE];
+#pragma unroll
+  for (int i = 0; i < VE; ++i) upper[i] = 0.f;
+  int s0w = -1;
+  for (int r = 0; r < rows; ++r) {
+    const int64_t j = row0 + r;
+    if ((r & 31) == 0) s0w = (r + lane < rows) ? so[a.level_off[0] + j + lane] : -1;
+    if constexpr (NL > 1) {
+      if (r == 0 || ((j + 1) & ((1 << log2p) - 1)) == 0) {
+#pragma unroll
+        for (int l = 1; l < NL; ++l) {
+          if (r == 0 || ((j + 1) & ((1ll << (l * log2p)) - 1)) == 0) {
+            const int64_t i = ((j + 1) >> (l * log2p)) - 1;
+            const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
+            if (s >= 0) {
+              load_vec_rw<__nv_bfloat16, VE>(os + (int64_t)s * D, up[l]);
+            } else {
+#pragma unroll
+              for (int c = 0; c < VE; ++c) up[l][c] = 0.f;
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < VE; ++c) {
+          float s = 0.f;
+#pragma unroll
+          for (int l = 1; l < NL; ++l) s += up[l][c];
+          upper[c] = s;
+        }
+      }
+    }
+    const int s0 = __shfl_sync(kFull, s0w, r & 31);
+    float y[VE];
+#pragma unroll
+    for (int c = 0; c < VE; ++c) y[c] = upper[c];
+    if (s0 >= 0) {
+      float v[VE];
+      load_vec_rw<__nv_bfloat16, VE>(os + (int64_t)s0 * D, v);
+#pragma unroll
+      for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
+    }
+    store_vec<T, VE>(out + (int64_t)r * D, y);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// scatter-back adjoint: dOs[s] = sum_{j in R(l,i)} dY_j (fp32), Delta[s] = dOs[s] . Os[s]
+// one warp per slot, R rows per warp instruction
+// ---------------------------------------------------------------------------
+struct ScatterAdjArgs {
+  const void* dy;
+  const int32_t* seq_map;
+  const __nv_bfloat16* os;
+  __nv_bfloat16* dos;
+  float* delta;
+  int* errw;
+  int64_t BH, N, S;
+  int L, log2p;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) scatter_adjoint_kernel(ScatterAdjArgs a) {
+  constexpr int VE = (sizeof(T) == 2 && D == 128) ? 8 : 4;
+  constexpr int LPR = D / VE, R = 32 / LPR;
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int64_t bh = wid / a.S;
+  if (bh >= a.BH) return;
+  const int64_t s = wid % a.S;
+  const int lr = lane / LPR, cv = lane % LPR;
+  const int32_t code = a.seq_map[bh * a.S + s];
+  const int l = code >> 28;
+  const int64_t i = code & ((1 << 28) - 1);
+  if (l >= a.L) {
+    if (lane == 0) report_error(a.errw, ERRW_BOUNDS);
+    return;
+  }
+  const int64_t b = (int64_t)1 << (l * a.log2p);
+  const int64_t r0 = min((i + 1) * b - 1, a.N), r1 = min((i + 2) * b - 1, a.N);
+  const int n = (int)(r1 - r0);
+  const T* src = static_cast<const T*>(a.dy) + (bh * a.N + r0) * D + cv * VE;
+  float acc[VE];
+#pragma unroll
+  for (int c = 0; c < VE; ++c) acc[c] = 0.f;
+  for (int g = 0; g < n; g += R * U) {
+    float x[U][VE];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int row = g + u * R + lr;
+      if (row < n) load_vec<T, VE>(src + (int64_t)row * D, x[u]);
+      else {
+#pragma unroll
+        for (int c = 0; c < VE; ++c) x[u][c] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int c = 0; c < VE; ++c) acc[c] += x[u][c];
+  }
+#pragma unroll
+  for (int c = 0; c < VE; ++c)
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) acc[c] += __shfl_xor_sync(kFull, acc[c], o);
+  // round to bf16 once; Delta from the rounded values and the bf16 Os
+  __nv_bfloat16 h[VE];
+  float o_row[VE];
+  load_vec_rw<__nv_bfloat16, VE>(a.os + (bh * a.S + s) * D + cv * VE, o_row);
+  float dot = 0.f;
+#pragma unroll
+  for (int c = 0; c < VE; ++c) {
+    h[c] = __float2bfloat16_rn(acc[c]);
+    dot = fmaf(__bfloat162float(h[c]), o_row[c], dot);
+  }
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(kFull, dot, o);
+  if (lr == 0) {
+    using V = typename RawVec<2 * VE>::type;
+    *reinterpret_cast<V*>(a.dos + (bh * a.S + s) * D + cv * VE) = *reinterpret_cast<const V*>(h);
+    if (cv == 0) a.delta[bh * a.S + s] = dot;
+  }
+}
+
+template <typename T, int D>
+cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t blocks, cudaStream_t st) {
+  switch (L) {
+#define LH_CASE(n) \
+  case n: scatter_back_kernel<T, D, n><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a); break;
+    LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
+                          const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st) {
+  GatherArgs a{};
+  a.x0[0] = q; a.x0[1] = k; a.x0[2] = v;
+  a.pyr[0] = pq; a.pyr[1] = pk; a.pyr[2] = pv;
+  a.sel = sel;
+  a.out[0] = static_cast<__nv_bfloat16*>(qs);
+  a.out[1] = static_cast<__nv_bfloat16*>(ks);
+  a.out[2] = static_cast<__nv_bfloat16*>(vs);
+  a.seq_map = seq_map;
+  a.slot_of = slot_of;
+  a.errw = errw;
+  a.BH = D.BH; a.N = D.N; a.S = D.S;
+  a.upper_entries = D.upper_entries; a.pyr_entries = D.pyr_entries; a.sel_per_head = D.sel_per_head;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+    a.level_len[l] = D.level_len[l];
+    a.level_off[l] = D.level_off[l];
+    a.upper_off[l] = D.upper_off[l];
+    a.sel_off[l] = D.sel_off[l];
+    a.kprime[l] = D.kprime[l];
+  }
+  a.cnt_off[0] = 0;
+  for (int l = 0; l < D.L - 1; ++l) a.cnt_off[l + 1] = a.cnt_off[l] + ((int64_t)D.kprime[l] << D.log2p);
+  a.L = D.L;
+  a.log2p = D.log2p;
+  cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * D.pyr_entries * sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (D.BH * D.S + kWarps - 1) / kWarps;
+  if (D.dtype == LH_BF16) {
+    if (D.d == 128) gather_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+    else gather_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+  } else {
+    if (D.d == 128) gather_kernel<float, 128><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+    else gather_kernel<float, 64><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_back(const Dims& D, const void* os, const int32_t* slot_of, void* y, cudaStream_t st) {
+  ScatterArgs a{};
+  a.os = static_cast<const __nv_bfloat16*>(os);
+  a.slot_of = slot_of;
+  a.y = y;
+  a.BH = D.BH; a.N = D.N; a.S = D.S; a.pyr_entries = D.pyr_entries;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) a.level_off[l] = D.level_off[l];
+  const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
+  a.task_rows = (int)(ptop > 64 ? ptop : 64);
+  a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
+  a.log2p = D.log2p;
+  const int64_t blocks = (D.BH * a.tasks_per_head + kWarps - 1) / kWarps;
+  if (D.dtype == LH_BF16) {
+    return D.d == 128 ? scatter_dispatch_L<__nv_bfloat16, 128>(D.L, a, blocks, st)
+                      : scatter_dispatch_L<__nv_bfloat16, 64>(D.L, a, blocks, st);
+  }
+  return D.d == 128 ? scatter_dispatch_L<float, 128>(D.L, a, blocks, st)
+                    : scatter_dispatch_L<float, 64>(D.L, a, blocks, st);
+}
+
+cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const void* os,
+                                   void* dos, float* delta, int* errw, cudaStream_t st) {
+  ScatterAdjArgs a{};
+  a.dy = dy;
+  a.seq_map = seq_map;
+  a.os = static_cast<const __nv_bfloat16*>(os);
+  a.dos = static_cast<__nv_bfloat16*>(dos);
+  a.delta = delta;
+  a.errw = errw;
+  a.BH = D.BH; a.N = D.N; a.S = D.S;
+  a.L = D.L;
+  a.log2p = D.log2p;
+  const int64_t blocks = (D.BH * D.S + kWarps - 1) / kWarps;
+  if (D.dtype == LH_BF16) {
+    if (D.d == 128) scatter_adjoint_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+    else scatter_adjoint_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+  } else {
+    if (D.d == 128) scatter_adjoint_kernel<float, 128><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+    else scatter_adjoint_kernel<float, 64><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lh

@@ -1,0 +1,228 @@
+/*
+ * lh.h - C ABI of liblh, one Lighthouse attention layer (forward and backward)
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * Lighthouse Attention (arXiv:2605.06554) wraps an unmodified causal attention
+ * in four stages.  Citations below name the two pages that describe it:
+ *   LH-summary: the aitrends.kr summary of Lighthouse Attention
+ *               ("Method", "Technical details" (1)-(4)).
+ *   LH-post:    the techllm.github.io post "Lighthouse Attention: long-context
+ *               pretraining" ("How it works" (1)-(4), "Key formulas").
+ *
+ * Conventions shared by every call
+ *  - Ownership: the caller allocates and frees every buffer.  liblh never
+ *    allocates device memory, never frees, and never synchronises a stream,
+ *    except lh_check_error.  All calls are asynchronous on `stream`.
+ *  - Pointers are device pointers (cudaMalloc / torch CUDA tensors) unless a
+ *    parameter says "host", and must be 16-byte aligned.
+ *  - Layouts are dense row-major.  "BH" = B*H flattened; Q, K, V, Y, dY, dQ,
+ *    dK, dV are [B][H][N][d] in cfg->dtype.  The gathered sequence tensors
+ *    Qs, Ks, Vs, Os, dOs are [BH][S][d] bf16; LSE and Delta are [BH][S] fp32;
+ *    dQs, dKs, dVs are [BH][S][d] fp32.
+ *  - Support: d in {64, 128}; p a power of two >= 2; 1 <= L <= 16;
+ *    N divisible by p^(L-1); N < 2^28; k >= 1; B*H <= 65535 * 65535.
+ *    dtype LH_FP32 pools and scores in fp32 and casts the gathered sequence
+ *    to bf16 for the tensor cores.
+ *  - Errors: argument checks run on the host and return a status at once
+ *    (no work is queued).  A failed launch returns LH_ERR_CUDA; details are
+ *    in lh_last_error_message().  Device-side problems (a bounded wait that
+ *    ran out, an index out of range) set the error word held in the first
+ *    LH_ERR_WORD_BYTES bytes of `ws`; lh_check_error reports and clears it.
+ *  - Re-entrancy: no global state except the per-thread error message; calls
+ *    on different streams are independent when each has its own ws and ctx.
+ */
+#ifndef LH_H
+#define LH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* a cudaStream_t; NULL is the legacy default stream */
+typedef struct CUstream_st *lh_stream_t;
+
+typedef enum {
+  LH_OK = 0,
+  LH_ERR_INVALID_ARG = 1,  /* NULL or misaligned pointer, negative size, bad enum */
+  LH_ERR_UNSUPPORTED = 2,  /* valid but outside the support list above */
+  LH_ERR_WORKSPACE = 3,    /* ctx_bytes or ws_bytes smaller than lh_plan asks */
+  LH_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  LH_ERR_TIMEOUT = 5,      /* a bounded device wait ran out (from lh_check_error) */
+  LH_ERR_DEVICE = 6        /* a device-side index check failed (from lh_check_error) */
+} lh_status;
+
+typedef enum { LH_BF16 = 0, LH_FP32 = 1 } lh_dtype;
+
+/* Level-0 score s0_t from the l2 norms of Q_t and K_t (LH-summary
+ * "Technical details" (2): ||Q_i||_2, ||K_i||_2 are the scores at level 0). */
+typedef enum {
+  LH_SCORE_QK_SUM = 0, /* ||Q_t|| + ||K_t|| */
+  LH_SCORE_K = 1,      /* ||K_t||  (the "projection-norm" scorer) */
+  LH_SCORE_Q = 2       /* ||Q_t|| */
+} lh_scorer;
+
+typedef struct {
+  int64_t B, H, N; /* batch, heads, sequence length */
+  int32_t d;       /* head dimension */
+  int32_t L;       /* pyramid levels */
+  int32_t p;       /* pooling factor */
+  int32_t k;       /* selection budget per level */
+  int32_t chunk;   /* top-k stratification chunk T (candidates); 0 = 2048 */
+  int32_t dtype;   /* lh_dtype of Q, K, V, Y, dY, dQ, dK, dV */
+  int32_t scorer;  /* lh_scorer */
+} lh_config;
+
+#define LH_MAX_LEVELS 16
+#define LH_ERR_WORD_BYTES 256
+
+/* Everything a caller needs to size and view the buffers.  Offsets are in
+ * bytes from the start of ctx or ws and are 256-byte aligned. */
+typedef struct {
+  int64_t S;                          /* gathered length N/p^(L-1) + sum_l p*kprime[l] */
+  int64_t pyr_entries;                /* sum over l of N/p^l */
+  int64_t level_len[LH_MAX_LEVELS];   /* N/p^l */
+  int64_t level_off[LH_MAX_LEVELS];   /* first row of level l in slot_of */
+  int64_t upper_off[LH_MAX_LEVELS];   /* first row of level l>=1 in the pyramid buffers */
+  int64_t upper_entries;              /* sum over l>=1 of N/p^l */
+  int32_t kprime[LH_MAX_LEVELS];      /* min(k, N/p^(l+1)) for l < L-1 */
+  int64_t sel_off[LH_MAX_LEVELS];     /* first entry of level l in sel */
+  int64_t sel_per_head;               /* sum of kprime */
+  /* stage-call buffer sizes (whole B*H) */
+  size_t pyr_bytes;     /* one of pyr_q/pyr_k/pyr_v: [BH][upper_entries][d] in dtype */
+  size_t norms_bytes;   /* [2][BH][N] fp32 */
+  size_t topk_ws_bytes; /* ws of lh_score_topk */
+  size_t sel_bytes;     /* [BH][sel_per_head] int32 */
+  size_t seq_bytes;     /* one of qs/ks/vs/os: [BH][S][d] bf16 */
+  size_t seq_map_bytes; /* [BH][S] int32 */
+  size_t slot_of_bytes; /* [BH][pyr_entries] int32 */
+  size_t lse_bytes;     /* [BH][S] fp32 (also Delta) */
+  size_t grad_seq_bytes;/* one of dqs/dks/dvs: [BH][S][d] fp32 */
+  size_t attn_bwd_ws_bytes;
+  /* lh_forward / lh_backward */
+  size_t ctx_bytes, ws_bytes;
+  size_t ctx_off_sel, ctx_off_seq_map, ctx_off_slot_of, ctx_off_qs, ctx_off_ks, ctx_off_vs, ctx_off_os,
+      ctx_off_lse;
+  size_t ws_off_pyr_q, ws_off_pyr_k, ws_off_pyr_v, ws_off_norms, ws_off_topk;
+  size_t ws_off_dos, ws_off_delta, ws_off_dqs, ws_off_dks, ws_off_dvs;
+} lh_plan_info;
+
+/* Validate cfg and fill *info (host only, no CUDA call).
+ * Cite: LH-post "Key formulas" (S = N/p^(L-1) + (L-1)*p*k; where k exceeds the
+ * M = N/p^(l+1) candidates of a level, kprime = min(k, M) is kept). */
+lh_status lh_plan(const lh_config *cfg, lh_plan_info *info);
+
+/* Stage 1 - symmetric pyramid pooling plus level-0 norms.
+ * Cite: LH-post "How it works" (1) (Q, K, V average-pooled with the same
+ * factor p over L levels); LH-summary "Technical details" (1)-(2).
+ * In:  q, k, v [BH][N][d] dtype.
+ * Out: pyr_q, pyr_k, pyr_v [BH][upper_entries][d] dtype: level l >= 1 starts
+ *      at row upper_off[l]; entry i is the mean of tokens [i p^l, (i+1) p^l),
+ *      summed in fp32 and rounded once.
+ *      norms [2][BH][N] fp32: plane 0 = ||Q_t||_2, plane 1 = ||K_t||_2.
+ * With L = 1 the pyramid buffers are not touched (may be NULL). */
+lh_status lh_pyramid_pool(const lh_config *cfg, const void *q, const void *k, const void *v, void *pyr_q,
+                          void *pyr_k, void *pyr_v, float *norms, lh_stream_t stream);
+
+/* Stage 2 - max-pooled scores and stratified chunked top-k.
+ * Cite: LH-summary "Technical details" (2) (coarser levels take max-pooled
+ * scores; top-K yields the index set I); LH-post "Limitations" (the top-K is
+ * stratified: every interval contributes a fixed number).
+ * In:  norms from lh_pyramid_pool; ws of topk_ws_bytes (score pyramid scratch,
+ *      preceded by the error word).
+ * Out: sel [BH][sel_per_head] int32: for level l < L-1, at sel_off[l],
+ *      kprime[l] parent indices at level l+1 in ascending order.  The M
+ *      candidates of a level are split into C = max(1, M / chunk) contiguous
+ *      chunks (the first M mod C one longer); chunk c keeps its
+ *      floor(k'/C) + [c < k' mod C] highest fp32 scores, ties to the lower index. */
+lh_status lh_score_topk(const lh_config *cfg, const float *norms, void *ws, int32_t *sel, lh_stream_t stream);
+
+/* Stage 3 - gather the kept entries into one causally ordered sequence.
+ * Cite: LH-post "How it works" (3) (kept entries sorted into causal order
+ * form a contiguous sequence of length S); LH-summary "Technical details" (3).
+ * Kept entries: the p children (l, m*p + c) of every parent m in sel level l,
+ * and every entry of the top level L-1.  Entry (l, i) has key
+ * (e = (i+1) p^l - 1, -l); slots are the ranks of the keys.
+ * In:  q, k, v (level 0) and pyr_q/k/v (levels >= 1), sel.
+ * Out: qs, ks, vs [BH][S][d] bf16; seq_map [BH][S] int32 = (l << 28) | i;
+ *      slot_of [BH][pyr_entries] int32 = slot of (l, i) at level_off[l] + i,
+ *      -1 if not kept. */
+lh_status lh_gather(const lh_config *cfg, const void *q, const void *k, const void *v, const void *pyr_q,
+                    const void *pyr_k, const void *pyr_v, const int32_t *sel, void *qs, void *ks, void *vs,
+                    int32_t *seq_map, int32_t *slot_of, lh_stream_t stream);
+
+/* Stage 4 - dense causal attention over the S-token sequence (tcgen05).
+ * Cite: LH-summary "Technical details" (3) (stock attention over the gathered
+ * S tokens); LH-post "How it works" (3).  Softmax scale 1/sqrt(d); slot t
+ * attends to slots u <= t.  Uses cfg->B, H, d only; S is any length >= 1.
+ * Out: os [BH][S][d] bf16; lse [BH][S] fp32, natural log of the row's sum of
+ *      exp(scaled logits).  ws: at least LH_ERR_WORD_BYTES (error word). */
+lh_status lh_attn_fwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs, void *os,
+                      float *lse, void *ws, lh_stream_t stream);
+
+/* Stage 4 backward.  Cite: LH-summary "Method" step 5 (the gradient flows
+ * back through the attention kernel).
+ * In:  qs, ks, vs, lse from the forward; dos [BH][S][d] bf16 and
+ *      delta [BH][S] fp32 (rowsum(dOs * Os)) from lh_scatter_back_adjoint.
+ * Out: dqs, dks, dvs [BH][S][d] fp32 (dqs is zeroed and accumulated here).
+ * ws: at least attn_bwd_ws_bytes (error word). */
+lh_status lh_attn_bwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs,
+                      const float *lse, const void *dos, const float *delta, float *dqs, float *dks, float *dvs,
+                      void *ws, lh_stream_t stream);
+
+/* Stage 5 - scatter-back.  Cite: LH-summary "Technical details" (4) (outputs
+ * return to the N positions and each position j sums over the ranges
+ * R(l, i)); LH-post "How it works" (4) (shifted ranges keep causality).
+ * Y_j = sum over l of Os[slot(l, floor((j+1)/p^l) - 1)] for kept entries,
+ * summed in fp32 from l = 0 up and rounded once; R(l, i) =
+ * [(i+1) p^l - 1, (i+2) p^l - 1).  Positions with no contributor get 0.
+ * Out: y [BH][N][d] dtype. */
+lh_status lh_scatter_back(const lh_config *cfg, const void *os, const int32_t *slot_of, void *y,
+                          lh_stream_t stream);
+
+/* Stage 5 backward: dOs[slot(l,i)] = sum of dY_j over j in R(l, i) (fp32,
+ * rounded once to bf16), and delta[s] = sum_c dOs[s,c] * Os[s,c] (fp32, from
+ * the bf16 values).  Cite: LH-summary "Method" step 5.
+ * Out: dos [BH][S][d] bf16, delta [BH][S] fp32. */
+lh_status lh_scatter_back_adjoint(const lh_config *cfg, const void *dy, const int32_t *seq_map, const void *os,
+                                  void *dos, float *delta, lh_stream_t stream);
+
+/* Stages 3 and 1 backward: dX_t = sum over l of p^-l * dXs[slot(l, floor(t/p^l))]
+ * for kept entries (fp32, rounded once), X in {Q, K, V}.  No gradient flows
+ * through the scores: the top-k is not differentiable (LH-post "How it
+ * works" (2)).  In: dqs, dks, dvs fp32.  Out: dq, dk, dv [BH][N][d] dtype. */
+lh_status lh_pool_adjoint(const lh_config *cfg, const float *dqs, const float *dks, const float *dvs,
+                          const int32_t *slot_of, void *dq, void *dk, void *dv, lh_stream_t stream);
+
+/* Whole forward: stages 1-5.  ctx (ctx_bytes) receives what the backward
+ * needs (sel, seq_map, slot_of, Qs, Ks, Vs, Os, LSE at the ctx_off_* offsets)
+ * and must live until lh_backward.  ws (ws_bytes) is scratch; its error word
+ * is cleared at entry. */
+lh_status lh_forward(const lh_config *cfg, const void *q, const void *k, const void *v, void *y, void *ctx,
+                     size_t ctx_bytes, void *ws, size_t ws_bytes, lh_stream_t stream);
+
+/* Whole backward: stage 5 adjoint, attention backward, pool/gather adjoint.
+ * ctx is read only.  ws (ws_bytes) is scratch; its error word is cleared at entry. */
+lh_status lh_backward(const lh_config *cfg, const void *dy, const void *ctx, size_t ctx_bytes, void *dq,
+                      void *dk, void *dv, void *ws, size_t ws_bytes, lh_stream_t stream);
+
+/* Synchronise `stream`, read the error word at the start of ws, clear it and
+ * return LH_OK, LH_ERR_TIMEOUT or LH_ERR_DEVICE (or LH_ERR_CUDA). */
+lh_status lh_check_error(void *ws, lh_stream_t stream);
+
+/* Zero the error word at the start of ws (asynchronous). */
+lh_status lh_clear_error(void *ws, lh_stream_t stream);
+
+/* Static text of a status. */
+const char *lh_status_string(lh_status status);
+
+/* Text of the last failure on the calling thread ("" if none). */
+const char *lh_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LH_H */

@@ -42,6 +42,11 @@ Readings of points the pages leave open (each one is listed in the design doc):
   R7  entry (l,i) returns its output to R(l,i) = [(i+1)p^l - 1, (i+2)p^l - 1)
       clipped to [0, N); every position sums what it receives.
   R9  selection is per (batch, head).
+  R11 the pages run the gathered sequence through stock FlashAttention, a
+      16-bit kernel (LH-summary Technical details (3); LH-post How it works
+      (3)), so the attention inputs Qs, Ks, Vs are rounded to bf16 (round to
+      nearest even) before the attention; the backward passes gradients
+      through that cast unchanged.  attn_dtype=None keeps them exact.
 
 All arrays are float64 numpy arrays; one head at a time is ``[N, d]``.
 """
@@ -221,6 +226,15 @@ def gather(levels, seq_level, seq_index) -> np.ndarray:
 # 5. dense causal softmax attention on the sequence (LH-summary Technical details (3))
 # ----------------------------------------------------------------------------
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest bf16 value (8 significant bits), ties to even,
+    straight from float64 (reading R11).  Exact for the normal bf16 range
+    (|x| >= 2^-126); the layer's values never come near it."""
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
 ROW_BLOCK = 512  # rows are independent; blocks only bound memory
 
 
@@ -272,10 +286,12 @@ def scatter_back(Os, seq_level, seq_index, N: int, p: int, L: int) -> np.ndarray
 # ----------------------------------------------------------------------------
 
 def forward_head(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum",
-                 sel=None):
+                 sel=None, attn_dtype="bf16"):
     """One head of the layer.  Returns (Y, saved) with everything the backward
     and the parity tests need.  ``sel`` freezes the selection (used by the
-    causality and finite-difference checks); by default it is computed."""
+    causality and finite-difference checks); by default it is computed.
+    ``attn_dtype`` = "bf16" rounds the attention inputs (reading R11); None
+    keeps them exact."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
@@ -287,6 +303,10 @@ def forward_head(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer
         spyr = None
     seq_level, seq_index = causal_order(selected_entries(sel, N, p, L), p)
     Qs, Ks, Vs = gather(pq, seq_level, seq_index), gather(pk, seq_level, seq_index), gather(pv, seq_level, seq_index)
+    if attn_dtype == "bf16":
+        Qs, Ks, Vs = round_bf16(Qs), round_bf16(Ks), round_bf16(Vs)
+    elif attn_dtype is not None:
+        raise ValueError(f"unknown attn_dtype {attn_dtype!r}")
     Os, lse = causal_attention(Qs, Ks, Vs)
     Y = scatter_back(Os, seq_level, seq_index, N, p, L)
     saved = dict(N=N, p=p, L=L, k=k, T=T, scorer=scorer, sel=sel, spyr=spyr,
@@ -371,10 +391,10 @@ def backward_head(dY, saved):
 # several heads: [BH, N, d], selection per head (reading R9)
 # ----------------------------------------------------------------------------
 
-def forward(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum"):
+def forward(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum", attn_dtype="bf16"):
     Ys, saves = [], []
     for h in range(Q.shape[0]):
-        Y, sv = forward_head(Q[h], K[h], V[h], p, L, k, T, scorer)
+        Y, sv = forward_head(Q[h], K[h], V[h], p, L, k, T, scorer, attn_dtype=attn_dtype)
         Ys.append(Y)
         saves.append(sv)
     return np.stack(Ys), saves

@@ -1,0 +1,99 @@
+"""The C ABI: liblh.so loads, exports every symbol include/lh.h declares, and
+its host-only logic (planning, argument checks, failure paths) behaves.
+No GPU is needed: every call here returns before any CUDA work is queued."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from hierarchical_sparse_attention_pyramid_b200 import _lib, plan, Layer
+from hierarchical_sparse_attention_pyramid_b200.synth import WORKLOADS
+from oracle import lighthouse_oracle as lo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lh.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lh_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from hierarchical_sparse_attention_pyramid_b200.build import build
+        build()
+    return _lib.load()
+
+
+def test_header_functions_are_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (lh_[a-z_]+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_plan_matches_oracle_sizes(lib, name):
+    w = WORKLOADS[name]
+    info = plan(Layer.of(w))
+    assert info.S == lo.gathered_length(w.N, w.p, w.L, w.k)
+    assert info.pyr_entries == lo.pyramid_entry_count(w.N, w.p, w.L)
+    assert list(info.kprime)[: w.L - 1] == lo.budgets(w.N, w.p, w.L, w.k)
+    assert info.ctx_bytes > 0 and info.ws_bytes > 0
+    for f in ("ctx_off_sel", "ctx_off_qs", "ctx_off_lse", "ws_off_pyr_q", "ws_off_dqs"):
+        assert getattr(info, f) % 256 == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2),            # unsupported head dim
+    (dict(p=3), 2),             # p not a power of two
+    (dict(N=1000, L=5), 2),     # N not divisible by p^(L-1)
+    (dict(L=9), 2),             # more levels than the kernels take
+    (dict(k=0), 1),             # invalid budget
+    (dict(chunk=8192), 2),      # chunk above the shared-memory bound
+    (dict(dtype=7), 1),         # bad enum
+])
+def test_plan_rejects(lib, kw, status):
+    base = dict(B=1, H=2, N=4096, d=128, L=3, p=2, k=16, chunk=0, dtype=0, scorer=0)
+    base.update(kw)
+    cfg = _lib.LhConfig(**base)
+    info = _lib.LhPlanInfo()
+    assert lib.lh_plan(ctypes.byref(cfg), ctypes.byref(info)) == status
+    assert lib.lh_last_error_message().decode()
+
+
+def test_failure_paths_return_before_any_gpu_work(lib):
+    cfg = _lib.LhConfig(1, 1, 4096, 64, 3, 2, 256, 0, 1, 0)
+    info = _lib.LhPlanInfo()
+    assert lib.lh_plan(ctypes.byref(cfg), ctypes.byref(info)) == 0
+    fake = ctypes.c_void_p(1 << 40)  # never dereferenced: every check below fails first
+    mis = ctypes.c_void_p((1 << 40) + 8)
+    # misaligned pointer
+    assert lib.lh_pyramid_pool(ctypes.byref(cfg), mis, fake, fake, fake, fake, fake, fake, None) == 1
+    # NULL pointer
+    assert lib.lh_scatter_back(ctypes.byref(cfg), None, fake, fake, None) == 1
+    # workspace too small
+    assert lib.lh_forward(ctypes.byref(cfg), fake, fake, fake, fake, fake, info.ctx_bytes - 1, fake,
+                          info.ws_bytes, None) == 3
+    assert lib.lh_backward(ctypes.byref(cfg), fake, fake, info.ctx_bytes, fake, fake, fake, fake,
+                           info.ws_bytes - 1, None) == 3
+    # unsupported head dim in the attention stage
+    bad = _lib.LhConfig(1, 1, 4096, 80, 3, 2, 256, 0, 0, 0)
+    assert lib.lh_attn_fwd(ctypes.byref(bad), 100, fake, fake, fake, fake, fake, fake, None) == 2
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.lh_status_string(s).decode()
+    assert lib.lh_status_string(99).decode() == "unknown status"

@@ -187,9 +187,24 @@ def torch_causal(Qs, Ks, Vs):
 def test_L1_is_dense_causal_attention():
     r = rng(9)
     Q, K, V = (r.standard_normal((300, 16)) for _ in range(3))
-    Y, sv = lo.forward_head(Q, K, V, p=2, L=1, k=5)
+    Y, sv = lo.forward_head(Q, K, V, p=2, L=1, k=5, attn_dtype=None)
     assert len(sv["seq_level"]) == 300
     np.testing.assert_allclose(Y, torch_causal(Q, K, V), rtol=0, atol=1e-12)
+    # with the attention inputs rounded to bf16 (reading R11): torch's own bf16 cast
+    Yb, _ = lo.forward_head(Q, K, V, p=2, L=1, k=5)
+    rq, rk, rv = (torch.from_numpy(x).float().to(torch.bfloat16).double().numpy() for x in (Q, K, V))
+    np.testing.assert_allclose(Yb, torch_causal(rq, rk, rv), rtol=0, atol=1e-12)
+
+
+def test_round_bf16_matches_torch_cast():
+    r = rng(19)
+    x = np.concatenate([r.standard_normal(20000) * 10.0 ** r.integers(-6, 6, 20000),
+                        [0.0, -0.0, 1.0, -3.0, 2.0 ** -100, 65504.0]]).astype(np.float32)
+    # float32 values including exact ties between bf16 neighbours (normal range)
+    ties = (((np.arange(0, 4000, dtype=np.uint32) * 7 % 0x7E00) + 0x0100) << 16 | 0x8000).view(np.float32)
+    x = np.concatenate([x, ties, -ties])
+    want = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(lo.round_bf16(x.astype(np.float64)), want)
 
 
 def test_attention_lse_and_rows_sum_to_one():
@@ -216,7 +231,7 @@ def test_full_budget_equals_dense_attention_over_sorted_pyramid():
     r = rng(11)
     N, p, L, d = 64, 2, 4, 8
     Q, K, V = (r.standard_normal((N, d)) for _ in range(3))
-    Y, sv = lo.forward_head(Q, K, V, p, L, k=10 ** 6)
+    Y, sv = lo.forward_head(Q, K, V, p, L, k=10 ** 6, attn_dtype=None)
     # independent construction: every pyramid entry, sorted with Python's sort
     pyr = [lo.pyramid_pool(X, p, L) for X in (Q, K, V)]
     entries = sorted(((i + 1) * p ** l - 1, -l, l, i) for l in range(L) for i in range(N // p ** l))
@@ -271,7 +286,7 @@ def test_finite_differences():
     r = rng(15)
     N, d, p, L, k = 32, 8, 2, 3, 2
     Q, K, V, G = (r.standard_normal((N, d)) for _ in range(4))
-    Y, sv = lo.forward_head(Q, K, V, p, L, k)
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, attn_dtype=None)
     dQ, dK, dV, _ = lo.backward_head(G, sv)
     h = 1e-6
     for X, dX, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
@@ -282,8 +297,8 @@ def test_finite_differences():
                 args_m = [Q.copy(), K.copy(), V.copy()]
                 args_p[which][t, c] += h
                 args_m[which][t, c] -= h
-                Yp, svp = lo.forward_head(*args_p, p, L, k)
-                Ym, svm = lo.forward_head(*args_m, p, L, k)
+                Yp, svp = lo.forward_head(*args_p, p, L, k, attn_dtype=None)
+                Ym, svm = lo.forward_head(*args_m, p, L, k, attn_dtype=None)
                 for a, b in zip(svp["sel"] + svm["sel"], sv["sel"] + sv["sel"]):
                     np.testing.assert_array_equal(a, b)  # selection unchanged at +-h
                 num[t, c] = (np.sum(Yp * G) - np.sum(Ym * G)) / (2 * h)
@@ -338,7 +353,7 @@ def test_backward_matches_torch_autograd():
     r = rng(18)
     N, d, p, L, k = 256, 16, 4, 3, 5
     Q, K, V, G = (r.standard_normal((N, d)) for _ in range(4))
-    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=32)
+    Y, sv = lo.forward_head(Q, K, V, p, L, k, T=32, attn_dtype=None)
     dQ, dK, dV, _ = lo.backward_head(G, sv)
     lv = torch.from_numpy(sv["seq_level"])
     ix = torch.from_numpy(sv["seq_index"])
