@@ -1,0 +1,484 @@
+"""Throughput of one Lighthouse attention layer, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = lh_forward + lh_backward of one layer (all heads) over one batch of
+seeded synthetic inputs already resident in HBM.  The default workload is the
+512K-token layer (B=1, H=16, d=128, L=5, p=4, k=384, S=8192).  Each rank runs
+its own layer (weak scaling, no collective on the data path); the step time is
+the max over ranks of CUDA-event time on the launching stream.  Rank 0 prints
+one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the layer) on the host cores, one head per step, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from hierarchical_sparse_attention_pyramid_b200 import _lib, synth  # noqa: E402
+from hierarchical_sparse_attention_pyramid_b200 import api as lh  # noqa: E402
+
+METRIC = "Lighthouse attn fwd+bwd tokens/s/layer at N=512K on 1 B200; % of roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ stage-by-stage timing
+
+def _vp(base: int, off: int = 0):
+    return ctypes.c_void_p(base + off)
+
+
+def stage_calls(layer: lh.Layer, bufs: lh.Buffers, x: dict, y, grads):
+    """The eight stage entry points in lh_forward/lh_backward order, on the
+    same buffers, so each can be timed alone."""
+    I = bufs.info
+    cfg = layer.cfg()
+    c = bufs.ctx.data_ptr()
+    w = bufs.ws.data_ptr()
+    q, k, v, dy = (x[n].data_ptr() for n in ("q", "k", "v", "dy"))
+    dq, dk, dv = (g.data_ptr() for g in grads)
+    st = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)  # noqa: E731
+    S = ctypes.c_int64(I.S)
+    call = _lib.call
+    return [
+        ("pool", lambda: call("lh_pyramid_pool", ctypes.byref(cfg), _vp(q), _vp(k), _vp(v), _vp(w, I.ws_off_pyr_q),
+                              _vp(w, I.ws_off_pyr_k), _vp(w, I.ws_off_pyr_v), _vp(w, I.ws_off_norms), st())),
+        ("score_topk", lambda: call("lh_score_topk", ctypes.byref(cfg), _vp(w, I.ws_off_norms), _vp(w, I.ws_off_topk),
+                                    _vp(c, I.ctx_off_sel), st())),
+        ("gather", lambda: call("lh_gather", ctypes.byref(cfg), _vp(q), _vp(k), _vp(v), _vp(w, I.ws_off_pyr_q),
+                                _vp(w, I.ws_off_pyr_k), _vp(w, I.ws_off_pyr_v), _vp(c, I.ctx_off_sel),
+                                _vp(c, I.ctx_off_qs), _vp(c, I.ctx_off_ks), _vp(c, I.ctx_off_vs),
+                                _vp(c, I.ctx_off_seq_map), _vp(c, I.ctx_off_slot_of), st())),
+        ("attn_fwd", lambda: call("lh_attn_fwd", ctypes.byref(cfg), S, _vp(c, I.ctx_off_qs), _vp(c, I.ctx_off_ks),
+                                  _vp(c, I.ctx_off_vs), _vp(c, I.ctx_off_os), _vp(c, I.ctx_off_lse), _vp(w), st())),
+        ("scatter_back", lambda: call("lh_scatter_back", ctypes.byref(cfg), _vp(c, I.ctx_off_os),
+                                      _vp(c, I.ctx_off_slot_of), _vp(y.data_ptr()), st())),
+        ("scatter_adjoint", lambda: call("lh_scatter_back_adjoint", ctypes.byref(cfg), _vp(dy), _vp(c, I.ctx_off_seq_map),
+                                         _vp(c, I.ctx_off_os), _vp(w, I.ws_off_dos), _vp(w, I.ws_off_delta), st())),
+        ("attn_bwd", lambda: call("lh_attn_bwd", ctypes.byref(cfg), S, _vp(c, I.ctx_off_qs), _vp(c, I.ctx_off_ks),
+                                  _vp(c, I.ctx_off_vs), _vp(c, I.ctx_off_lse), _vp(w, I.ws_off_dos),
+                                  _vp(w, I.ws_off_delta), _vp(w, I.ws_off_dqs), _vp(w, I.ws_off_dks),
+                                  _vp(w, I.ws_off_dvs), _vp(w), st())),
+        ("pool_adjoint", lambda: call("lh_pool_adjoint", ctypes.byref(cfg), _vp(w, I.ws_off_dqs), _vp(w, I.ws_off_dks),
+                                      _vp(w, I.ws_off_dvs), _vp(c, I.ctx_off_slot_of), _vp(dq), _vp(dk), _vp(dv),
+                                      st())),
+    ]
+
+
+def stage_work(layer: lh.Layer, info) -> dict:
+    """Algorithmic bytes (HBM stages) or flops (attention) of one launch over the whole layer."""
+    e = 2 if layer.dtype == "bf16" else 4
+    BH, N, d, S = layer.BH, layer.N, layer.d, info.S
+    U, E = info.upper_entries, info.pyr_entries
+    return {
+        "pool": ("hbm", 3 * BH * N * d * e + 3 * BH * U * d * e + 2 * BH * N * 4),
+        "score_topk": ("hbm", 2 * BH * N * 4 + 2 * BH * U * 4 + BH * info.sel_per_head * 4),
+        "gather": ("hbm", 3 * BH * S * d * (e + 2) + BH * S * 4 + BH * E * 4),
+        "attn_fwd": ("tensor", 2 * S * S * d * BH),
+        "scatter_back": ("hbm", BH * N * d * e + BH * S * d * 2 + BH * E * 4),
+        "scatter_adjoint": ("hbm", BH * N * d * e + 2 * BH * S * d * 2 + BH * S * 8),
+        "attn_bwd": ("tensor", 5 * S * S * d * BH),
+        "pool_adjoint": ("hbm", 3 * BH * N * d * e + 3 * BH * S * d * 4 + BH * E * 4),
+    }
+
+
+def time_stages(calls, iters: int) -> dict:
+    """Average CUDA-event duration of each stage call on the current stream."""
+    st = torch.cuda.current_stream()
+    evs = {n: [] for n, _ in calls}
+    for _ in range(iters):
+        for n, f in calls:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            f()
+            b.record(st)
+            evs[n].append((a, b))
+    torch.cuda.synchronize()
+    return {n: float(np.mean([a.elapsed_time(b) for a, b in v])) for n, v in evs.items()}
+
+
+def source_sha(kernel: str) -> str:
+    files = {"pool": "lh_pool.cu", "pool_adjoint": "lh_pool.cu", "score_topk": "lh_select.cu",
+             "gather": "lh_gather.cu", "scatter_back": "lh_gather.cu", "scatter_adjoint": "lh_gather.cu",
+             "attn_fwd": "lh_attn_fwd.cu", "attn_bwd": "lh_attn_bwd.cu"}
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_sparse_attention_pyramid_b200", "csrc")
+    for f in (files[kernel], "lh_common.cuh", "sm100.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        ent = t.get(workload, {}).get(kernel)
+        if ent and ent.get("source_sha") == source_sha(kernel):
+            return ent["dram_bytes_per_launch"]
+    except Exception:  # noqa: BLE001
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w: synth.Workload, heads: int = 1, max_seconds: float = 60.0) -> dict:
+    """fp64 oracle forward + backward on `heads` head(s) of the workload; returns seconds per head."""
+    from oracle import lighthouse_oracle as lo
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    times = []
+    for h in range(heads):
+        x = synth.head_inputs(w, h)
+        arr = {n: t.double().numpy() for n, t in x.items()}
+        t0 = time.perf_counter()
+        Y, sv = lo.forward_head(arr["q"], arr["k"], arr["v"], w.p, w.L, w.k, w.chunk, w.scorer)
+        lo.backward_head(arr["dy"], sv)
+        times.append(time.perf_counter() - t0)
+        if sum(times) > max_seconds:
+            break
+    return {"sec_per_head": float(np.mean(times)), "heads": len(times), "cores": cores}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    # one head per step; the oracle keeps no state between steps, so warm-up
+    # steps only load the code paths
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(w.with_(N=min(w.N, 4096)), 1)
+    r_times = []
+    cores = None
+    for s in range(args.steps):
+        r = oracle_sample(w, 1)
+        r_times.append(r["sec_per_head"])
+        cores = r["cores"]
+    sec_layer = float(np.mean(r_times)) * w.B * w.H
+    value = w.B * w.N / sec_layer
+    sample = f"one of {w.B * w.H} heads per step (fp64 forward + backward), scaled to the layer"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: synth.Workload) -> dict:
+    info = lh.plan(lh.Layer.of(w))
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "L": w.L, "p": w.p, "k": w.k,
+            "chunk": w.chunk, "scorer": w.scorer, "S": int(info.S), "parallelism": "replicas (one layer per GPU)",
+            "l2": "inputs larger than L2 (Q,K,V,dY %.1f GB per GPU)" % (4 * w.B * w.H * w.N * w.d * 2 / 1e9)}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="sparse64_512k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    layer = lh.Layer.of(w)
+    x = synth.cuda_inputs(w, dev, seed=w.seed + 16 * rank)
+    bufs = lh.Buffers(layer, dev)
+    shp = (w.B, w.H, w.N, w.d)
+    y = torch.empty(shp, dtype=layer.torch_dtype, device=dev)
+    grads = tuple(torch.empty(shp, dtype=layer.torch_dtype, device=dev) for _ in range(3))
+
+    def step():
+        lh.forward(layer, x["q"], x["k"], x["v"], bufs, y)
+        lh.backward(layer, x["dy"], bufs, grads)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    lh.check_error(bufs)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    lh.check_error(bufs)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    value = world * w.B * w.N / (ms / 1e3)
+
+    # per-stage durations (same buffers, stage entry points one at a time)
+    calls = stage_calls(layer, bufs, x, y, grads)
+    stage_ms = time_stages(calls, max(3, min(args.steps, 10)))
+    lh.check_error(bufs)
+    pk, pk_src = peaks()
+    work = stage_work(layer, bufs.info)
+    stages = {}
+    for n, t in stage_ms.items():
+        kind, amount = work[n]
+        if kind == "hbm":
+            ach = amount / (t / 1e3) / 1e9
+            stages[n] = {"ms": t, "bound": "hbm", "achieved": ach, "unit": "GB/s", "frac": ach / pk["hbm_gbs"]}
+        else:
+            ach = amount / (t / 1e3) / 1e12
+            stages[n] = {"ms": t, "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                         "frac": ach / pk["bf16_tflops"]}
+    top = max(stage_ms, key=stage_ms.get)
+    ts = stages[top]
+    roofline = {"bound": ts["bound"], "kernel": top, "achieved": ts["achieved"],
+                "peak": pk["hbm_gbs"] if ts["bound"] == "hbm" else pk["bf16_tflops"], "unit": ts["unit"],
+                "frac": ts["frac"], "traffic": measured_traffic(top, w.name), "peak_source": pk_src,
+                "share_of_step": stage_ms[top] / sum(stage_ms.values())}
+    # whole-layer roofline: algorithmic bytes (Q,K,V,dY in; Y,dQ,dK,dV out) at the HBM
+    # peak plus the attention flops at the tensor peak
+    e = 2 if layer.dtype == "bf16" else 4
+    alg_bytes = 8 * layer.BH * w.N * w.d * e
+    t_roof = alg_bytes / (pk["hbm_gbs"] * 1e9) + (work["attn_fwd"][1] + work["attn_bwd"][1]) / (pk["bf16_tflops"] * 1e12)
+    layer_roof = {"t_roof_ms": t_roof * 1e3, "t_meas_ms": ms, "frac": t_roof * 1e3 / ms,
+                  "alg_bytes": alg_bytes, "attn_flops": work["attn_fwd"][1] + work["attn_bwd"][1]}
+
+    launches = lh.kernels_per_step(layer)
+
+    # end to end through the C ABI with host buffers: H2D of q,k,v,dy from pinned
+    # memory, forward + backward, D2H of y,dq,dk,dv, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "dy")}
+        hout = [torch.empty(shp, dtype=layer.torch_dtype).pin_memory() for _ in range(4)]
+        dx = {n: torch.empty_like(x[n]) for n in hx}
+        h2d = sum(t.numel() * t.element_size() for t in hx.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+
+        def e2e_step():
+            for n in hx:
+                dx[n].copy_(hx[n], non_blocking=True)
+            lh.forward(layer, dx["q"], dx["k"], dx["v"], bufs, y)
+            lh.backward(layer, dx["dy"], bufs, grads)
+            for t, s in zip(hout, (y, *grads)):
+                t.copy_(s, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        k_e = max(2, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(k_e):
+            e2e_step()
+        b.record(st)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e = max_over_ranks(a.elapsed_time(b) / k_e, world, dev)
+        e2e = {"value": world * w.B * w.N / (ms_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e, "steps": k_e}
+        del hx, hout, dx
+
+    dense = None
+    if not args.no_dense and rank == 0 and world == 1:
+        dense = dense_sdpa(x, ms, stage_ms)
+
+    cpu = None
+    if not args.no_cpu and rank == 0 and world == 1:
+        r = oracle_sample(w, 1)
+        sec_layer = r["sec_per_head"] * w.B * w.H
+        cpu = {"value": w.B * w.N / sec_layer, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+               "sample": f"one of {w.B * w.H} heads, fp64 forward + backward ({r['sec_per_head']:.1f} s), scaled to the layer"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic",
+            "config": workload_config(w), "clocks": clocks, "e2e": e2e, "gpu_launches": launches * args.steps,
+            "roofline": roofline, "layer_roofline": layer_roof, "stages": stages, "cpu_baseline": cpu,
+            "dense_sdpa": dense,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def dense_sdpa(x, lh_ms, stage_ms):
+    """Dense causal attention over all N tokens (cuDNN SDPA) for the speedup figure."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    q, k, v, dy = (x[n] for n in ("q", "k", "v", "dy"))
+    try:
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            def fwd():
+                return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+            fwd()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fwd()
+            b.record()
+            torch.cuda.synchronize()
+            t_fwd = a.elapsed_time(b)
+            qq, kk, vv = (t.detach().requires_grad_(True) for t in (q, k, v))
+            o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+            o.backward(dy)
+            torch.cuda.synchronize()
+            a.record()
+            o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+            o.backward(dy)
+            b.record()
+            torch.cuda.synchronize()
+            t_fb = a.elapsed_time(b)
+        lh_fwd = sum(stage_ms[n] for n in ("pool", "score_topk", "gather", "attn_fwd", "scatter_back"))
+        return {"backend": "cudnn", "fwd_ms": t_fwd, "fwdbwd_ms": t_fb, "speedup_fwd": t_fwd / lh_fwd,
+                "speedup_fwdbwd": t_fb / lh_ms}
+    except Exception as ex:  # noqa: BLE001
+        return {"error": str(ex)[:200]}
+
+
+if __name__ == "__main__":
+    main()

@@ -26,7 +26,7 @@ class LhConfig(ctypes.Structure):
                 ("k", c_int32), ("chunk", c_int32), ("dtype", c_int32), ("scorer", c_int32)]
 
 
-_SIZES = ["pyr_bytes", "norms_bytes", "topk_ws_bytes", "sel_bytes", "seq_bytes", "seq_map_bytes", "slot_of_bytes",
+_SIZES = ["pyr_bytes", "norms_bytes", "topk_ws_bytes", "sel_bytes", "seq_bytes", "os_bytes", "seq_map_bytes", "slot_of_bytes",
           "lse_bytes", "grad_seq_bytes", "attn_bwd_ws_bytes", "ctx_bytes", "ws_bytes",
           "ctx_off_sel", "ctx_off_seq_map", "ctx_off_slot_of", "ctx_off_qs", "ctx_off_ks", "ctx_off_vs",
           "ctx_off_os", "ctx_off_lse",

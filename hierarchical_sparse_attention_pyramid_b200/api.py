@@ -116,9 +116,9 @@ def gather(layer: Layer, q, k, v, pq, pk, pv, sel):
 
 
 def attn_fwd(layer: Layer, qs, ks, vs, ws=None):
-    """Causal attention over the sequence -> os [BH, S, d] bf16, lse [BH, S] fp32."""
+    """Causal attention over the sequence -> os [BH, S, d] fp32, lse [BH, S] fp32."""
     BH, S, d = qs.shape
-    os_ = _empty((BH, S, d), torch.bfloat16, qs.device)
+    os_ = _empty((BH, S, d), torch.float32, qs.device)
     lse = _empty((BH, S), torch.float32, qs.device)
     ws = _ws(0, qs.device) if ws is None else ws
     call("lh_attn_fwd", ctypes.byref(layer.cfg()), ctypes.c_int64(S), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse),
@@ -161,6 +161,18 @@ def pool_adjoint(layer: Layer, dqs, dks, dvs, slot_of):
 
 # ------------------------------------------------------------------ whole layer
 
+def kernels_per_step(layer: Layer) -> int:
+    """liblh kernel launches of one lh_forward + lh_backward (memsets excluded):
+    pool, score pyramid (one launch per 11/log2(p) levels), top-k, gather,
+    attention forward, scatter-back; scatter adjoint, attention backward,
+    pool adjoint."""
+    if layer.L == 1:
+        return 7
+    log2p = layer.p.bit_length() - 1
+    per_launch = 11 // log2p
+    return 8 + -(-(layer.L - 1) // per_launch)
+
+
 class Buffers:
     """Saved context and scratch of one layer shape, reusable across steps."""
 
@@ -186,7 +198,7 @@ class Buffers:
             qs=view(I.ctx_off_qs, BH * S * d, torch.bfloat16, (BH, S, d)),
             ks=view(I.ctx_off_ks, BH * S * d, torch.bfloat16, (BH, S, d)),
             vs=view(I.ctx_off_vs, BH * S * d, torch.bfloat16, (BH, S, d)),
-            os=view(I.ctx_off_os, BH * S * d, torch.bfloat16, (BH, S, d)),
+            os=view(I.ctx_off_os, BH * S * d, torch.float32, (BH, S, d)),
             lse=view(I.ctx_off_lse, BH * S, torch.float32, (BH, S)),
         )
 

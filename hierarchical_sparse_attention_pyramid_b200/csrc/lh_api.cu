@@ -93,6 +93,7 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   info->topk_ws_bytes = LH_ERR_WORD_BYTES + align_up((size_t)BH * upper * 4);
   info->sel_bytes = (size_t)BH * selsum * 4;
   info->seq_bytes = (size_t)BH * S * d * 2;
+  info->os_bytes = (size_t)BH * S * d * 4;
   info->seq_map_bytes = (size_t)BH * S * 4;
   info->slot_of_bytes = (size_t)BH * pyr * 4;
   info->lse_bytes = (size_t)BH * S * 4;
@@ -107,7 +108,7 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   info->ctx_off_qs = take(info->seq_bytes);
   info->ctx_off_ks = take(info->seq_bytes);
   info->ctx_off_vs = take(info->seq_bytes);
-  info->ctx_off_os = take(info->seq_bytes);
+  info->ctx_off_os = take(info->os_bytes);
   info->ctx_off_lse = take(info->lse_bytes);
   info->ctx_bytes = off;
 
@@ -209,7 +210,7 @@ lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const vo
   return LH_OK;
 }
 
-lh_status lh_attn_fwd(const lh_config* cfg, int64_t S, const void* qs, const void* ks, const void* vs, void* os,
+lh_status lh_attn_fwd(const lh_config* cfg, int64_t S, const void* qs, const void* ks, const void* vs, float* os,
                       float* lse, void* ws, lh_stream_t stream) {
   if (!cfg) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd: NULL cfg");
   if (cfg->B < 1 || cfg->H < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd: sizes must be positive");
@@ -240,7 +241,7 @@ lh_status lh_attn_bwd(const lh_config* cfg, int64_t S, const void* qs, const voi
   return LH_OK;
 }
 
-lh_status lh_scatter_back(const lh_config* cfg, const void* os, const int32_t* slot_of, void* y,
+lh_status lh_scatter_back(const lh_config* cfg, const float* os, const int32_t* slot_of, void* y,
                           lh_stream_t stream) {
   lh_plan_info info;
   Dims D;
@@ -251,7 +252,7 @@ lh_status lh_scatter_back(const lh_config* cfg, const void* os, const int32_t* s
   return LH_OK;
 }
 
-lh_status lh_scatter_back_adjoint(const lh_config* cfg, const void* dy, const int32_t* seq_map, const void* os,
+lh_status lh_scatter_back_adjoint(const lh_config* cfg, const void* dy, const int32_t* seq_map, const float* os,
                                   void* dos, float* delta, lh_stream_t stream) {
   lh_plan_info info;
   Dims D;
@@ -299,7 +300,7 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   void* qs = c + I.ctx_off_qs;
   void* ks = c + I.ctx_off_ks;
   void* vs = c + I.ctx_off_vs;
-  void* os = c + I.ctx_off_os;
+  float* os = reinterpret_cast<float*>(c + I.ctx_off_os);
   float* lse = reinterpret_cast<float*>(c + I.ctx_off_lse);
   LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st), "lh_forward: pool");
   LH_CUDA(launch_score_topk(D, norms, spyr, sel, errw, st), "lh_forward: score_topk");
@@ -327,7 +328,7 @@ lh_status lh_backward(const lh_config* cfg, const void* dy, const void* ctx, siz
   const void* qs = c + I.ctx_off_qs;
   const void* ks = c + I.ctx_off_ks;
   const void* vs = c + I.ctx_off_vs;
-  const void* os = c + I.ctx_off_os;
+  const float* os = reinterpret_cast<const float*>(c + I.ctx_off_os);
   const float* lse = reinterpret_cast<const float*>(c + I.ctx_off_lse);
   void* dos = w + I.ws_off_dos;
   float* delta = reinterpret_cast<float*>(w + I.ws_off_delta);

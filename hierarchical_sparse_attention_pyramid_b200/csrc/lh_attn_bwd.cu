@@ -9,8 +9,9 @@
 // One CTA owns a 128-row key/value tile of one (batch, head) and walks the
 // query tiles from the diagonal to the end.  Warp roles:
 //   warps 0-3  thread t owns key row t for S^T/dP^T (TMEM lane t): writes
-//              P^T and dS^T (bf16) to shared memory, then reads dQ row t of
-//              the query tile from TMEM and adds it to dQs with fp32 vector
+//              P^T, then dS^T, to shared memory as bf16 hi + lo pairs (so the
+//              products keep fp32-level accuracy), then reads dQ row t of the
+//              query tile from TMEM and adds it to dQs with fp32 vector
 //              atomics; at the end writes dKs and dVs rows
 //   warp 4     TMA producer: K, V once; Q and dO per query tile
 //   warp 5     MMA issuer (one thread) and TMEM owner
@@ -39,9 +40,9 @@ struct BwdSmem {
   static constexpr int oV = oK + kTile;
   static constexpr int oQ = oV + kTile;
   static constexpr int oO = oQ + kTile;  // dO
-  static constexpr int oPt = oO + kTile;
-  static constexpr int oSt = oPt + 2 * kChunk;  // dS^T
-  static constexpr int oVec = oSt + 2 * kChunk;  // LSE*log2e [128], Delta [128]
+  static constexpr int oHi = oO + kTile;        // P^T, then dS^T: bf16 high part
+  static constexpr int oLo = oHi + 2 * kChunk;  // bf16 of the remainder
+  static constexpr int oVec = oLo + 2 * kChunk;  // LSE*log2e [128], Delta [128]
   static constexpr int oBar = oVec + 1024;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
@@ -63,9 +64,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bKV = bars + 0;     // K, V landed
   uint64_t* bQO = bars + 1;     // Q_i, dO_i landed
   uint64_t* bSdP = bars + 2;    // S^T and dP^T in TMEM
-  uint64_t* bPS = bars + 3;     // P^T and dS^T in shared memory (128 arrivals)
-  uint64_t* bMM = bars + 4;     // dV, dK, dQ MMAs of the tile done
+  uint64_t* bP = bars + 3;      // P^T hi/lo in shared memory (128 arrivals)
+  uint64_t* bMM = bars + 4;     // dK, dQ MMAs of the tile done
   uint64_t* bDQfree = bars + 5; // dQ read out of TMEM (128 arrivals)
+  uint64_t* bPfree = bars + 6;  // dV MMAs done: the hi/lo buffers may take dS^T
+  uint64_t* bDS = bars + 7;     // dS^T hi/lo in shared memory (128 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
   float* sLSE = reinterpret_cast<float*>(smem + Lay::oVec);
@@ -81,9 +84,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bKV, 1);
     mbar_init(bQO, 1);
     mbar_init(bSdP, 1);
-    mbar_init(bPS, 128);
+    mbar_init(bP, 128);
     mbar_init(bMM, 1);
     mbar_init(bDQfree, 128);
+    mbar_init(bPfree, 1);
+    mbar_init(bDS, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idMM = idesc_bf16(128, D, true, true);   // A MN-major, B MN-major
       const uint32_t sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sO = smem_u32(smem + Lay::oO);
-      const uint32_t sPt = smem_u32(smem + Lay::oPt), sSt = smem_u32(smem + Lay::oSt);
+      const uint32_t sHi = smem_u32(smem + Lay::oHi), sLo = smem_u32(smem + Lay::oLo);
       bool ok = mbar_wait(bKV, 0, abort_flag);
       for (int it = 0; ok && it < n_q; ++it) {
         if (!mbar_wait(bQO, it & 1, abort_flag)) break;
@@ -142,25 +147,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     kk > 0 ? 1u : 0u);
         }
         umma_commit(bSdP);
-        if (!mbar_wait(bPS, it & 1, abort_flag)) break;
+        if (!mbar_wait(bP, it & 1, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q   (M = keys, K = queries, N = d)
+        // dV += P^T dO   (M = keys, K = queries, N = d), P^T = hi + lo
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          const uint32_t boff = kk * 2048;
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16(tmem + tDV, sdesc_sw128(sPt + aoff, 16, 1024), sdesc_sw128(sO + boff, Lay::kChunk, 1024), idKM,
-                    acc);
-          umma_bf16(tmem + tDK, sdesc_sw128(sSt + aoff, 16, 1024), sdesc_sw128(sQ + boff, Lay::kChunk, 1024), idKM,
-                    acc);
+          const uint64_t b = sdesc_sw128(sO + kk * 2048, Lay::kChunk, 1024);
+          umma_bf16(tmem + tDV, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + tDV, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
+        }
+        umma_commit(bPfree);
+        if (!mbar_wait(bDS, it & 1, abort_flag)) break;
+        tc_fence_after();
+        // dK += dS^T Q   (M = keys, K = queries, N = d), dS^T = hi + lo
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
+          const uint64_t b = sdesc_sw128(sQ + kk * 2048, Lay::kChunk, 1024);
+          umma_bf16(tmem + tDK, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + tDK, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
         }
         // dQ = dS K  (M = queries, K = keys, N = d): dS^T read M-major
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint32_t off = kk * 2048;
-          umma_bf16(tmem + tDP, sdesc_sw128(sSt + off, Lay::kChunk, 1024), sdesc_sw128(sK + off, Lay::kChunk, 1024),
-                    idMM, kk > 0 ? 1u : 0u);
+          const uint64_t b = sdesc_sw128(sK + off, Lay::kChunk, 1024);
+          umma_bf16(tmem + tDP, sdesc_sw128(sHi + off, Lay::kChunk, 1024), b, idMM, kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + tDP, sdesc_sw128(sLo + off, Lay::kChunk, 1024), b, idMM, 1u);
         }
         umma_commit(bMM);
       }
@@ -170,9 +184,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = threadIdx.x;  // 0..127
     const int kv_g = kt * BN + t;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* sPtb = smem + Lay::oPt;
-    uint8_t* sStb = smem + Lay::oSt;
+    uint8_t* sHib = smem + Lay::oHi;
+    uint8_t* sLob = smem + Lay::oLo;
     bool ok = true;
+    // write 32 consecutive query columns (chunk c) of this key row as bf16 hi + lo
+    auto put_row_chunk = [&](int c, const float (&x)[32]) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = x[8 * q + 2 * e], b = x[8 * q + 2 * e + 1];
+          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[e] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
+        }
+        const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
+        const int off = (c >> 1) * Lay::kChunk + t * 128 + ((ch ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4*>(sHib + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(sLob + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    };
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (kt + it) * BM;
       wg_sync();  // every thread is done with the previous tile's LSE / Delta
@@ -185,39 +217,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bSdP, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
+      // pass 1: P^T
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tl + tS + c * 32, sr);
+        tmem_ld_wait();
+        float pv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int qi = c * 32 + e;
+          pv[e] = (q0 + qi) >= kv_g ? exp2f(__uint_as_float(sr[e]) * scale_log2 - sLSE[qi]) : 0.f;
+        }
+        put_row_chunk(c, pv);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bP);
+      // pass 2: dS^T, once the dV MMAs have read P^T
+      if (!mbar_wait(bPfree, it & 1, abort_flag)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t sr[32], dr[32];
         tmem_ld32(tl + tS + c * 32, sr);
         tmem_ld32(tl + tDP + c * 32, dr);
         tmem_ld_wait();
-        uint32_t pp[16], dd[16];
+        float dv[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int qi = c * 32 + e + h;
-            const bool live = (q0 + qi) >= kv_g;
-            const float p = live ? exp2f(__uint_as_float(sr[e + h]) * scale_log2 - sLSE[qi]) : 0.f;
-            pv[h] = p;
-            dv[h] = p * (__uint_as_float(dr[e + h]) - sDel[qi]) * scale;
-          }
-          pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dd[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+        for (int e = 0; e < 32; ++e) {
+          const int qi = c * 32 + e;
+          const float p = (q0 + qi) >= kv_g ? exp2f(__uint_as_float(sr[e]) * scale_log2 - sLSE[qi]) : 0.f;
+          dv[e] = p * (__uint_as_float(dr[e]) - sDel[qi]) * scale;
         }
-        // columns c*32 .. c*32+31 = 4 chunks of 16 bytes in region c/2
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
-          const int off = (c >> 1) * Lay::kChunk + t * 128 + ((ch ^ (t & 7)) << 4);
-          *reinterpret_cast<uint4*>(sPtb + off) = make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
-          *reinterpret_cast<uint4*>(sStb + off) = make_uint4(dd[4 * q], dd[4 * q + 1], dd[4 * q + 2], dd[4 * q + 3]);
-        }
+        put_row_chunk(c, dv);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bPS);
+      mbar_arrive(bDS);
       // dQ of query row q0 + t
       if (!mbar_wait(bMM, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();

@@ -32,8 +32,9 @@ struct FwdSmem {
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kTile;
   static constexpr int oV = oK + 2 * kTile;
-  static constexpr int oP = oV + 2 * kTile;
-  static constexpr int oBar = oP + 2 * kChunk;
+  static constexpr int oP = oV + 2 * kTile;     // P_hi: bf16(P)
+  static constexpr int oPl = oP + 2 * kChunk;   // P_lo: bf16(P - P_hi)
+  static constexpr int oBar = oPl + 2 * kChunk;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -41,7 +42,7 @@ struct FwdSmem {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O, float* __restrict__ LSE,
+                    const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, float* __restrict__ LSE,
                     int* errw, int S, float scale_log2) {
   using Lay = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idPV = idesc_bf16(BM, D, false, true);
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sK = smem_u32(smem + Lay::oK);
       const uint32_t sV = smem_u32(smem + Lay::oV), sP = smem_u32(smem + Lay::oP);
+      const uint32_t sPl = smem_u32(smem + Lay::oPl);
       auto issue_pv = [&](int jj) -> bool {
         const int st = jj & 1;
         if (!mbar_wait(bP, jj & 1, abort_flag)) return false;
@@ -118,9 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vb = sV + st * Lay::kTile;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sP + (kk >> 2) * Lay::kChunk + (kk & 3) * 32, 16, 1024);
+          const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
           const uint64_t b = sdesc_sw128(vb + kk * 2048, Lay::kChunk, 1024);
-          umma_bf16(tmem + 256, a, b, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + 256, sdesc_sw128(sP + aoff, 16, 1024), b, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + 256, sdesc_sw128(sPl + aoff, 16, 1024), b, idPV, 1u);
         }
         umma_commit(bO);
         umma_commit(&bKVfree[st]);
@@ -150,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_g = qt * BM + row;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     uint8_t* sPb = smem + Lay::oP;
+    uint8_t* sPlb = smem + Lay::oPl;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
@@ -177,15 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_run, mx);
       const float alpha = exp2f(m_run - m_new);
       float rs = 0.f;
-      uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = exp2f(s[2 * c] - m_new), p1 = exp2f(s[2 * c + 1] - m_new);
-        rs += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
+      for (int c = 0; c < 128; ++c) {
+        s[c] = exp2f(s[c] - m_new);
+        rs += s[c];
       }
       if (j >= 1) {
-        // PV of the previous tile must be done: O is stable and the P buffer free
+        // PV of the previous tile must be done: O is stable and the P buffers free
         if (!mbar_wait(bO, (j - 1) & 1, abort_flag)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
@@ -204,11 +206,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l_run = l_run * alpha + rs;
       m_run = m_new;
+      // P = P_hi + P_lo, both bf16, so that P V keeps fp32-level accuracy
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
-        const int region = ch >> 3, cc = ch & 7;
-        const uint4 val = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(sPb + region * Lay::kChunk + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a = s[8 * ch + 2 * q], b = s[8 * ch + 2 * q + 1];
+          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          hi[q] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[q] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
+        }
+        const int off = (ch >> 3) * Lay::kChunk + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(sPb + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(sPlb + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -224,14 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tl + 256 + c * 32, o);
         tmem_ld_wait();
         if (row_g < S) {
-          uint4* dst = reinterpret_cast<uint4*>(O + ((int64_t)bh * S + row_g) * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(O + ((int64_t)bh * S + row_g) * D + c * 32);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l),
-                                pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l));
-          }
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                 __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
         }
       }
       if (row_g < S) LSE[(int64_t)bh * S + row_g] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
@@ -273,7 +281,7 @@ bool make_seq_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, in
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, void* os,
+cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
                             float* lse, int* errw, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_seq_map(&mq, qs, BH, S, d, BM) || !make_seq_map(&mk, ks, BH, S, d, BN) ||
@@ -285,13 +293,13 @@ cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const 
     const int smem = FwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(os), lse, errw,
+    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw,
                                                         (int)S, scale_log2);
   } else {
     const int smem = FwdSmem<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(os), lse, errw,
+    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw,
                                                        (int)S, scale_log2);
   }
   return cudaGetLastError();

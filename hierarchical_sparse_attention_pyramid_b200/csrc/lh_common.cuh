@@ -109,12 +109,12 @@ cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, in
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
                           const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
                           int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st);
-cudaError_t launch_scatter_back(const Dims& D, const void* os, const int32_t* slot_of, void* y, cudaStream_t st);
-cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const void* os,
+cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st);
+cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
                                    void* dos, float* delta, int* errw, cudaStream_t st);
 cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dks, const float* dvs,
                                 const int32_t* slot_of, void* dq, void* dk, void* dv, cudaStream_t st);
-cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, void* os,
+cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
                             float* lse, int* errw, cudaStream_t st);
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,

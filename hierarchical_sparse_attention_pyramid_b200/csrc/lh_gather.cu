@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(GatherArgs a) {
 // one row per warp instruction; levels >= 1 are cached between their boundaries
 // ---------------------------------------------------------------------------
 struct ScatterArgs {
-  const __nv_bfloat16* os;
+  const float* os;
   const int32_t* slot_of;
   void* y;
   int64_t BH, N, S, pyr_entries;
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
   const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
   const int log2p = a.log2p;
   const int32_t* so = a.slot_of + bh * a.pyr_entries;
-  const __nv_bfloat16* os = a.os + bh * a.S * D + lane * VE;
+  const float* os = a.os + bh * a.S * D + lane * VE;
   T* out = static_cast<T*>(a.y) + (bh * a.N + row0) * D + lane * VE;
 
   float up[NL + 1][VE];
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
             const int64_t i = ((j + 1) >> (l * log2p)) - 1;
             const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
             if (s >= 0) {
-              load_vec_rw<__nv_bfloat16, VE>(os + (int64_t)s * D, up[l]);
+              load_f32<VE>(os + (int64_t)s * D, up[l]);
             } else {
 #pragma unroll
               for (int c = 0; c < VE; ++c) up[l][c] = 0.f;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
     for (int c = 0; c < VE; ++c) y[c] = upper[c];
     if (s0 >= 0) {
       float v[VE];
-      load_vec_rw<__nv_bfloat16, VE>(os + (int64_t)s0 * D, v);
+      load_f32<VE>(os + (int64_t)s0 * D, v);
 #pragma unroll
       for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
     }
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 struct ScatterAdjArgs {
   const void* dy;
   const int32_t* seq_map;
-  const __nv_bfloat16* os;
+  const float* os;
   __nv_bfloat16* dos;
   float* delta;
   int* errw;
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_adjoint_kernel(ScatterAdj
   // round to bf16 once; Delta from the rounded values and the bf16 Os
   __nv_bfloat16 h[VE];
   float o_row[VE];
-  load_vec_rw<__nv_bfloat16, VE>(a.os + (bh * a.S + s) * D + cv * VE, o_row);
+  load_f32<VE>(a.os + (bh * a.S + s) * D + cv * VE, o_row);
   float dot = 0.f;
 #pragma unroll
   for (int c = 0; c < VE; ++c) {
@@ -313,9 +313,9 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter_back(const Dims& D, const void* os, const int32_t* slot_of, void* y, cudaStream_t st) {
+cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st) {
   ScatterArgs a{};
-  a.os = static_cast<const __nv_bfloat16*>(os);
+  a.os = os;
   a.slot_of = slot_of;
   a.y = y;
   a.BH = D.BH; a.N = D.N; a.S = D.S; a.pyr_entries = D.pyr_entries;
@@ -333,12 +333,12 @@ cudaError_t launch_scatter_back(const Dims& D, const void* os, const int32_t* sl
                     : scatter_dispatch_L<float, 64>(D.L, a, blocks, st);
 }
 
-cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const void* os,
+cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
                                    void* dos, float* delta, int* errw, cudaStream_t st) {
   ScatterAdjArgs a{};
   a.dy = dy;
   a.seq_map = seq_map;
-  a.os = static_cast<const __nv_bfloat16*>(os);
+  a.os = os;
   a.dos = static_cast<__nv_bfloat16*>(dos);
   a.delta = delta;
   a.errw = errw;

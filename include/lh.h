@@ -17,8 +17,8 @@
  *    parameter says "host", and must be 16-byte aligned.
  *  - Layouts are dense row-major.  "BH" = B*H flattened; Q, K, V, Y, dY, dQ,
  *    dK, dV are [B][H][N][d] in cfg->dtype.  The gathered sequence tensors
- *    Qs, Ks, Vs, Os, dOs are [BH][S][d] bf16; LSE and Delta are [BH][S] fp32;
- *    dQs, dKs, dVs are [BH][S][d] fp32.
+ *    Qs, Ks, Vs, dOs are [BH][S][d] bf16; Os, dQs, dKs, dVs are [BH][S][d]
+ *    fp32; LSE and Delta are [BH][S] fp32.
  *  - Support: d in {64, 128}; p a power of two >= 2; 1 <= L <= 16;
  *    N divisible by p^(L-1); N < 2^28; k >= 1; B*H <= 65535 * 65535.
  *    dtype LH_FP32 pools and scores in fp32 and casts the gathered sequence
@@ -95,7 +95,8 @@ typedef struct {
   size_t norms_bytes;   /* [2][BH][N] fp32 */
   size_t topk_ws_bytes; /* ws of lh_score_topk */
   size_t sel_bytes;     /* [BH][sel_per_head] int32 */
-  size_t seq_bytes;     /* one of qs/ks/vs/os: [BH][S][d] bf16 */
+  size_t seq_bytes;     /* one of qs/ks/vs/dos: [BH][S][d] bf16 */
+  size_t os_bytes;      /* os: [BH][S][d] fp32 */
   size_t seq_map_bytes; /* [BH][S] int32 */
   size_t slot_of_bytes; /* [BH][pyr_entries] int32 */
   size_t lse_bytes;     /* [BH][S] fp32 (also Delta) */
@@ -157,13 +158,16 @@ lh_status lh_gather(const lh_config *cfg, const void *q, const void *k, const vo
  * Cite: LH-summary "Technical details" (3) (stock attention over the gathered
  * S tokens); LH-post "How it works" (3).  Softmax scale 1/sqrt(d); slot t
  * attends to slots u <= t.  Uses cfg->B, H, d only; S is any length >= 1.
- * Out: os [BH][S][d] bf16; lse [BH][S] fp32, natural log of the row's sum of
+ * The bf16 inputs are multiplied exactly and accumulated in fp32; the
+ * probabilities enter P V as a bf16 pair (hi + lo), so O keeps fp32 accuracy.
+ * Out: os [BH][S][d] fp32; lse [BH][S] fp32, natural log of the row's sum of
  *      exp(scaled logits).  ws: at least LH_ERR_WORD_BYTES (error word). */
-lh_status lh_attn_fwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs, void *os,
+lh_status lh_attn_fwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs, float *os,
                       float *lse, void *ws, lh_stream_t stream);
 
 /* Stage 4 backward.  Cite: LH-summary "Method" step 5 (the gradient flows
- * back through the attention kernel).
+ * back through the attention kernel).  P and dS enter their products as bf16
+ * hi + lo pairs, so dQs, dKs, dVs keep fp32 accuracy for bf16 inputs.
  * In:  qs, ks, vs, lse from the forward; dos [BH][S][d] bf16 and
  *      delta [BH][S] fp32 (rowsum(dOs * Os)) from lh_scatter_back_adjoint.
  * Out: dqs, dks, dvs [BH][S][d] fp32 (dqs is zeroed and accumulated here).
@@ -176,17 +180,17 @@ lh_status lh_attn_bwd(const lh_config *cfg, int64_t S, const void *qs, const voi
  * return to the N positions and each position j sums over the ranges
  * R(l, i)); LH-post "How it works" (4) (shifted ranges keep causality).
  * Y_j = sum over l of Os[slot(l, floor((j+1)/p^l) - 1)] for kept entries,
- * summed in fp32 from l = 0 up and rounded once; R(l, i) =
+ * summed in fp32 and rounded once; R(l, i) =
  * [(i+1) p^l - 1, (i+2) p^l - 1).  Positions with no contributor get 0.
  * Out: y [BH][N][d] dtype. */
-lh_status lh_scatter_back(const lh_config *cfg, const void *os, const int32_t *slot_of, void *y,
+lh_status lh_scatter_back(const lh_config *cfg, const float *os, const int32_t *slot_of, void *y,
                           lh_stream_t stream);
 
 /* Stage 5 backward: dOs[slot(l,i)] = sum of dY_j over j in R(l, i) (fp32,
  * rounded once to bf16), and delta[s] = sum_c dOs[s,c] * Os[s,c] (fp32, from
- * the bf16 values).  Cite: LH-summary "Method" step 5.
+ * the bf16 dOs and the fp32 Os).  Cite: LH-summary "Method" step 5.
  * Out: dos [BH][S][d] bf16, delta [BH][S] fp32. */
-lh_status lh_scatter_back_adjoint(const lh_config *cfg, const void *dy, const int32_t *seq_map, const void *os,
+lh_status lh_scatter_back_adjoint(const lh_config *cfg, const void *dy, const int32_t *seq_map, const float *os,
                                   void *dos, float *delta, lh_stream_t stream);
 
 /* Stages 3 and 1 backward: dX_t = sum over l of p^-l * dXs[slot(l, floor(t/p^l))]

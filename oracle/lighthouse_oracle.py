@@ -44,9 +44,10 @@ Readings of points the pages leave open (each one is listed in the design doc):
   R9  selection is per (batch, head).
   R11 the pages run the gathered sequence through stock FlashAttention, a
       16-bit kernel (LH-summary Technical details (3); LH-post How it works
-      (3)), so the attention inputs Qs, Ks, Vs are rounded to bf16 (round to
-      nearest even) before the attention; the backward passes gradients
-      through that cast unchanged.  attn_dtype=None keeps them exact.
+      (3)), so the attention inputs Qs, Ks, Vs, and the output gradient dOs
+      that its backward takes, are rounded to bf16 (round to nearest even);
+      the backward passes gradients through those casts unchanged.
+      attn_dtype=None keeps them exact.
 
 All arrays are float64 numpy arrays; one head at a time is ``[N, d]``.
 """
@@ -309,7 +310,7 @@ def forward_head(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer
         raise ValueError(f"unknown attn_dtype {attn_dtype!r}")
     Os, lse = causal_attention(Qs, Ks, Vs)
     Y = scatter_back(Os, seq_level, seq_index, N, p, L)
-    saved = dict(N=N, p=p, L=L, k=k, T=T, scorer=scorer, sel=sel, spyr=spyr,
+    saved = dict(N=N, p=p, L=L, k=k, T=T, scorer=scorer, attn_dtype=attn_dtype, sel=sel, spyr=spyr,
                  pyr_q=pq, pyr_k=pk, pyr_v=pv,
                  seq_level=seq_level, seq_index=seq_index,
                  slot_of=slot_table(seq_level, seq_index, N, p, L),
@@ -372,7 +373,10 @@ def pyramid_pool_adjoint(dlevels, p: int) -> np.ndarray:
     of its parent's gradient, added to its own."""
     acc = dlevels[-1]
     for l in range(len(dlevels) - 2, -1, -1):
-        acc = dlevels[l] + np.repeat(acc, p, axis=0) / p
+        n, d = acc.shape
+        child = np.array(dlevels[l], dtype=np.float64).reshape(n, p, d)
+        child += (acc / p)[:, None, :]
+        acc = child.reshape(n * p, d)
     return acc
 
 
@@ -382,6 +386,8 @@ def backward_head(dY, saved):
     N, p, L = saved["N"], saved["p"], saved["L"]
     sl, si = saved["seq_level"], saved["seq_index"]
     dOs = scatter_adjoint(dY, sl, si, N, p)
+    if saved.get("attn_dtype") == "bf16":
+        dOs = round_bf16(dOs)
     dQs, dKs, dVs = causal_attention_backward(saved["Qs"], saved["Ks"], saved["Vs"], dOs)
     grads = [pyramid_pool_adjoint(gather_adjoint(g, sl, si, N, p, L), p) for g in (dQs, dKs, dVs)]
     return grads[0], grads[1], grads[2], dict(dOs=dOs, dQs=dQs, dKs=dKs, dVs=dVs)

@@ -142,7 +142,7 @@ def test_scatter_back(name):
     w, x, heads = case(name)
     L = layer_of(w)
     info = lh.plan(L)
-    os_ = torch.stack([_bf16(o["saved"]["Os"]) for o in heads]).cuda()
+    os_ = torch.stack([torch.from_numpy(o["saved"]["Os"]).float() for o in heads]).cuda()
     slot_of = torch.stack([torch.from_numpy(pu.oracle_slot_of(o["saved"]).astype(np.int32)) for o in heads]).cuda()
     y = lh.scatter_back(L, os_, slot_of)
     torch.cuda.synchronize()
@@ -158,7 +158,7 @@ def test_scatter_back(name):
 def test_scatter_adjoint(name):
     w, x, heads = case(name)
     L = layer_of(w)
-    os_ = torch.stack([_bf16(o["saved"]["Os"]) for o in heads]).cuda()
+    os_ = torch.stack([torch.from_numpy(o["saved"]["Os"]).float() for o in heads]).cuda()
     seq_map = torch.stack([torch.from_numpy(pu.oracle_seq_map(o["saved"]).astype(np.int32)) for o in heads]).cuda()
     dos, delta = lh.scatter_back_adjoint(L, x["dy"], seq_map, os_)
     torch.cuda.synchronize()
