@@ -109,7 +109,9 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(GatherArgs a) {
 
 // ---------------------------------------------------------------------------
 // scatter-back: Y_j = sum_l [kept] Os[slot(l, ((j+1) >> l log2p) - 1)]
-// one row per warp instruction; levels >= 1 are cached between their boundaries
+// 16-byte output lanes, R (1 or 2) rows per warp instruction.  Each lane keeps
+// the summed contribution of levels >= 1 for its own row and refreshes it when
+// that row's level-1 entry changes (coarser boundaries are level-1 boundaries).
 // ---------------------------------------------------------------------------
 struct ScatterArgs {
   const float* os;
@@ -121,10 +123,20 @@ struct ScatterArgs {
   int task_rows, log2p;
 };
 
+template <typename T, int D>
+struct RowLayout {
+  static constexpr int VE = 16 / sizeof(T) <= D / 16 ? 16 / sizeof(T) : D / 16;  // elements per lane
+  static constexpr int LPR = D / VE;                                            // lanes per row
+  static constexpr int R = 32 / LPR;                                            // rows per instruction
+  static_assert(R == 1 || R == 2, "layout");
+};
+
 template <typename T, int D, int NL>
 __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a) {
-  constexpr int VE = D / 32;
+  using Lay = RowLayout<T, D>;
+  constexpr int VE = Lay::VE, LPR = Lay::LPR, R = Lay::R;
   const int lane = threadIdx.x & 31;
+  const int lr = lane / LPR, cv = lane % LPR;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t bh = wid / a.tasks_per_head;
   if (bh >= a.BH) return;
@@ -132,42 +144,37 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
   const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
   const int log2p = a.log2p;
   const int32_t* so = a.slot_of + bh * a.pyr_entries;
-  const float* os = a.os + bh * a.S * D + lane * VE;
-  T* out = static_cast<T*>(a.y) + (bh * a.N + row0) * D + lane * VE;
+  const float* os = a.os + bh * a.S * D + cv * VE;
+  T* out = static_cast<T*>(a.y) + (bh * a.N + row0) * D + cv * VE;
 
-  float up[NL + 1][VE];
   float upper[VE];
 #pragma unroll
-  for (int i = 0; i < VE; ++i) upper[i] = 0.f;
+  for (int c = 0; c < VE; ++c) upper[c] = 0.f;
+  int64_t cur1 = -2;  // level-1 entry of this lane's previous row
   int s0w = -1;
-  for (int r = 0; r < rows; ++r) {
-    const int64_t j = row0 + r;
-    if ((r & 31) == 0) s0w = (r + lane < rows) ? so[a.level_off[0] + j + lane] : -1;
+  for (int r = 0; r < rows; r += R) {
+    const int64_t j = row0 + r + lr;  // this lane's row
+    if ((r & 31) == 0) s0w = (r + lane < rows) ? so[a.level_off[0] + row0 + r + lane] : -1;
     if constexpr (NL > 1) {
-      if (r == 0 || ((j + 1) & ((1 << log2p) - 1)) == 0) {
+      const int64_t i1 = ((j + 1) >> log2p) - 1;
+      if (i1 != cur1) {
+        cur1 = i1;
+#pragma unroll
+        for (int c = 0; c < VE; ++c) upper[c] = 0.f;
 #pragma unroll
         for (int l = 1; l < NL; ++l) {
-          if (r == 0 || ((j + 1) & ((1ll << (l * log2p)) - 1)) == 0) {
-            const int64_t i = ((j + 1) >> (l * log2p)) - 1;
-            const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
-            if (s >= 0) {
-              load_f32<VE>(os + (int64_t)s * D, up[l]);
-            } else {
+          const int64_t i = ((j + 1) >> (l * log2p)) - 1;
+          const int s = (i >= 0 && j < a.N) ? so[a.level_off[l] + i] : -1;
+          if (s >= 0) {
+            float v[VE];
+            load_f32<VE>(os + (int64_t)s * D, v);
 #pragma unroll
-              for (int c = 0; c < VE; ++c) up[l][c] = 0.f;
-            }
+            for (int c = 0; c < VE; ++c) upper[c] += v[c];
           }
-        }
-#pragma unroll
-        for (int c = 0; c < VE; ++c) {
-          float s = 0.f;
-#pragma unroll
-          for (int l = 1; l < NL; ++l) s += up[l][c];
-          upper[c] = s;
         }
       }
     }
-    const int s0 = __shfl_sync(kFull, s0w, r & 31);
+    const int s0 = __shfl_sync(kFull, s0w, (r & 31) + lr);
     float y[VE];
 #pragma unroll
     for (int c = 0; c < VE; ++c) y[c] = upper[c];
@@ -177,7 +184,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 #pragma unroll
       for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
     }
-    store_vec<T, VE>(out + (int64_t)r * D, y);
+    if (r + lr < rows) store_vec<T, VE>(out + (int64_t)(r + lr) * D, y);
   }
 }
 

@@ -18,16 +18,6 @@ constexpr int kWarps = 8;   // warps per block
 constexpr int kUnroll = 8;  // row groups loaded ahead per warp
 constexpr unsigned kFull = 0xffffffffu;
 
-// 16-byte lanes for bf16 d=128 (8 elements), 8- or 16-byte lanes otherwise;
-// R rows per warp instruction, and R <= 2 <= p always.
-template <typename T, int D>
-struct PoolLayout {
-  static constexpr int VE = (sizeof(T) == 2 && D == 128) ? 8 : 4;
-  static constexpr int LPR = D / VE;  // lanes per row
-  static constexpr int R = 32 / LPR;  // rows per warp instruction
-  static_assert(R == 1 || R == 2, "layout");
-};
-
 struct PoolArgs {
   const void* x[3];
   void* pyr[3];
@@ -38,11 +28,45 @@ struct PoolArgs {
   int task_rows, log2p;
 };
 
+// Butterfly reduce-scatter of U (8 or 16) per-lane partial sums, one per row
+// of a batch, over the 32 lanes.  Halving stages (xor 16, 8, ...) leave each
+// lane with one row's partial; the remaining xor stages complete the sum.
+// Afterwards the lanes with (lane % (32 / U)) == 0 hold the full sum of row
+// scatter_row<U>(lane).
+template <int U>
+__device__ __forceinline__ int scatter_row(int lane) {
+  int r = 0;
+#pragma unroll
+  for (int b = 4, w = U / 2; w >= 1; --b, w >>= 1) r += ((lane >> b) & 1) * w;
+  return r;
+}
+
+template <int U>
+__device__ __forceinline__ float reduce_scatter(float (&v)[U], int lane) {
+#pragma unroll
+  for (int half = U / 2, b = 16; half >= 1; half >>= 1, b >>= 1) {
+    const bool up = lane & b;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? v[i] : v[i + half];
+      const float keep = up ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(kFull, send, b);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int b = 16 / U; b >= 1; b >>= 1) t += __shfl_xor_sync(kFull, t, b);
+  return t;
+}
+
+// One warp walks task_rows consecutive rows of one head of one of Q, K, V.
+// Lane l holds channels [l*VE, l*VE+VE) of every row, so the pooled sums need
+// no cross-lane work; only the norms of Q and K rows are reduced across lanes.
 template <typename T, int D, int NL>
-__global__ void __launch_bounds__(kWarps * 32) pool_kernel(PoolArgs a) {
-  using Lay = PoolLayout<T, D>;
-  constexpr int VE = Lay::VE, LPR = Lay::LPR, R = Lay::R;
-  constexpr int GPW = 32 / R;  // row groups per 32-row window of norms
+__global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
+  constexpr int VE = D / 32;
+  constexpr int U = sizeof(T) * VE >= 16 ? 8 : 16;  // rows loaded per batch
+  using Raw = typename RawVec<sizeof(T) * VE>::type;
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int tensor = (int)(wid % 3);
@@ -51,81 +75,52 @@ __global__ void __launch_bounds__(kWarps * 32) pool_kernel(PoolArgs a) {
   if (bh >= a.BH) return;
   const int64_t row0 = (rest % a.tasks_per_head) * a.task_rows;
   const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
-  const int lr = lane / LPR, cv = lane % LPR;
   const int log2p = a.log2p;
-  const T* src = static_cast<const T*>(a.x[tensor]) + (bh * a.N + row0) * D + cv * VE;
-  T* dst = static_cast<T*>(a.pyr[tensor]);
-  const int n_rg = (rows + R - 1) / R;
+  const Raw* src = reinterpret_cast<const Raw*>(static_cast<const T*>(a.x[tensor]) + (bh * a.N + row0) * D) + lane;
+  T* dst = static_cast<T*>(a.pyr[tensor]) + bh * a.upper_entries * D + lane * VE;
   const bool want_norm = tensor < 2;
   float* norm_out = a.norms + ((int64_t)tensor * a.BH + bh) * a.N + row0;
+  const int rid = scatter_row<U>(lane);
 
   float acc[NL + 1][VE];
 #pragma unroll
   for (int l = 0; l <= NL; ++l)
 #pragma unroll
     for (int i = 0; i < VE; ++i) acc[l][i] = 0.f;
-  float mynorm = 0.f;
 
-  auto write_level = [&](int l, int64_t e_rel, const float (&v)[VE]) {
-    if (lr != 0) return;
-    float m[VE];
-    const float inv = ldexpf(1.f, -l * log2p);  // exact power of two
+  auto load = [&](Raw (&x)[U], int r0) {
 #pragma unroll
-    for (int i = 0; i < VE; ++i) m[i] = v[i] * inv;
-    const int64_t e = (row0 >> (l * log2p)) + e_rel;
-    store_vec<T, VE>(dst + (bh * a.upper_entries + a.upper_off[l] + e) * D + cv * VE, m);
-  };
-
-  for (int g0 = 0; g0 < n_rg; g0 += kUnroll) {
-    float x[kUnroll][VE];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int row = (g0 + u) * R + lr;
-      if (g0 + u < n_rg && row < rows) {
-        load_vec<T, VE>(src + (int64_t)row * D, x[u]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < VE; ++i) x[u][i] = 0.f;
-      }
+    for (int u = 0; u < U; ++u) {
+      if (r0 + u < rows) x[u] = __ldg(src + (int64_t)(r0 + u) * (D / VE));
+      else x[u] = Raw{};
     }
+  };
+  auto process = [&](const Raw (&x)[U], int r0) {
+    float sq[U];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int g = g0 + u;
-      if (g >= n_rg) break;
-      if (want_norm) {
-        float sq = 0.f;
+    for (int u = 0; u < U; ++u) {
+      const T* e = reinterpret_cast<const T*>(&x[u]);
+      float v[VE];
 #pragma unroll
-        for (int i = 0; i < VE; ++i) sq = fmaf(x[u][i], x[u][i], sq);
+      for (int i = 0; i < VE; ++i) v[i] = Elem<T>::to_f(e[i]);
+      float q = 0.f;
 #pragma unroll
-        for (int o = LPR / 2; o >= 1; o >>= 1) sq += __shfl_xor_sync(kFull, sq, o);
-        const float t = __shfl_sync(kFull, sq, (lane % R) * LPR);
-        if (lane / R == g % GPW) mynorm = sqrtf(t);
-        if (g % GPW == GPW - 1 || g == n_rg - 1) {
-          const int r = (g / GPW) * 32 + lane;
-          if (r < rows) norm_out[r] = mynorm;
-        }
-      }
+      for (int i = 0; i < VE; ++i) q = fmaf(v[i], v[i], q);
+      sq[u] = q;
       if constexpr (NL > 1) {
 #pragma unroll
-        for (int i = 0; i < VE; ++i) acc[1][i] += x[u][i];
-        const int done = (g + 1) * R;  // rows of this task consumed so far
-        if ((done & ((1 << log2p) - 1)) == 0) {
-          // a level-1 entry is complete: add the R row lanes together
-          float s1[VE];
+        for (int i = 0; i < VE; ++i) acc[1][i] += v[i];
+        const int done = r0 + u + 1;  // rows of this task consumed
+        if (done <= rows && (done & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
-          for (int i = 0; i < VE; ++i) {
-            float v = acc[1][i];
-#pragma unroll
-            for (int o = LPR; o < 32; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
-            s1[i] = v;
-            acc[1][i] = 0.f;
-            acc[2][i] += v;
-          }
-          write_level(1, (done >> log2p) - 1, s1);
-#pragma unroll
-          for (int l = 2; l < NL; ++l) {
+          for (int l = 1; l < NL; ++l) {
             if ((done & ((1 << (l * log2p)) - 1)) != 0) break;
-            write_level(l, (done >> (l * log2p)) - 1, acc[l]);
+            const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
+            float m[VE];
+#pragma unroll
+            for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
+            const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
+            store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
 #pragma unroll
             for (int i = 0; i < VE; ++i) {
               acc[l + 1][i] += acc[l][i];
@@ -135,13 +130,31 @@ __global__ void __launch_bounds__(kWarps * 32) pool_kernel(PoolArgs a) {
         }
       }
     }
+    if (want_norm) {
+      const float tot = reduce_scatter<U>(sq, lane);
+      const int r = r0 + rid;
+      if ((lane & (32 / U - 1)) == 0 && r < rows) norm_out[r] = sqrtf(tot);
+    }
+  };
+
+  // two batches in flight: the loads of the next batch are issued before the
+  // current one is processed
+  Raw xa[U], xb[U];
+  load(xa, 0);
+  for (int r0 = 0; r0 < rows; r0 += 2 * U) {
+    if (r0 + U < rows) load(xb, r0 + U);
+    process(xa, r0);
+    if (r0 + U >= rows) break;
+    if (r0 + 2 * U < rows) load(xa, r0 + 2 * U);
+    process(xb, r0 + U);
   }
 }
 
 // ---------------------------------------------------------------------------
 // adjoint: dX_t = sum_l [kept(l, t >> l log2p)] p^-l dXs[slot]  (fp32, rounded once)
-// one row per warp instruction; contributions of levels >= 1 are cached and
-// refreshed only when t crosses a level-1 boundary.
+// 16-byte output lanes, R (1 or 2) rows per warp instruction; the rows of an
+// instruction share every entry of level >= 1 (t is even when R = 2 and p >= 2),
+// whose scaled contributions are cached and refreshed at level-1 boundaries.
 // ---------------------------------------------------------------------------
 struct PoolAdjArgs {
   const float* dxs[3];
@@ -153,10 +166,20 @@ struct PoolAdjArgs {
   int task_rows, log2p;
 };
 
+template <typename T, int D>
+struct RowLayout {
+  static constexpr int VE = 16 / sizeof(T) <= D / 16 ? 16 / sizeof(T) : D / 16;  // elements per lane
+  static constexpr int LPR = D / VE;                                            // lanes per row
+  static constexpr int R = 32 / LPR;                                            // rows per instruction
+  static_assert(R == 1 || R == 2, "layout");
+};
+
 template <typename T, int D, int NL>
 __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a) {
-  constexpr int VE = D / 32;
+  using Lay = RowLayout<T, D>;
+  constexpr int VE = Lay::VE, LPR = Lay::LPR, R = Lay::R;
   const int lane = threadIdx.x & 31;
+  const int lr = lane / LPR, cv = lane % LPR;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int tensor = (int)(wid % 3);
   const int64_t rest = wid / 3;
@@ -166,45 +189,34 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
   const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
   const int log2p = a.log2p;
   const int32_t* so = a.slot_of + bh * a.pyr_entries;
-  const float* xs = a.dxs[tensor] + bh * a.S * D + lane * VE;
-  T* out = static_cast<T*>(a.dx[tensor]) + (bh * a.N + row0) * D + lane * VE;
+  const float* xs = a.dxs[tensor] + bh * a.S * D + cv * VE;
+  T* out = static_cast<T*>(a.dx[tensor]) + (bh * a.N + row0) * D + cv * VE;
 
-  float up[NL + 1][VE];
   float upper[VE];
 #pragma unroll
   for (int i = 0; i < VE; ++i) upper[i] = 0.f;
   int s0w = -1;
-  for (int r = 0; r < rows; ++r) {
-    const int64_t t = row0 + r;
+  for (int r = 0; r < rows; r += R) {
+    const int64_t t = row0 + r;  // first row of this instruction
     if ((r & 31) == 0) s0w = (r + lane < rows) ? so[a.level_off[0] + t + lane] : -1;
     if constexpr (NL > 1) {
       if ((t & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
+        for (int i = 0; i < VE; ++i) upper[i] = 0.f;
+#pragma unroll
         for (int l = 1; l < NL; ++l) {
-          if ((t & ((1ll << (l * log2p)) - 1)) == 0) {
-            const int s = so[a.level_off[l] + (t >> (l * log2p))];
-            if (s >= 0) {
-              float v[VE];
-              load_f32<VE>(xs + (int64_t)s * D, v);
-              const float inv = ldexpf(1.f, -l * log2p);
+          const int s = so[a.level_off[l] + (t >> (l * log2p))];
+          if (s >= 0) {
+            float v[VE];
+            load_f32<VE>(xs + (int64_t)s * D, v);
+            const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
 #pragma unroll
-              for (int i = 0; i < VE; ++i) up[l][i] = v[i] * inv;
-            } else {
-#pragma unroll
-              for (int i = 0; i < VE; ++i) up[l][i] = 0.f;
-            }
+            for (int i = 0; i < VE; ++i) upper[i] = fmaf(v[i], inv, upper[i]);
           }
-        }
-#pragma unroll
-        for (int i = 0; i < VE; ++i) {
-          float s = 0.f;
-#pragma unroll
-          for (int l = NL - 1; l >= 1; --l) s += up[l][i];
-          upper[i] = s;
         }
       }
     }
-    const int s0 = __shfl_sync(kFull, s0w, r & 31);
+    const int s0 = __shfl_sync(kFull, s0w, (r & 31) + lr);
     float y[VE];
 #pragma unroll
     for (int i = 0; i < VE; ++i) y[i] = upper[i];
@@ -214,7 +226,7 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
 #pragma unroll
       for (int i = 0; i < VE; ++i) y[i] += v[i];
     }
-    store_vec<T, VE>(out + (int64_t)r * D, y);
+    if (r + lr < rows) store_vec<T, VE>(out + (int64_t)(r + lr) * D, y);
   }
 }
 
@@ -244,7 +256,7 @@ cudaError_t pool_adj_dispatch_L(int L, const PoolAdjArgs& a, int64_t blocks, cud
 
 int task_rows_for(const Dims& D) {
   const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
-  return (int)(ptop > 32 ? ptop : 32);
+  return (int)(ptop > 64 ? ptop : 64);
 }
 
 }  // namespace
