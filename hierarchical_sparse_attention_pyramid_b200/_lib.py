@@ -49,6 +49,7 @@ SIGNATURES = {
     "lh_plan": [_CFG, POINTER(LhPlanInfo)],
     "lh_pyramid_pool": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_score_topk": [_CFG, _P, _P, _P, _P],
+    "lh_score_topk_static": [_CFG, _P, _P, _P],
     "lh_gather": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_fwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_bwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],

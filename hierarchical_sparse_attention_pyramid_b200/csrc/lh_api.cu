@@ -162,6 +162,9 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
 int* err_word(void* ws) { return static_cast<int*>(ws); }
 
 }  // namespace
+
+lh_status make_dims(const lh_config* cfg, lh_plan_info* info, Dims* D) { return plan_impl(cfg, info, D); }
+
 }  // namespace lh
 
 using namespace lh;

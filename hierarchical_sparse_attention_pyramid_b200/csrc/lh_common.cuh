@@ -123,4 +123,7 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const 
 // message of the last failure on this thread (set by the API layer)
 void set_error_message(const char* fmt, ...);
 
+// validate cfg and fill the plan and the kernel-side shape (lh_plan's checks)
+lh_status make_dims(const lh_config* cfg, lh_plan_info* info, Dims* D);
+
 }  // namespace lh

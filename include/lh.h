@@ -140,6 +140,21 @@ lh_status lh_pyramid_pool(const lh_config *cfg, const void *q, const void *k, co
  *      floor(k'/C) + [c < k' mod C] highest fp32 scores, ties to the lower index. */
 lh_status lh_score_topk(const lh_config *cfg, const float *norms, void *ws, int32_t *sel, lh_stream_t stream);
 
+/* Stage 2 without workspace, for callers that cannot allocate device memory
+ * (a host whose allocator owns every device buffer, a runtime whose memory
+ * plan is fixed, a plugin that only receives its inputs and outputs).  The
+ * pages have no counterpart: this is lh_score_topk with its score pyramid
+ * kept in a file-scope device array of 16 MiB (B*H * upper_entries * 4 bytes
+ * at most; larger configurations return LH_ERR_UNSUPPORTED) that every GPU
+ * loading the library holds until exit.  It calls no allocator.
+ * In:  norms as for lh_score_topk.  Out: sel as for lh_score_topk.
+ * The first call on a device looks up the array's device address (with
+ * cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller.  The
+ * array keeps the last call's contents; every call rewrites all it reads. */
+lh_status lh_score_topk_static(const lh_config *cfg, const float *norms, int32_t *sel, lh_stream_t stream);
+
 /* Stage 3 - gather the kept entries into one causally ordered sequence.
  * Cite: LH-post "How it works" (3) (kept entries sorted into causal order
  * form a contiguous sequence of length S); LH-summary "Technical details" (3).
