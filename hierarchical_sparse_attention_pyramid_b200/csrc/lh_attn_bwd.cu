@@ -5,17 +5,21 @@
 // With P = softmax(Qs Ks^T / sqrt(d)) (causal) recomputed from the saved LSE,
 //   dVs = P^T dOs,  dP = dOs Vs^T,  dS = P * (dP - Delta) / sqrt(d),
 //   dQs = dS Ks,    dKs = dS^T Qs,  Delta = rowsum(dOs * Os).
+// P^T and dS^T enter their products as bf16 (hi + lo) pairs, so the bf16
+// roundings of the probabilities and of dS do not show in the gradients.
 //
 // One CTA owns a 128-row key/value tile of one (batch, head) and walks the
 // query tiles from the diagonal to the end.  Warp roles:
-//   warps 0-3  thread t owns key row t for S^T/dP^T (TMEM lane t): writes
-//              P^T, then dS^T, to shared memory as bf16 hi + lo pairs (so the
-//              products keep fp32-level accuracy), then reads dQ row t of the
-//              query tile from TMEM and adds it to dQs with fp32 vector
-//              atomics; at the end writes dKs and dVs rows
-//   warp 4     TMA producer: K, V once; Q and dO per query tile
-//   warp 5     MMA issuer (one thread) and TMEM owner
-// TMEM columns: S^T [0,128), dP^T / dQ [128,256), dV [256,256+D), dK [256+D,256+2D).
+//   warps 0-7  two compute warpgroups; thread (g, t) owns key row t (TMEM lane
+//              t) and query columns [64g, 64g+64) of the tile.  One pass turns
+//              S^T and dP^T into P^T (hi/lo, written back into the S^T
+//              columns of TMEM, where the dV product reads it as its A
+//              operand) and dS^T (hi/lo, to shared memory); then each reads
+//              half of the tile's dQ from TMEM and adds it to dQs with fp32
+//              vector atomics; at the end they write dKs and dVs
+//   warp 8     TMA producer: K, V once; Q and dO per query tile
+//   warp 9     MMA issuer (one thread) and TMEM owner
+// TMEM columns: S^T/P^T [0,128), dP^T/dQ [128,256), dV [256,256+D), dK [256+D,256+2D).
 #include <math.h>
 
 #include "lh_common.cuh"
@@ -30,7 +34,8 @@ using namespace sm100;
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // key rows per CTA
-constexpr int kThreads = 192;
+constexpr int kCompute = 256;
+constexpr int kThreads = kCompute + 64;
 
 template <int D>
 struct BwdSmem {
@@ -39,16 +44,16 @@ struct BwdSmem {
   static constexpr int oK = 0;
   static constexpr int oV = oK + kTile;
   static constexpr int oQ = oV + kTile;
-  static constexpr int oO = oQ + kTile;  // dO
-  static constexpr int oHi = oO + kTile;        // P^T, then dS^T: bf16 high part
-  static constexpr int oLo = oHi + 2 * kChunk;  // bf16 of the remainder
+  static constexpr int oO = oQ + kTile;          // dO
+  static constexpr int oHi = oO + kTile;         // dS^T, bf16 high part
+  static constexpr int oLo = oHi + 2 * kChunk;   // bf16 of the remainder
   static constexpr int oVec = oLo + 2 * kChunk;  // LSE*log2e [128], Delta [128]
   static constexpr int oBar = oVec + 1024;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-__device__ __forceinline__ void wg_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -61,18 +66,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
-  uint64_t* bKV = bars + 0;     // K, V landed
-  uint64_t* bQO = bars + 1;     // Q_i, dO_i landed
-  uint64_t* bSdP = bars + 2;    // S^T and dP^T in TMEM
-  uint64_t* bP = bars + 3;      // P^T hi/lo in shared memory (128 arrivals)
-  uint64_t* bMM = bars + 4;     // dK, dQ MMAs of the tile done
-  uint64_t* bDQfree = bars + 5; // dQ read out of TMEM (128 arrivals)
-  uint64_t* bPfree = bars + 6;  // dV MMAs done: the hi/lo buffers may take dS^T
-  uint64_t* bDS = bars + 7;     // dS^T hi/lo in shared memory (128 arrivals)
+  uint64_t* bKV = bars + 0;      // K, V landed
+  uint64_t* bQO = bars + 1;      // Q_i, dO_i landed
+  uint64_t* bQOfree = bars + 2;  // dV, dK products of tile i done: Q, dO buffers free
+  uint64_t* bSdP = bars + 3;     // S^T and dP^T of tile i in TMEM
+  uint64_t* bPS = bars + 4;      // P^T in TMEM and dS^T in shared memory (256 arrivals)
+  uint64_t* bDQ = bars + 5;      // dQ of tile i in TMEM (all products of tile i done)
+  uint64_t* bDQfree = bars + 6;  // dQ read out of TMEM (256 arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
-  float* sLSE = reinterpret_cast<float*>(smem + Lay::oVec);
-  float* sDel = sLSE + 128;
+  float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);  // [0,128) LSE*log2e, [128,256) Delta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
@@ -83,23 +86,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bKV, 1);
     mbar_init(bQO, 1);
+    mbar_init(bQOfree, 1);
     mbar_init(bSdP, 1);
-    mbar_init(bP, 128);
-    mbar_init(bMM, 1);
-    mbar_init(bDQfree, 128);
-    mbar_init(bPfree, 1);
-    mbar_init(bDS, 128);
+    mbar_init(bPS, kCompute);
+    mbar_init(bDQ, 1);
+    mbar_init(bDQfree, kCompute);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmO);
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int it = 0; it < n_q; ++it) {
         const int i = kt + it;
-        if (it >= 1 && !mbar_wait(bMM, (it - 1) & 1, abort_flag)) break;
+        if (it >= 1 && !mbar_wait(bQOfree, (it - 1) & 1, abort_flag)) break;
         mbar_expect_tx(bQO, 2 * BM * D * 2);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_3d(smem + Lay::oQ + c * Lay::kChunk, &tmQ, bQO, c * 64, i * BM, bh);
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idKM = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
@@ -130,14 +134,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; ok && it < n_q; ++it) {
         if (!mbar_wait(bQO, it & 1, abort_flag)) break;
         tc_fence_after();
-        // S^T = K Q^T  (M = keys, N = queries, K = d)
+        // S^T = K Q^T  (M = keys, N = queries, K = d); the S^T columns held P^T of
+        // the previous tile, whose dV product was issued before this one
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
           umma_bf16(tmem + tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idSS,
                     kk > 0 ? 1u : 0u);
         }
-        // dP^T = V dO^T into the dQ region, once the previous dQ has been read out
+        // dP^T = V dO^T into the dQ columns, once the previous dQ has been read out
         if (it >= 1 && !mbar_wait(bDQfree, (it - 1) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
@@ -147,20 +152,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     kk > 0 ? 1u : 0u);
         }
         umma_commit(bSdP);
-        if (!mbar_wait(bP, it & 1, abort_flag)) break;
+        if (!mbar_wait(bPS, it & 1, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO   (M = keys, K = queries, N = d), P^T = hi + lo
+        // dV += P^T dO: A = P^T (hi, lo) from TMEM, B = dO MN-major (K = queries)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
+          const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint64_t b = sdesc_sw128(sO + kk * 2048, Lay::kChunk, 1024);
-          umma_bf16(tmem + tDV, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + tDV, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
+          umma_bf16_tmem_a(tmem + tDV, a, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + tDV, a + 16, b, idKM, 1u);
         }
-        umma_commit(bPfree);
-        if (!mbar_wait(bDS, it & 1, abort_flag)) break;
-        tc_fence_after();
-        // dK += dS^T Q   (M = keys, K = queries, N = d), dS^T = hi + lo
+        // dK += dS^T Q: A = dS^T (hi, lo) K-major from shared memory
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + tDK, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
           umma_bf16(tmem + tDK, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
         }
+        umma_commit(bQOfree);
         // dQ = dS K  (M = queries, K = keys, N = d): dS^T read M-major
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -176,98 +179,92 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + tDP, sdesc_sw128(sHi + off, Lay::kChunk, 1024), b, idMM, kk > 0 ? 1u : 0u);
           umma_bf16(tmem + tDP, sdesc_sw128(sLo + off, Lay::kChunk, 1024), b, idMM, 1u);
         }
-        umma_commit(bMM);
+        umma_commit(bDQ);
       }
     }
   } else {
-    // ------------------------------------------------------------ compute warpgroup
-    const int t = threadIdx.x;  // 0..127
+    // ------------------------------------------------------------ compute warpgroups
+    const int ct = threadIdx.x;            // 0..255
+    const int g = warp >> 2;               // warpgroup: query columns [64g, 64g+64)
+    const int t = (warp & 3) * 32 + lane;  // key row of the tile (TMEM lane)
     const int kv_g = kt * BN + t;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint8_t* sHib = smem + Lay::oHi;
     uint8_t* sLob = smem + Lay::oLo;
     bool ok = true;
-    // write 32 consecutive query columns (chunk c) of this key row as bf16 hi + lo
-    auto put_row_chunk = [&](int c, const float (&x)[32]) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = x[8 * q + 2 * e], b = x[8 * q + 2 * e + 1];
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[e] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
-        }
-        const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 128-byte row
-        const int off = (c >> 1) * Lay::kChunk + t * 128 + ((ch ^ (t & 7)) << 4);
-        *reinterpret_cast<uint4*>(sHib + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sLob + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
+    // LSE (ct < 128) or Delta (ct >= 128) of one query row of the tile at q0
+    auto vec_of = [&](int q0) -> float {
+      const int qg = q0 + (ct & 127);
+      if (ct < 128) return qg < S ? LSE[(int64_t)bh * S + qg] * 1.4426950408889634f : INFINITY;
+      return qg < S ? Delta[(int64_t)bh * S + qg] : 0.f;
     };
+    float vec_next = vec_of(kt * BM);
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (kt + it) * BM;
-      wg_sync();  // every thread is done with the previous tile's LSE / Delta
-      {
-        const int qg = q0 + t;
-        sLSE[t] = qg < S ? LSE[(int64_t)bh * S + qg] * 1.4426950408889634f : INFINITY;
-        sDel[t] = qg < S ? Delta[(int64_t)bh * S + qg] : 0.f;
-      }
-      wg_sync();
+      const float vec_cur = vec_next;
+      if (it + 1 < n_q) vec_next = vec_of(q0 + BM);  // one tile ahead
+      compute_sync();  // every thread is done with the previous tile's LSE / Delta
+      sVec[ct] = vec_cur;
+      compute_sync();
       if (!mbar_wait(bSdP, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      // pass 1: P^T
+      const bool diag = (it == 0);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(tl + tS + c * 32, sr);
-        tmem_ld_wait();
-        float pv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int qi = c * 32 + e;
-          pv[e] = (q0 + qi) >= kv_g ? exp2f(__uint_as_float(sr[e]) * scale_log2 - sLSE[qi]) : 0.f;
-        }
-        put_row_chunk(c, pv);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bP);
-      // pass 2: dS^T, once the dV MMAs have read P^T
-      if (!mbar_wait(bPfree, it & 1, abort_flag)) { ok = false; break; }
-      __syncwarp();
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * g + cc;  // 32-column chunk of the tile
         uint32_t sr[32], dr[32];
         tmem_ld32(tl + tS + c * 32, sr);
         tmem_ld32(tl + tDP + c * 32, dr);
         tmem_ld_wait();
-        float dv[32];
+        uint32_t phi[16], plo[16], dhi[16], dlo[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int qi = c * 32 + e;
-          const float p = (q0 + qi) >= kv_g ? exp2f(__uint_as_float(sr[e]) * scale_log2 - sLSE[qi]) : 0.f;
-          dv[e] = p * (__uint_as_float(dr[e]) - sDel[qi]) * scale;
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int qi = c * 32 + e + h;
+            float p = fast_exp2(__uint_as_float(sr[e + h]) * scale_log2 - sVec[qi]);
+            if (diag && q0 + qi < kv_g) p = 0.f;
+            pv[h] = p;
+            dv[h] = p * (__uint_as_float(dr[e + h]) - sVec[128 + qi]) * scale;
+          }
+          const __nv_bfloat162 ph = __floats2bfloat162_rn(pv[0], pv[1]);
+          const __nv_bfloat162 dh = __floats2bfloat162_rn(dv[0], dv[1]);
+          phi[e >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
+          dhi[e >> 1] = *reinterpret_cast<const uint32_t*>(&dh);
+          plo[e >> 1] = pack_bf16x2(pv[0] - __low2float(ph), pv[1] - __high2float(ph));
+          dlo[e >> 1] = pack_bf16x2(dv[0] - __low2float(dh), dv[1] - __high2float(dh));
         }
-        put_row_chunk(c, dv);
+        // P^T over the S^T columns just read: hi in the first 16, lo in the last 16
+        tmem_st16(tl + tS + c * 32, phi);
+        tmem_st16(tl + tS + c * 32 + 16, plo);
+        // dS^T row t, query columns c*32..c*32+31: 4 chunks of 16 bytes in region c/2
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int ch = (c & 1) * 4 + q;
+          const int off = (c >> 1) * Lay::kChunk + t * 128 + ((ch ^ (t & 7)) << 4);
+          *reinterpret_cast<uint4*>(sHib + off) = make_uint4(dhi[4 * q], dhi[4 * q + 1], dhi[4 * q + 2], dhi[4 * q + 3]);
+          *reinterpret_cast<uint4*>(sLob + off) = make_uint4(dlo[4 * q], dlo[4 * q + 1], dlo[4 * q + 2], dlo[4 * q + 3]);
+        }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bDS);
-      // dQ of query row q0 + t
-      if (!mbar_wait(bMM, it & 1, abort_flag)) { ok = false; break; }
+      mbar_arrive(bPS);
+      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1))
+      if (!mbar_wait(bDQ, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
       const int qg = q0 + t;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = g * (D / 2) + c * 32;
         uint32_t r[32];
-        tmem_ld32(tl + tDP + c * 32, r);
+        tmem_ld32(tl + tDP + col, r);
         tmem_ld_wait();
         if (qg < S) {
-          float4* dst = reinterpret_cast<float4*>(dQ + ((int64_t)bh * S + qg) * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(dQ + ((int64_t)bh * S + qg) * D + col);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             atomicAdd(dst + q, make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
@@ -278,18 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bDQfree);
     }
     if (ok && !*abort_flag) {
-      // bMM of the last tile has completed: dV and dK are final
+      // bDQ of the last tile has completed: dV and dK are final
       __syncwarp();
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = g * (D / 2) + c * 32;
         uint32_t rv[32], rk[32];
-        tmem_ld32(tl + tDV + c * 32, rv);
-        tmem_ld32(tl + tDK + c * 32, rk);
+        tmem_ld32(tl + tDV + col, rv);
+        tmem_ld32(tl + tDK + col, rk);
         tmem_ld_wait();
         if (kv_g < S) {
-          float4* dv4 = reinterpret_cast<float4*>(dV + ((int64_t)bh * S + kv_g) * D + c * 32);
-          float4* dk4 = reinterpret_cast<float4*>(dK + ((int64_t)bh * S + kv_g) * D + c * 32);
+          float4* dv4 = reinterpret_cast<float4*>(dV + ((int64_t)bh * S + kv_g) * D + col);
+          float4* dk4 = reinterpret_cast<float4*>(dK + ((int64_t)bh * S + kv_g) * D + col);
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             dv4[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
@@ -303,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

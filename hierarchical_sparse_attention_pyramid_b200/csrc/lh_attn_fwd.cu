@@ -2,16 +2,21 @@
 // sequence (aitrends.kr summary of Lighthouse Attention, Technical details
 // (3): the kept Q/K/V form S tokens and an unmodified attention runs on them).
 //
-// One CTA owns a 128-row query tile of one (batch, head) and walks the key
-// tiles 0..qt (causal; the diagonal tile is masked).  Warp roles:
-//   warps 0-3  softmax: thread t owns query row t (TMEM lane t); reads S from
-//              TMEM, keeps the running max / sum, writes P (bf16) to shared
-//              memory in the 128-byte-swizzled K-major layout, rescales O in
-//              TMEM when the max moves, and writes O / LSE at the end
-//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring
-//   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM
-//              buffers, O += P V into a third; owns the TMEM allocation
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
+// One CTA owns two 128-row query tiles (A = 2c, B = 2c+1) of one (batch,
+// head) and streams the key/value tiles 0..2c+1 once for both (causal; each
+// tile's diagonal block is masked).  Warp roles:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t owns
+//              query row t (TMEM lane t); reads S from TMEM twice (row max,
+//              then exponentials), keeps the running max / sum, rescales O in
+//              TMEM when the max moves, and writes P back over the S columns
+//              it came from as a bf16 pair (per 32 keys: 16 columns of hi,
+//              16 of lo), where the P V product reads it
+//   warp 8     TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
+//   warp 9     MMA issuer (one thread): for each key tile, P_A V, then the next
+//              S_A = Q_A K^T, then P_B V and the next S_B, so the tensor core
+//              works on one tile while the other tile's softmax runs
+// TMEM columns: S_A/P_A [0,128), S_B/P_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
+// The P pair keeps P V at fp32 accuracy; O is written in fp32.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -23,18 +28,17 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kThreads = 192;
+constexpr int kSoftmax = 256;
+constexpr int kThreads = kSoftmax + 64;
 
 template <int D>
 struct FwdSmem {
   static constexpr int kChunk = 128 * 128;  // [128 rows][64 bf16] region
   static constexpr int kTile = D / 64 * kChunk;
-  static constexpr int oQ = 0;
-  static constexpr int oK = oQ + kTile;
-  static constexpr int oV = oK + 2 * kTile;
-  static constexpr int oP = oV + 2 * kTile;     // P_hi: bf16(P)
-  static constexpr int oPl = oP + 2 * kChunk;   // P_lo: bf16(P - P_hi)
-  static constexpr int oBar = oPl + 2 * kChunk;
+  static constexpr int oQ = 0;              // Q_A, Q_B
+  static constexpr int oK = oQ + 2 * kTile; // 2 stages
+  static constexpr int oV = oK + 2 * kTile; // 2 stages
+  static constexpr int oBar = oV + 2 * kTile;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -49,21 +53,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bQ = bars + 0;
-  uint64_t* bK = bars + 1;       // [2]
+  uint64_t* bK = bars + 1;       // [2] stages
   uint64_t* bV = bars + 3;       // [2]
   uint64_t* bKVfree = bars + 5;  // [2]
-  uint64_t* bS = bars + 7;       // [2]
-  uint64_t* bSfree = bars + 9;   // [2]
-  uint64_t* bP = bars + 11;
-  uint64_t* bO = bars + 12;
+  uint64_t* bS = bars + 7;       // [2] tiles: S of the tile in TMEM (and its previous P V done)
+  uint64_t* bP = bars + 9;       // [2] tiles: P in TMEM, O rescaled (128 arrivals)
+  uint64_t* bO = bars + 11;      // [2] tiles: a P V product of the tile done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
-  const int qt = n_qt - 1 - (int)blockIdx.x;  // longest rows first
+  const int n_pairs = (n_qt + 1) / 2;
+  const int c = n_pairs - 1 - (int)blockIdx.x;  // longest rows first
   const int bh = (int)blockIdx.y;
-  const int n_kv = qt + 1;
+  const int qtile[2] = {2 * c, 2 * c + 1};
+  const bool hasB = qtile[1] < n_qt;
+  const int last[2] = {qtile[0], hasB ? qtile[1] : -1};  // last key tile of each query tile
+  const int n_kv = (hasB ? qtile[1] : qtile[0]) + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(bQ, 1);
@@ -72,170 +79,177 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bV[s], 1);
       mbar_init(&bKVfree[s], 1);
       mbar_init(&bS[s], 1);
-      mbar_init(&bSfree[s], 128);
+      mbar_init(&bP[s], 128);
+      mbar_init(&bO[s], 1);
     }
-    mbar_init(bP, 128);
-    mbar_init(bO, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(bQ, BM * D * 2);
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(smem + Lay::oQ + c * Lay::kChunk, &tmQ, bQ, c * 64, qt * BM, bh);
+      mbar_expect_tx(bQ, (hasB ? 2 : 1) * BM * D * 2);
+      for (int x = 0; x < (hasB ? 2 : 1); ++x)
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(smem + Lay::oQ + x * Lay::kTile + ch * Lay::kChunk, &tmQ, bQ, ch * 64, qtile[x] * BM, bh);
       for (int j = 0; j < n_kv; ++j) {
         const int st = j & 1, use = j >> 1;
         if (j >= 2 && !mbar_wait(&bKVfree[st], (use - 1) & 1, abort_flag)) break;
         mbar_expect_tx(&bK[st], BN * D * 2);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oK + st * Lay::kTile + c * Lay::kChunk, &tmK, &bK[st], c * 64, j * BN, bh);
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(smem + Lay::oK + st * Lay::kTile + ch * Lay::kChunk, &tmK, &bK[st], ch * 64, j * BN, bh);
         mbar_expect_tx(&bV[st], BN * D * 2);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oV + st * Lay::kTile + c * Lay::kChunk, &tmV, &bV[st], c * 64, j * BN, bh);
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(smem + Lay::oV + st * Lay::kTile + ch * Lay::kChunk, &tmV, &bV[st], ch * 64, j * BN, bh);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idQK = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idPV = idesc_bf16(BM, D, false, true);
-      const uint32_t sQ = smem_u32(smem + Lay::oQ), sK = smem_u32(smem + Lay::oK);
-      const uint32_t sV = smem_u32(smem + Lay::oV), sP = smem_u32(smem + Lay::oP);
-      const uint32_t sPl = smem_u32(smem + Lay::oPl);
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj & 1;
-        if (!mbar_wait(bP, jj & 1, abort_flag)) return false;
-        if (!mbar_wait(&bV[st], (jj >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vb = sV + st * Lay::kTile;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          const uint64_t b = sdesc_sw128(vb + kk * 2048, Lay::kChunk, 1024);
-          umma_bf16(tmem + 256, sdesc_sw128(sP + aoff, 16, 1024), b, idPV, (jj > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + 256, sdesc_sw128(sPl + aoff, 16, 1024), b, idPV, 1u);
-        }
-        umma_commit(bO);
-        umma_commit(&bKVfree[st]);
-        return true;
-      };
-      bool ok = mbar_wait(bQ, 0, abort_flag);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j & 1, use = j >> 1;
-        if (!mbar_wait(&bK[st], use & 1, abort_flag)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&bSfree[st], (use - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sK + st * Lay::kTile;
+      const uint32_t sQ = smem_u32(smem + Lay::oQ), sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
+      auto issue_s = [&](int x, int j) {
+        const uint32_t qb = sQ + x * Lay::kTile, kb = sK + (j & 1) * Lay::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * Lay::kChunk + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(kb + (kk >> 2) * Lay::kChunk + (kk & 3) * 32, 16, 1024);
-          umma_bf16(tmem + st * 128, a, b, idQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
+          umma_bf16(tmem + x * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idQK,
+                    kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bS[st]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        umma_commit(&bS[x]);
+      };
+      bool ok = mbar_wait(bQ, 0, abort_flag) && mbar_wait(&bK[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (hasB) issue_s(1, 0);
       }
-      if (ok) issue_pv(n_kv - 1);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int st = j & 1;
+        bool v_ready = false, k_next_ready = false;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j > last[x]) continue;
+          if (!mbar_wait(&bP[x], j & 1, abort_flag)) { ok = false; break; }
+          if (!v_ready) {
+            if (!mbar_wait(&bV[st], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            v_ready = true;
+          }
+          tc_fence_after();
+          const uint32_t vb = sV + st * Lay::kTile;
+          const uint32_t pa = tmem + x * 128;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t b = sdesc_sw128(vb + kk * 2048, Lay::kChunk, 1024);
+            const uint32_t a = pa + (kk >> 1) * 32 + (kk & 1) * 8;  // hi of keys 16kk..16kk+15
+            umma_bf16_tmem_a(tmem + 256 + x * D, a, b, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_tmem_a(tmem + 256 + x * D, a + 16, b, idPV, 1u);
+          }
+          umma_commit(&bO[x]);
+          if (j + 1 <= last[x]) {
+            if (!k_next_ready) {
+              if (!mbar_wait(&bK[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+              k_next_ready = true;
+              tc_fence_after();
+            }
+            issue_s(x, j + 1);  // after P V of this tile: the S columns hold P until then
+          }
+        }
+        if (ok) umma_commit(&bKVfree[st]);
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int row = threadIdx.x;  // 0..127
-    const int row_g = qt * BM + row;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* sPb = smem + Lay::oP;
-    uint8_t* sPlb = smem + Lay::oPl;
+    const int x = warp >> 2;               // query tile of this warpgroup
+    const int row = (warp & 3) * 32 + lane;
+    const int row_g = qtile[x] * BM + row;
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t ts = tl + x * 128, to = tl + 256 + x * D;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&bS[st], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+    bool ok = last[x] >= 0;
+    for (int j = 0; ok && j <= last[x]; ++j) {
+      if (!mbar_wait(&bS[x], j & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tl + st * 128 + c * 32, r[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bSfree[st]);
-      float s[128];
+      const bool diag = (j == last[x]);
+      // pass 1: row max of the raw scores (the scale is positive)
       float mx = -INFINITY;
-      const bool diag = (j == n_kv - 1);
-      const int lim = row_g - j * BN;  // columns c > lim are in the future
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(ts + ch * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = __uint_as_float(r[c >> 5][c & 31]) * scale_log2;
-        if (diag && c > lim) v = -INFINITY;
-        s[c] = v;
-        mx = fmaxf(mx, v);
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = exp2f(m_run - m_new);
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        s[c] = exp2f(s[c] - m_new);
-        rs += s[c];
-      }
-      if (j >= 1) {
-        // PV of the previous tile must be done: O is stable and the P buffers free
-        if (!mbar_wait(bO, (j - 1) & 1, abort_flag)) { ok = false; break; }
-        __syncwarp();
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tl + 256 + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + 256 + c * 32, o);
-          }
-          tmem_st_wait();
+        for (int i = 0; i < 32; ++i) {
+          const int col = ch * 32 + i;
+          if (!(diag && col > row)) mx = fmaxf(mx, __uint_as_float(r[i]));  // later keys are masked
         }
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      // P = P_hi + P_lo, both bf16, so that P V keeps fp32-level accuracy
+      const float m_new = fmaxf(m_run, mx * scale_log2);
+      const float alpha = fast_exp2(m_run - m_new);
+      // the previous P V of this tile is done (its completion preceded this S)
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(to + ch * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t hi[4], lo[4];
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(to + ch * 32, o);
+        }
+      }
+      // pass 2: P = exp2(s - m) as a bf16 pair written back over the chunk it
+      // came from: chunk ch (keys 32ch..32ch+31) holds hi in its first 16
+      // columns and lo in its last 16
+      float rs = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(ts + ch * 32, r);
+        tmem_ld_wait();
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = s[8 * ch + 2 * q], b = s[8 * ch + 2 * q + 1];
+        for (int q = 0; q < 16; ++q) {
+          const int col = ch * 32 + 2 * q;
+          float a = fast_exp2(fmaf(__uint_as_float(r[2 * q]), scale_log2, -m_new));
+          float b = fast_exp2(fmaf(__uint_as_float(r[2 * q + 1]), scale_log2, -m_new));
+          if (diag && col > row) a = 0.f;
+          if (diag && col + 1 > row) b = 0.f;
+          rs += a + b;
           const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
           hi[q] = *reinterpret_cast<const uint32_t*>(&h);
           lo[q] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
         }
-        const int off = (ch >> 3) * Lay::kChunk + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(sPb + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sPlb + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        tmem_st16(ts + ch * 32, hi);
+        tmem_st16(ts + ch * 32 + 16, lo);
       }
-      fence_proxy_async_smem();
+      l_run = l_run * alpha + rs;
+      m_run = m_new;
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bP);
+      mbar_arrive(&bP[x]);
     }
-    if (ok && mbar_wait(bO, (n_kv - 1) & 1, abort_flag)) {
+    if (ok && mbar_wait(&bO[x], last[x] & 1, abort_flag)) {
       __syncwarp();
       tc_fence_after();
       const float inv_l = 1.f / l_run;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
-        tmem_ld32(tl + 256 + c * 32, o);
+        tmem_ld32(to + ch * 32, o);
         tmem_ld_wait();
         if (row_g < S) {
-          float4* dst = reinterpret_cast<float4*>(O + ((int64_t)bh * S + row_g) * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(O + ((int64_t)bh * S + row_g) * D + ch * 32);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
@@ -247,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -288,19 +302,18 @@ cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const 
       !make_seq_map(&mv, vs, BH, S, d, BN))
     return cudaErrorInvalidValue;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-  const dim3 grid((unsigned)((S + BM - 1) / BM), (unsigned)BH);
+  const int64_t n_qt = (S + BM - 1) / BM;
+  const dim3 grid((unsigned)((n_qt + 1) / 2), (unsigned)BH);
   if (d == 128) {
     const int smem = FwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw,
-                                                        (int)S, scale_log2);
+    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2);
   } else {
     const int smem = FwdSmem<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw,
-                                                       (int)S, scale_log2);
+    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2);
   }
   return cudaGetLastError();
 }
