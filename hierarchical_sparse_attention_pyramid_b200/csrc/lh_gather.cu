@@ -131,6 +131,10 @@ struct RowLayout {
   static_assert(R == 1 || R == 2, "layout");
 };
 
+// Rows are visited in instruction steps u = 0, R, 2R, ...; step u covers rows
+// u - (R-1) .. u.  With R = 2 the pair (u-1, u) has (j+1) in {u, u+1}, u even,
+// so both rows take the same entry at every level >= 1 and the refresh of the
+// cached contribution is uniform over the warp.
 template <typename T, int D, int NL>
 __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a) {
   using Lay = RowLayout<T, D>;
@@ -140,31 +144,36 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t bh = wid / a.tasks_per_head;
   if (bh >= a.BH) return;
-  const int64_t row0 = (wid % a.tasks_per_head) * a.task_rows;
-  const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
+  const int64_t u0 = (wid % a.tasks_per_head) * a.task_rows;
+  const int steps = (int)min((int64_t)a.task_rows, a.N + R - 1 - u0);
   const int log2p = a.log2p;
   const int32_t* so = a.slot_of + bh * a.pyr_entries;
   const float* os = a.os + bh * a.S * D + cv * VE;
-  T* out = static_cast<T*>(a.y) + (bh * a.N + row0) * D + cv * VE;
+  T* out = static_cast<T*>(a.y) + bh * a.N * D + cv * VE;
 
   float upper[VE];
 #pragma unroll
   for (int c = 0; c < VE; ++c) upper[c] = 0.f;
-  int64_t cur1 = -2;  // level-1 entry of this lane's previous row
+  int64_t cur1 = -2;  // level-1 entry of the previous step
   int s0w = -1;
-  for (int r = 0; r < rows; r += R) {
-    const int64_t j = row0 + r + lr;  // this lane's row
-    if ((r & 31) == 0) s0w = (r + lane < rows) ? so[a.level_off[0] + row0 + r + lane] : -1;
+  for (int r = 0; r < steps; r += R) {
+    const int64_t u = u0 + r;
+    const int64_t j = u - (R - 1) + lr;  // this lane's row
+    if ((r & 31) == 0) {
+      const int64_t jw = u - (R - 1) + lane;
+      s0w = (jw >= 0 && jw < a.N && r + lane < steps) ? so[a.level_off[0] + jw] : -1;
+    }
     if constexpr (NL > 1) {
-      const int64_t i1 = ((j + 1) >> log2p) - 1;
+      const int64_t key = (R == 2) ? u : u + 1;  // (j+1) rounded down to the step, same for both rows
+      const int64_t i1 = (key >> log2p) - 1;
       if (i1 != cur1) {
         cur1 = i1;
 #pragma unroll
         for (int c = 0; c < VE; ++c) upper[c] = 0.f;
 #pragma unroll
         for (int l = 1; l < NL; ++l) {
-          const int64_t i = ((j + 1) >> (l * log2p)) - 1;
-          const int s = (i >= 0 && j < a.N) ? so[a.level_off[l] + i] : -1;
+          const int64_t i = (key >> (l * log2p)) - 1;
+          const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
           if (s >= 0) {
             float v[VE];
             load_f32<VE>(os + (int64_t)s * D, v);
@@ -184,7 +193,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 #pragma unroll
       for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
     }
-    if (r + lr < rows) store_vec<T, VE>(out + (int64_t)(r + lr) * D, y);
+    if (j >= 0 && j < a.N) store_vec<T, VE>(out + j * D, y);
   }
 }
 
@@ -329,7 +338,7 @@ cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* s
   for (int l = 0; l < LH_MAX_LEVELS; ++l) a.level_off[l] = D.level_off[l];
   const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
   a.task_rows = (int)(ptop > 64 ? ptop : 64);
-  a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
+  a.tasks_per_head = (D.N + 1 + a.task_rows - 1) / a.task_rows;  // steps cover rows -1 .. N-1
   a.log2p = D.log2p;
   const int64_t blocks = (D.BH * a.tasks_per_head + kWarps - 1) / kWarps;
   if (D.dtype == LH_BF16) {
