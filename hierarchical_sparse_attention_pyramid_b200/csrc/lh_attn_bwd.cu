@@ -16,8 +16,9 @@
 //              columns of TMEM, where the dV product reads it as its A
 //              operand) and dS^T (hi/lo, to shared memory); then each reads
 //              half of the tile's dQ from TMEM and adds it to dQs with fp32
-//              vector atomics; at the end they write dKs and dVs
-//   warp 8     TMA producer: K, V once; Q and dO per query tile
+//              vector reductions at the L2; at the end they write dKs and dVs
+//   warp 8     TMA producer: K, V once; Q and dO per query tile, each as
+//              soon as the product that last reads it (dK, dV) is done
 //   warp 9     MMA issuer (one thread) and TMEM owner
 // TMEM columns: S^T/P^T [0,128), dP^T/dQ [128,256), dV [256,256+D), dK [256+D,256+2D).
 #include <math.h>
@@ -67,8 +68,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bKV = bars + 0;      // K, V landed
-  uint64_t* bQO = bars + 1;      // Q_i, dO_i landed
-  uint64_t* bQOfree = bars + 2;  // dV, dK products of tile i done: Q, dO buffers free
+  uint64_t* bQ = bars + 1;       // Q_i landed
+  uint64_t* bQfree = bars + 2;   // dK product of tile i done: Q buffer free
+  uint64_t* bO = bars + 7;       // dO_i landed
+  uint64_t* bOfree = bars + 8;   // dV product of tile i done: dO buffer free
   uint64_t* bSdP = bars + 3;     // S^T and dP^T of tile i in TMEM
   uint64_t* bPS = bars + 4;      // P^T in TMEM and dS^T in shared memory (256 arrivals)
   uint64_t* bDQ = bars + 5;      // dQ of tile i in TMEM (all products of tile i done)
@@ -85,8 +88,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bKV, 1);
-    mbar_init(bQO, 1);
-    mbar_init(bQOfree, 1);
+    mbar_init(bQ, 1);
+    mbar_init(bQfree, 1);
+    mbar_init(bO, 1);
+    mbar_init(bOfree, 1);
     mbar_init(bSdP, 1);
     mbar_init(bPS, kCompute);
     mbar_init(bDQ, 1);
@@ -111,14 +116,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(smem + Lay::oK + c * Lay::kChunk, &tmK, bKV, c * 64, kt * BN, bh);
         tma_load_3d(smem + Lay::oV + c * Lay::kChunk, &tmV, bKV, c * 64, kt * BN, bh);
       }
+      // Q is released by the dK product and dO by the dV product of the
+      // previous tile; each reloads as soon as its buffer is free
       for (int it = 0; it < n_q; ++it) {
         const int i = kt + it;
-        if (it >= 1 && !mbar_wait(bQOfree, (it - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bQO, 2 * BM * D * 2);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + Lay::oQ + c * Lay::kChunk, &tmQ, bQO, c * 64, i * BM, bh);
-          tma_load_3d(smem + Lay::oO + c * Lay::kChunk, &tmO, bQO, c * 64, i * BM, bh);
-        }
+        if (it >= 1 && !mbar_wait(bQfree, (it - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bQ, BM * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oQ + c * Lay::kChunk, &tmQ, bQ, c * 64, i * BM, bh);
+        if (it >= 1 && !mbar_wait(bOfree, (it - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(bO, BM * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oO + c * Lay::kChunk, &tmO, bO, c * 64, i * BM, bh);
       }
     }
   } else if (warp == 9) {
@@ -132,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sHi = smem_u32(smem + Lay::oHi), sLo = smem_u32(smem + Lay::oLo);
       bool ok = mbar_wait(bKV, 0, abort_flag);
       for (int it = 0; ok && it < n_q; ++it) {
-        if (!mbar_wait(bQO, it & 1, abort_flag)) break;
+        if (!mbar_wait(bQ, it & 1, abort_flag)) break;
         tc_fence_after();
         // S^T = K Q^T  (M = keys, N = queries, K = d); the S^T columns held P^T of
         // the previous tile, whose dV product was issued before this one
@@ -142,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idSS,
                     kk > 0 ? 1u : 0u);
         }
-        // dP^T = V dO^T into the dQ columns, once the previous dQ has been read out
+        // dP^T = V dO^T into the dQ columns, once dO has landed and the previous
+        // dQ has been read out
+        if (!mbar_wait(bO, it & 1, abort_flag)) break;
         if (it >= 1 && !mbar_wait(bDQfree, (it - 1) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
@@ -154,15 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(bSdP);
         if (!mbar_wait(bPS, it & 1, abort_flag)) break;
         tc_fence_after();
-        // dV += P^T dO: A = P^T (hi, lo) from TMEM, B = dO MN-major (K = queries)
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint64_t b = sdesc_sw128(sO + kk * 2048, Lay::kChunk, 1024);
-          umma_bf16_tmem_a(tmem + tDV, a, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16_tmem_a(tmem + tDV, a + 16, b, idKM, 1u);
-        }
-        // dK += dS^T Q: A = dS^T (hi, lo) K-major from shared memory
+        // dK += dS^T Q: A = dS^T (hi, lo) K-major from shared memory; then Q is free
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
@@ -170,7 +173,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + tDK, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
           umma_bf16(tmem + tDK, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
         }
-        umma_commit(bQOfree);
+        umma_commit(bQfree);
+        // dV += P^T dO: A = P^T (hi, lo) from TMEM, B = dO MN-major (K = queries); then dO is free
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint64_t b = sdesc_sw128(sO + kk * 2048, Lay::kChunk, 1024);
+          umma_bf16_tmem_a(tmem + tDV, a, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + tDV, a + 16, b, idKM, 1u);
+        }
+        umma_commit(bOfree);
         // dQ = dS K  (M = queries, K = keys, N = d): dS^T read M-major
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -218,23 +230,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tl + tDP + c * 32, dr);
         tmem_ld_wait();
         uint32_t phi[16], plo[16], dhi[16], dlo[16];
+        const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int qi = c * 32 + e + h;
-            float p = fast_exp2(__uint_as_float(sr[e + h]) * scale_log2 - sVec[qi]);
-            if (diag && q0 + qi < kv_g) p = 0.f;
-            pv[h] = p;
-            dv[h] = p * (__uint_as_float(dr[e + h]) - sVec[128 + qi]) * scale;
+          const int qi = c * 32 + e;
+          const float2 lse2 = *reinterpret_cast<const float2*>(sVec + qi);
+          const float2 del2 = *reinterpret_cast<const float2*>(sVec + 128 + qi);
+          float pa, pb;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-lse2.x, -lse2.y)),
+                    pa, pb);
+          pa = fast_exp2(pa);
+          pb = fast_exp2(pb);
+          if (diag) {
+            if (q0 + qi < kv_g) pa = 0.f;
+            if (q0 + qi + 1 < kv_g) pb = 0.f;
           }
-          const __nv_bfloat162 ph = __floats2bfloat162_rn(pv[0], pv[1]);
-          const __nv_bfloat162 dh = __floats2bfloat162_rn(dv[0], dv[1]);
-          phi[e >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
-          dhi[e >> 1] = *reinterpret_cast<const uint32_t*>(&dh);
-          plo[e >> 1] = pack_bf16x2(pv[0] - __low2float(ph), pv[1] - __high2float(ph));
-          dlo[e >> 1] = pack_bf16x2(dv[0] - __low2float(dh), dv[1] - __high2float(dh));
+          const uint64_t p2 = f2_pack(pa, pb);
+          const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(del2.x, del2.y));
+          float da, db;
+          f2_unpack(f2_mul(f2_mul(p2, sc2), diff2), da, db);
+          split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
+          split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
         }
         // P^T over the S^T columns just read: hi in the first 16, lo in the last 16
         tmem_st16(tl + tS + c * 32, phi);
@@ -264,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tl + tDP + col, r);
         tmem_ld_wait();
         if (qg < S) {
-          float4* dst = reinterpret_cast<float4*>(dQ + ((int64_t)bh * S + qg) * D + col);
+          float* dst = dQ + ((int64_t)bh * S + qg) * D + col;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            atomicAdd(dst + q, make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
+            red_add_v4(dst + 4 * q, __uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                       __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
         }
       }
       tc_fence_before();

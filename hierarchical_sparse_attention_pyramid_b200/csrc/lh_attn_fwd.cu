@@ -188,16 +188,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(ts + ch * 32, r);
         tmem_ld_wait();
+        if (diag) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = ch * 32 + i;
-          if (!(diag && col > row)) mx = fmaxf(mx, __uint_as_float(r[i]));  // later keys are masked
+          for (int i = 0; i < 32; ++i)
+            if (ch * 32 + i <= row) mx = fmaxf(mx, __uint_as_float(r[i]));  // later keys are masked
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
         }
       }
-      const float m_new = fmaxf(m_run, mx * scale_log2);
-      const float alpha = fast_exp2(m_run - m_new);
+      // Lazy rescaling: the reference m_run moves only when the row max exceeds
+      // it by more than 8 (so every P stays <= 2^8); O and l share the
+      // reference, so the result is exact either way.
+      const float m_tile = mx * scale_log2;
+      const bool move = m_tile > m_run + 8.f;
+      const float m_new = move ? m_tile : m_run;
+      const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;
       // the previous P V of this tile is done (its completion preceded this S)
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (j >= 1 && __any_sync(0xffffffffu, move)) {
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t o[32];
@@ -208,10 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(to + ch * 32, o);
         }
       }
-      // pass 2: P = exp2(s - m) as a bf16 pair written back over the chunk it
-      // came from: chunk ch (keys 32ch..32ch+31) holds hi in its first 16
+      // pass 2: P = exp2(s*scale - m) as a bf16 pair written back over the chunk
+      // it came from: chunk ch (keys 32ch..32ch+31) holds hi in its first 16
       // columns and lo in its last 16
-      float rs = 0.f;
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
+      uint64_t rs2 = f2_pack(0.f, 0.f);
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t r[32];
@@ -220,20 +229,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const int col = ch * 32 + 2 * q;
-          float a = fast_exp2(fmaf(__uint_as_float(r[2 * q]), scale_log2, -m_new));
-          float b = fast_exp2(fmaf(__uint_as_float(r[2 * q + 1]), scale_log2, -m_new));
-          if (diag && col > row) a = 0.f;
-          if (diag && col + 1 > row) b = 0.f;
-          rs += a + b;
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          hi[q] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[q] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
+          float a, b;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), c2, nm2), a, b);
+          a = fast_exp2(a);
+          b = fast_exp2(b);
+          if (diag) {
+            const int col = ch * 32 + 2 * q;
+            if (col > row) a = 0.f;
+            if (col + 1 > row) b = 0.f;
+          }
+          rs2 = f2_add(rs2, f2_pack(a, b));
+          split_bf16x2(a, b, hi[q], lo[q]);
         }
         tmem_st16(ts + ch * 32, hi);
         tmem_st16(ts + ch * 32 + 16, lo);
       }
-      l_run = l_run * alpha + rs;
+      float rsa, rsb;
+      f2_unpack(rs2, rsa, rsb);
+      l_run = l_run * alpha + (rsa + rsb);
       m_run = m_new;
       tmem_st_wait();
       tc_fence_before();
