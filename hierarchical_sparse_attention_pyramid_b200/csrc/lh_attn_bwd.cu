@@ -139,6 +139,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sO = smem_u32(smem + Lay::oO);
       const uint32_t sHi = smem_u32(smem + Lay::oHi), sLo = smem_u32(smem + Lay::oLo);
+      // base descriptors: an operand at byte offset off is base + (off >> 4)
+      const uint64_t kK = sdesc_sw128(sK, 16, 1024), kQ = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t kV = sdesc_sw128(sV, 16, 1024), kO = sdesc_sw128(sO, 16, 1024);
+      const uint64_t kHi = sdesc_sw128(sHi, 16, 1024), kLo = sdesc_sw128(sLo, 16, 1024);
+      const uint64_t mO = sdesc_sw128(sO, Lay::kChunk, 1024), mQ = sdesc_sw128(sQ, Lay::kChunk, 1024);
+      const uint64_t mK = sdesc_sw128(sK, Lay::kChunk, 1024);
+      const uint64_t mHi = sdesc_sw128(sHi, Lay::kChunk, 1024), mLo = sdesc_sw128(sLo, Lay::kChunk, 1024);
       bool ok = mbar_wait(bKV, 0, abort_flag);
       for (int it = 0; ok && it < n_q; ++it) {
         if (!mbar_wait(bQ, it & 1, abort_flag)) break;
@@ -147,9 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the previous tile, whose dV product was issued before this one
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          umma_bf16(tmem + tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idSS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + tS, kK + off, kQ + off, idSS, kk > 0 ? 1u : 0u);
         }
         // dP^T = V dO^T into the dQ columns, once dO has landed and the previous
         // dQ has been read out
@@ -158,9 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          umma_bf16(tmem + tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024), idSS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + tDP, kV + off, kO + off, idSS, kk > 0 ? 1u : 0u);
         }
         umma_commit(bSdP);
         if (!mbar_wait(bPS, it & 1, abort_flag)) break;
@@ -168,17 +173,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dK += dS^T Q: A = dS^T (hi, lo) K-major from shared memory; then Q is free
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          const uint64_t b = sdesc_sw128(sQ + kk * 2048, Lay::kChunk, 1024);
-          umma_bf16(tmem + tDK, sdesc_sw128(sHi + aoff, 16, 1024), b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + tDK, sdesc_sw128(sLo + aoff, 16, 1024), b, idKM, 1u);
+          const uint32_t aoff = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
+          const uint64_t b = mQ + ((kk * 2048) >> 4);
+          umma_bf16(tmem + tDK, kHi + aoff, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16(tmem + tDK, kLo + aoff, b, idKM, 1u);
         }
         umma_commit(bQfree);
         // dV += P^T dO: A = P^T (hi, lo) from TMEM, B = dO MN-major (K = queries); then dO is free
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint64_t b = sdesc_sw128(sO + kk * 2048, Lay::kChunk, 1024);
+          const uint64_t b = mO + ((kk * 2048) >> 4);
           umma_bf16_tmem_a(tmem + tDV, a, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
           umma_bf16_tmem_a(tmem + tDV, a + 16, b, idKM, 1u);
         }
@@ -186,10 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dQ = dS K  (M = queries, K = keys, N = d): dS^T read M-major
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t off = kk * 2048;
-          const uint64_t b = sdesc_sw128(sK + off, Lay::kChunk, 1024);
-          umma_bf16(tmem + tDP, sdesc_sw128(sHi + off, Lay::kChunk, 1024), b, idMM, kk > 0 ? 1u : 0u);
-          umma_bf16(tmem + tDP, sdesc_sw128(sLo + off, Lay::kChunk, 1024), b, idMM, 1u);
+          const uint32_t off = (kk * 2048) >> 4;
+          umma_bf16(tmem + tDP, mHi + off, mK + off, idMM, kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + tDP, mLo + off, mK + off, idMM, 1u);
         }
         umma_commit(bDQ);
       }

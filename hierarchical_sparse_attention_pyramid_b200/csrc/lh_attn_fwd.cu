@@ -118,13 +118,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idQK = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idPV = idesc_bf16(BM, D, false, true);
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
+      // base descriptors: an operand at byte offset off is base + (off >> 4)
+      const uint64_t kQ = sdesc_sw128(sQ, 16, 1024), kK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t mV = sdesc_sw128(sV, Lay::kChunk, 1024);
       auto issue_s = [&](int x, int j) {
-        const uint32_t qb = sQ + x * Lay::kTile, kb = sK + (j & 1) * Lay::kTile;
+        const uint64_t qb = kQ + ((x * Lay::kTile) >> 4), kb = kK + (((j & 1) * Lay::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::kChunk + (kk & 3) * 32;
-          umma_bf16(tmem + x * 128, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idQK,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + x * 128, qb + off, kb + off, idQK, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bS[x]);
       };
@@ -145,11 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             v_ready = true;
           }
           tc_fence_after();
-          const uint32_t vb = sV + st * Lay::kTile;
+          const uint64_t vb = mV + ((st * Lay::kTile) >> 4);
           const uint32_t pa = tmem + x * 128;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t b = sdesc_sw128(vb + kk * 2048, Lay::kChunk, 1024);
+            const uint64_t b = vb + ((kk * 2048) >> 4);
             const uint32_t a = pa + (kk >> 1) * 32 + (kk & 1) * 8;  // hi of keys 16kk..16kk+15
             umma_bf16_tmem_a(tmem + 256 + x * D, a, b, idPV, (j > 0 || kk > 0) ? 1u : 0u);
             umma_bf16_tmem_a(tmem + 256 + x * D, a + 16, b, idPV, 1u);
