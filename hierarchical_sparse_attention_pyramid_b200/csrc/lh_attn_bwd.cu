@@ -15,8 +15,9 @@
 //              S^T and dP^T into P^T (hi/lo, written back into the S^T
 //              columns of TMEM, where the dV product reads it as its A
 //              operand) and dS^T (hi/lo, to shared memory); then each reads
-//              half of the tile's dQ from TMEM and adds it to dQs with fp32
-//              vector reductions at the L2; at the end they write dKs and dVs
+//              half of the tile's dQ from TMEM into shared memory, and one
+//              thread adds the tile to dQs with a TMA reduce-add; at the end
+//              they write dKs and dVs
 //   warp 8     TMA producer: K, V once; Q and dO per query tile, each as
 //              soon as the product that last reads it (dK, dV) is done
 //   warp 9     MMA issuer (one thread) and TMEM owner
@@ -29,6 +30,9 @@
 namespace lh {
 
 bool make_seq_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int D, int box_rows);
+
+// [BH][rows][D] fp32 viewed as (D, rows, BH); box of 32 x box_rows x 1, 128-byte swizzle
+bool make_f32_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int D, int box_rows);
 
 namespace {
 using namespace sm100;
@@ -46,7 +50,7 @@ struct BwdSmem {
   static constexpr int oV = oK + kTile;
   static constexpr int oQ = oV + kTile;
   static constexpr int oO = oQ + kTile;          // dO
-  static constexpr int oHi = oO + kTile;         // dS^T, bf16 high part
+  static constexpr int oHi = oO + kTile;         // dS^T, bf16 high part; later the fp32 dQ tile
   static constexpr int oLo = oHi + 2 * kChunk;   // bf16 of the remainder
   static constexpr int oVec = oLo + 2 * kChunk;  // LSE*log2e [128], Delta [128]
   static constexpr int oBar = oVec + 1024;
@@ -60,7 +64,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dQ,
+                    const __grid_constant__ CUtensorMap tmDQ,
+                    const float* __restrict__ LSE, const float* __restrict__ Delta,
                     float* __restrict__ dK, float* __restrict__ dV, int* errw, int S, float scale_log2,
                     float scale) {
   using Lay = BwdSmem<D>;
@@ -219,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (kt + it) * BM;
       const float vec_cur = vec_next;
       if (it + 1 < n_q) vec_next = vec_of(q0 + BM);  // one tile ahead
+      if (ct == 0) bulk_wait_read_all();  // the previous dQ reduce has read its staging tile
       compute_sync();  // every thread is done with the previous tile's LSE / Delta
       sVec[ct] = vec_cur;
       compute_sync();
@@ -272,27 +278,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bPS);
-      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1))
+      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1)): TMEM -> shared memory
+      // (the dS buffers are free once the dQ product is done), then one TMA
+      // reduce-add of the whole tile into dQs
       if (!mbar_wait(bDQ, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      const int qg = q0 + t;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
-        const int col = g * (D / 2) + c * 32;
+        const int cc = g * (D / 64) + c;  // 32-float column chunk of the tile
         uint32_t r[32];
-        tmem_ld32(tl + tDP + col, r);
+        tmem_ld32(tl + tDP + cc * 32, r);
         tmem_ld_wait();
-        if (qg < S) {
-          float* dst = dQ + ((int64_t)bh * S + qg) * D + col;
+        uint8_t* dst = smem + Lay::oHi + cc * (128 * 128) + t * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            red_add_v4(dst + 4 * q, __uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                       __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-        }
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(dst + ((k ^ (t & 7)) << 4)) = make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
       }
       tc_fence_before();
       mbar_arrive(bDQfree);
+      fence_proxy_async_smem();
+      compute_sync();
+      if (ct == 0) {
+        for (int cc = 0; cc < D / 32; ++cc)
+          tma_reduce_add_3d(&tmDQ, smem + Lay::oHi + cc * (128 * 128), cc * 32, q0, bh);
+        bulk_commit_group();
+      }
     }
     if (ok && !*abort_flag) {
       // bDQ of the last tile has completed: dV and dK are final
@@ -319,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  if (threadIdx.x == 0) bulk_wait_all();  // every dQ reduce has landed
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -333,9 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
                             float* dvs, int* errw, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq;
   if (!make_seq_map(&mq, qs, BH, S, d, BM) || !make_seq_map(&mk, ks, BH, S, d, BN) ||
-      !make_seq_map(&mv, vs, BH, S, d, BN) || !make_seq_map(&mo, dos, BH, S, d, BM))
+      !make_seq_map(&mv, vs, BH, S, d, BN) || !make_seq_map(&mo, dos, BH, S, d, BM) ||
+      !make_f32_map(&mdq, dqs, BH, S, d, BM))
     return cudaErrorInvalidValue;
   const double scale = 1.0 / sqrt((double)d);
   const float scale_log2 = (float)(1.4426950408889634 * scale);
@@ -344,13 +357,13 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const 
     const int smem = BwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_bwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, lse, delta, dqs, dks, dvs, errw, (int)S,
+    attn_bwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mdq, lse, delta, dks, dvs, errw, (int)S,
                                                         scale_log2, (float)scale);
   } else {
     const int smem = BwdSmem<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_bwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, lse, delta, dqs, dks, dvs, errw, (int)S,
+    attn_bwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mdq, lse, delta, dks, dvs, errw, (int)S,
                                                        scale_log2, (float)scale);
   }
   return cudaGetLastError();
