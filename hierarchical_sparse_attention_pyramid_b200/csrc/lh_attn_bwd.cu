@@ -59,6 +59,8 @@ struct BwdSmem {
 };
 
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// the 128 threads of compute warpgroup g
+__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -224,7 +226,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (kt + it) * BM;
       const float vec_cur = vec_next;
       if (it + 1 < n_q) vec_next = vec_of(q0 + BM);  // one tile ahead
-      if (ct == 0) bulk_wait_read_all();  // the previous dQ reduce has read its staging tile
       compute_sync();  // every thread is done with the previous tile's LSE / Delta
       sVec[ct] = vec_cur;
       compute_sync();
@@ -265,7 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P^T over the S^T columns just read: hi in the first 16, lo in the last 16
         tmem_st16(tl + tS + c * 32, phi);
         tmem_st16(tl + tS + c * 32 + 16, plo);
-        // dS^T row t, query columns c*32..c*32+31: 4 chunks of 16 bytes in region c/2
+        if (cc == 0) {
+          // this group's previous dQ reduce must have read the regions it reuses
+          if (t == 0) bulk_wait_read_all();
+          group_sync(g);
+        }
+        // dS^T row t, query columns c*32..c*32+31: 4 chunks of 16 bytes in region c/2 = g
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int ch = (c & 1) * 4 + q;
@@ -278,19 +284,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bPS);
-      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1)): TMEM -> shared memory
-      // (the dS buffers are free once the dQ product is done), then one TMA
-      // reduce-add of the whole tile into dQs
+      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1)): TMEM -> shared memory,
+      // into the two regions (hi and lo, region g) that this group's dS writes
+      // use, then one TMA reduce-add per 32-column chunk into dQs, issued by
+      // the group; the dS buffers are free once the dQ product is done
       if (!mbar_wait(bDQ, it & 1, abort_flag)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
-        const int cc = g * (D / 64) + c;  // 32-float column chunk of the tile
+        const int col = g * (D / 2) + c * 32;
         uint32_t r[32];
-        tmem_ld32(tl + tDP + cc * 32, r);
+        tmem_ld32(tl + tDP + col, r);
         tmem_ld_wait();
-        uint8_t* dst = smem + Lay::oHi + cc * (128 * 128) + t * 128;
+        uint8_t* dst = smem + (c == 0 ? Lay::oHi : Lay::oLo) + g * (128 * 128) + t * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           *reinterpret_cast<uint4*>(dst + ((k ^ (t & 7)) << 4)) = make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
@@ -298,10 +305,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bDQfree);
       fence_proxy_async_smem();
-      compute_sync();
-      if (ct == 0) {
-        for (int cc = 0; cc < D / 32; ++cc)
-          tma_reduce_add_3d(&tmDQ, smem + Lay::oHi + cc * (128 * 128), cc * 32, q0, bh);
+      group_sync(g);
+      if (t == 0) {
+        for (int c = 0; c < D / 64; ++c)
+          tma_reduce_add_3d(&tmDQ, smem + (c == 0 ? Lay::oHi : Lay::oLo) + g * (128 * 128), g * (D / 2) + c * 32, q0, bh);
         bulk_commit_group();
       }
     }
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  if (threadIdx.x == 0) bulk_wait_all();  // every dQ reduce has landed
+  if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait_all();  // every dQ reduce has landed
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
