@@ -308,6 +308,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads instead (a smaller cut for profiling)")
     args = ap.parse_args()
 
     world, rank, local = dist_setup()
@@ -320,6 +322,8 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
     layer = lh.Layer.of(w)
     x = synth.cuda_inputs(w, dev, seed=w.seed + 16 * rank)
     bufs = lh.Buffers(layer, dev)

@@ -151,10 +151,21 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
   const float* os = a.os + bh * a.S * D + cv * VE;
   T* out = static_cast<T*>(a.y) + bh * a.N * D + cv * VE;
 
-  float upper[VE];
+  // contribution of level 1, refreshed when the level-1 entry changes, and the
+  // summed contribution of levels >= 2, refreshed when the level-2 entry does
+  float up1[VE], high[VE];
 #pragma unroll
-  for (int c = 0; c < VE; ++c) upper[c] = 0.f;
-  int64_t cur1 = -2;  // level-1 entry of the previous step
+  for (int c = 0; c < VE; ++c) up1[c] = high[c] = 0.f;
+  auto contribution = [&](int l, int64_t i, float (&acc)[VE]) {
+    const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
+    if (s >= 0) {
+      float v[VE];
+      load_f32<VE>(os + (int64_t)s * D, v);
+#pragma unroll
+      for (int c = 0; c < VE; ++c) acc[c] += v[c];
+    }
+  };
+  int64_t cur1 = -2, cur2 = -2;  // level-1 and level-2 entries of the previous step
   int s0w = -1;
   for (int r = 0; r < steps; r += R) {
     const int64_t u = u0 + r;
@@ -169,16 +180,16 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
       if (i1 != cur1) {
         cur1 = i1;
 #pragma unroll
-        for (int c = 0; c < VE; ++c) upper[c] = 0.f;
+        for (int c = 0; c < VE; ++c) up1[c] = 0.f;
+        contribution(1, i1, up1);
+        if constexpr (NL > 2) {
+          const int64_t i2 = (key >> (2 * log2p)) - 1;
+          if (i2 != cur2) {
+            cur2 = i2;
 #pragma unroll
-        for (int l = 1; l < NL; ++l) {
-          const int64_t i = (key >> (l * log2p)) - 1;
-          const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
-          if (s >= 0) {
-            float v[VE];
-            load_f32<VE>(os + (int64_t)s * D, v);
+            for (int c = 0; c < VE; ++c) high[c] = 0.f;
 #pragma unroll
-            for (int c = 0; c < VE; ++c) upper[c] += v[c];
+            for (int l = NL - 1; l >= 2; --l) contribution(l, (key >> (l * log2p)) - 1, high);
           }
         }
       }
@@ -186,7 +197,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
     const int s0 = __shfl_sync(kFull, s0w, (r & 31) + lr);
     float y[VE];
 #pragma unroll
-    for (int c = 0; c < VE; ++c) y[c] = upper[c];
+    for (int c = 0; c < VE; ++c) y[c] = up1[c] + high[c];
     if (s0 >= 0) {
       float v[VE];
       load_f32<VE>(os + (int64_t)s0 * D, v);

@@ -192,9 +192,21 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
   const float* xs = a.dxs[tensor] + bh * a.S * D + cv * VE;
   T* out = static_cast<T*>(a.dx[tensor]) + (bh * a.N + row0) * D + cv * VE;
 
-  float upper[VE];
+  // contribution of level 1, refreshed at level-1 boundaries, and the summed
+  // contribution of levels >= 2, refreshed at level-2 boundaries
+  float up1[VE], high[VE];
 #pragma unroll
-  for (int i = 0; i < VE; ++i) upper[i] = 0.f;
+  for (int i = 0; i < VE; ++i) up1[i] = high[i] = 0.f;
+  auto contribution = [&](int l, int64_t i, float (&acc)[VE]) {
+    const int s = so[a.level_off[l] + i];
+    if (s >= 0) {
+      float v[VE];
+      load_f32<VE>(xs + (int64_t)s * D, v);
+      const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
+#pragma unroll
+      for (int c = 0; c < VE; ++c) acc[c] = fmaf(v[c], inv, acc[c]);
+    }
+  };
   int s0w = -1;
   for (int r = 0; r < rows; r += R) {
     const int64_t t = row0 + r;  // first row of this instruction
@@ -202,16 +214,14 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
     if constexpr (NL > 1) {
       if ((t & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
-        for (int i = 0; i < VE; ++i) upper[i] = 0.f;
+        for (int c = 0; c < VE; ++c) up1[c] = 0.f;
+        contribution(1, t >> log2p, up1);
+        if constexpr (NL > 2) {
+          if ((t & ((1 << (2 * log2p)) - 1)) == 0) {
 #pragma unroll
-        for (int l = 1; l < NL; ++l) {
-          const int s = so[a.level_off[l] + (t >> (l * log2p))];
-          if (s >= 0) {
-            float v[VE];
-            load_f32<VE>(xs + (int64_t)s * D, v);
-            const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
+            for (int c = 0; c < VE; ++c) high[c] = 0.f;
 #pragma unroll
-            for (int i = 0; i < VE; ++i) upper[i] = fmaf(v[i], inv, upper[i]);
+            for (int l = NL - 1; l >= 2; --l) contribution(l, t >> (l * log2p), high);
           }
         }
       }
@@ -219,12 +229,12 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
     const int s0 = __shfl_sync(kFull, s0w, (r & 31) + lr);
     float y[VE];
 #pragma unroll
-    for (int i = 0; i < VE; ++i) y[i] = upper[i];
+    for (int c = 0; c < VE; ++c) y[c] = up1[c] + high[c];
     if (s0 >= 0) {
       float v[VE];
       load_f32<VE>(xs + (int64_t)s0 * D, v);
 #pragma unroll
-      for (int i = 0; i < VE; ++i) y[i] += v[i];
+      for (int c = 0; c < VE; ++c) y[c] += v[c];
     }
     if (r + lr < rows) store_vec<T, VE>(out + (int64_t)(r + lr) * D, y);
   }
