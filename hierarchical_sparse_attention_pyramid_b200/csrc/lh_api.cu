@@ -165,6 +165,14 @@ int* err_word(void* ws) { return static_cast<int*>(ws); }
 
 lh_status make_dims(const lh_config* cfg, lh_plan_info* info, Dims* D) { return plan_impl(cfg, info, D); }
 
+int materialized_level(const Dims& D) {
+  // level l (< top) costs N/p^l rows to write whole, or p^(l+1) k' rows to
+  // read back for its kept entries; coarser levels only favour writing more
+  for (int l = 1; l < D.L - 1; ++l)
+    if ((D.level_len[l]) <= ((int64_t)D.kprime[l] << ((l + 1) * D.log2p))) return l;
+  return D.L > 1 ? D.L - 1 : 1;
+}
+
 }  // namespace lh
 
 using namespace lh;
@@ -305,9 +313,11 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   void* vs = c + I.ctx_off_vs;
   float* os = reinterpret_cast<float*>(c + I.ctx_off_os);
   float* lse = reinterpret_cast<float*>(c + I.ctx_off_lse);
-  LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st), "lh_forward: pool");
+  const int first = materialized_level(D);
+  LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st, first), "lh_forward: pool");
   LH_CUDA(launch_score_topk(D, norms, spyr, sel, errw, st), "lh_forward: score_topk");
-  LH_CUDA(launch_gather(D, q, k, v, pq, pk, pv, sel, qs, ks, vs, seq_map, slot_of, errw, st), "lh_forward: gather");
+  LH_CUDA(launch_gather(D, q, k, v, pq, pk, pv, sel, qs, ks, vs, seq_map, slot_of, errw, st, first),
+          "lh_forward: gather");
   LH_CUDA(launch_attn_fwd(D.BH, D.S, D.d, qs, ks, vs, os, lse, errw, st), "lh_forward: attn_fwd");
   LH_CUDA(launch_scatter_back(D, os, slot_of, y, st), "lh_forward: scatter_back");
   return LH_OK;

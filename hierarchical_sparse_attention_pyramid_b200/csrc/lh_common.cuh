@@ -102,13 +102,20 @@ __device__ __forceinline__ void load_f32(const float* src, float (&x)[VE]) {
 // ---------------------------------------------------------------------------
 // launchers (host side, one per stage); all return cudaGetLastError()
 // ---------------------------------------------------------------------------
+// levels below first_level are not written (their sums still carry upward)
 cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void* v, void* pq, void* pk, void* pv,
-                        float* norms, cudaStream_t st);
+                        float* norms, cudaStream_t st, int first_level = 1);
 cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, int32_t* sel, int* errw,
                               cudaStream_t st);
+// kept entries of levels 1 .. first_level-1 are averaged from level 0 here
+// instead of being read from the pyramid
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
                           const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
-                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st);
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level = 1);
+
+// first pyramid level lh_forward materialises: finer kept entries are cheaper
+// to average from level 0 in the gather than to write whole levels
+int materialized_level(const Dims& D);
 cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st);
 cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
                                    void* dos, float* delta, int* errw, cudaStream_t st);

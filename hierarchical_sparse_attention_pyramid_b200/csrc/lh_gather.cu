@@ -34,7 +34,7 @@ struct GatherArgs {
   int64_t sel_off[LH_MAX_LEVELS];
   int64_t cnt_off[LH_MAX_LEVELS + 1];  // first sequence entry id of each level's kept list
   int32_t kprime[LH_MAX_LEVELS];
-  int L, log2p;
+  int L, log2p, first_level;
 };
 
 // kept entries of level lv with index < X
@@ -89,8 +89,40 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(GatherArgs a) {
     a.seq_map[bh * a.S + slot] = (int32_t)(((int64_t)l << 28) | i);
     a.slot_of[bh * a.pyr_entries + a.level_off[l] + i] = (int32_t)slot;
   }
-  // copy the three rows, 8 elements per lane step, converting to bf16
   constexpr int CH = D / 8;
+  if (l >= 1 && l < a.first_level) {
+    // entry not materialised: average its p^l level-0 rows (fp32, rounded once)
+    const int nr = 1 << (l * a.log2p);
+    const float inv = __int_as_float((127 - l * a.log2p) << 23);  // 2^(-l log2p), exact
+    for (int c = lane; c < 3 * CH; c += 32) {
+      const int t = c / CH, off = (c % CH) * 8;
+      const T* src = static_cast<const T*>(a.x0[t]) + (bh * a.N + (i << (l * a.log2p))) * D + off;
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+      for (int r = 0; r < nr; ++r) {
+        float x[8];
+        if constexpr (sizeof(T) == 2) {
+          load_vec<T, 8>(src + (int64_t)r * D, x);
+        } else {
+          load_f32<4>(reinterpret_cast<const float*>(src + (int64_t)r * D), *reinterpret_cast<float(*)[4]>(x));
+          load_f32<4>(reinterpret_cast<const float*>(src + (int64_t)r * D) + 4, *reinterpret_cast<float(*)[4]>(x + 4));
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += x[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] *= inv;
+      if constexpr (sizeof(T) == 2) {
+        // the materialised pyramid rounds the mean to bf16 once; do the same
+        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.S + slot) * D + off, acc);
+      } else {
+        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.S + slot) * D + off, acc);
+      }
+    }
+    return;
+  }
+  // copy the three rows, 8 elements per lane step, converting to bf16
   for (int c = lane; c < 3 * CH; c += 32) {
     const int t = c / CH, off = (c % CH) * 8;
     const T* src = (l == 0) ? static_cast<const T*>(a.x0[t]) + (bh * a.N + i) * D
@@ -303,7 +335,7 @@ cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t blocks, cuda
 
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
                           const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
-                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st) {
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level) {
   GatherArgs a{};
   a.x0[0] = q; a.x0[1] = k; a.x0[2] = v;
   a.pyr[0] = pq; a.pyr[1] = pk; a.pyr[2] = pv;
@@ -327,6 +359,7 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
   for (int l = 0; l < D.L - 1; ++l) a.cnt_off[l + 1] = a.cnt_off[l] + ((int64_t)D.kprime[l] << D.log2p);
   a.L = D.L;
   a.log2p = D.log2p;
+  a.first_level = first_level;
   cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * D.pyr_entries * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (D.BH * D.S + kWarps - 1) / kWarps;

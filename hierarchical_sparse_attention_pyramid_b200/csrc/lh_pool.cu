@@ -25,7 +25,7 @@ struct PoolArgs {
   int64_t BH, N, upper_entries;
   int64_t upper_off[LH_MAX_LEVELS];
   int64_t tasks_per_head;
-  int task_rows, log2p;
+  int task_rows, log2p, first_level;
 };
 
 // Butterfly reduce-scatter of U (8 or 16) per-lane partial sums, one per row
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
 #pragma unroll
             for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
             const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
-            store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
+            if (l >= a.first_level) store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
 #pragma unroll
             for (int i = 0; i < VE; ++i) {
               acc[l + 1][i] += acc[l][i];
@@ -272,7 +272,7 @@ int task_rows_for(const Dims& D) {
 }  // namespace
 
 cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void* v, void* pq, void* pk, void* pv,
-                        float* norms, cudaStream_t st) {
+                        float* norms, cudaStream_t st, int first_level) {
   PoolArgs a{};
   a.x[0] = q; a.x[1] = k; a.x[2] = v;
   a.pyr[0] = pq; a.pyr[1] = pk; a.pyr[2] = pv;
@@ -282,6 +282,7 @@ cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void*
   a.task_rows = task_rows_for(D);
   a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
   a.log2p = D.log2p;
+  a.first_level = first_level;
   const int64_t warps = 3 * D.BH * a.tasks_per_head;
   const int64_t blocks = (warps + kWarps - 1) / kWarps;
   if (D.dtype == LH_BF16) {
