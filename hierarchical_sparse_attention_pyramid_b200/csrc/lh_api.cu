@@ -245,7 +245,6 @@ lh_status lh_attn_bwd(const lh_config* cfg, int64_t S, const void* qs, const voi
   LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(lse); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
   LH_CHECK_PTR(dqs); LH_CHECK_PTR(dks); LH_CHECK_PTR(dvs); LH_CHECK_PTR(ws);
   const int64_t BH = cfg->B * cfg->H;
-  LH_CUDA(cudaMemsetAsync(dqs, 0, (size_t)BH * S * cfg->d * sizeof(float), (cudaStream_t)stream), "lh_attn_bwd");
   LH_CUDA(launch_attn_bwd(BH, S, cfg->d, qs, ks, vs, lse, dos, delta, dqs, dks, dvs, err_word(ws),
                           (cudaStream_t)stream),
           "lh_attn_bwd");
@@ -349,7 +348,6 @@ lh_status lh_backward(const lh_config* cfg, const void* dy, const void* ctx, siz
   float* dks = reinterpret_cast<float*>(w + I.ws_off_dks);
   float* dvs = reinterpret_cast<float*>(w + I.ws_off_dvs);
   LH_CUDA(launch_scatter_adjoint(D, dy, seq_map, os, dos, delta, errw, st), "lh_backward: scatter_adjoint");
-  LH_CUDA(cudaMemsetAsync(dqs, 0, I.grad_seq_bytes, st), "lh_backward");
   LH_CUDA(launch_attn_bwd(D.BH, D.S, D.d, qs, ks, vs, lse, dos, delta, dqs, dks, dvs, errw, st),
           "lh_backward: attn_bwd");
   LH_CUDA(launch_pool_adjoint(D, dqs, dks, dvs, slot_of, dq, dk, dv, st), "lh_backward: pool_adjoint");

@@ -5,23 +5,28 @@
 // With P = softmax(Qs Ks^T / sqrt(d)) (causal) recomputed from the saved LSE,
 //   dVs = P^T dOs,  dP = dOs Vs^T,  dS = P * (dP - Delta) / sqrt(d),
 //   dQs = dS Ks,    dKs = dS^T Qs,  Delta = rowsum(dOs * Os).
-// P^T and dS^T enter their products as bf16 (hi + lo) pairs, so the bf16
+// P and dS enter their products as bf16 (hi + lo) pairs, so the bf16
 // roundings of the probabilities and of dS do not show in the gradients.
 //
-// One CTA owns a 128-row key/value tile of one (batch, head) and walks the
-// query tiles from the diagonal to the end.  Warp roles:
-//   warps 0-7  two compute warpgroups; thread (g, t) owns key row t (TMEM lane
-//              t) and query columns [64g, 64g+64) of the tile.  One pass turns
-//              S^T and dP^T into P^T (hi/lo, written back into the S^T
-//              columns of TMEM, where the dV product reads it as its A
-//              operand) and dS^T (hi/lo, to shared memory); then each reads
-//              half of the tile's dQ from TMEM into shared memory, and one
-//              thread adds the tile to dQs with a TMA reduce-add; at the end
-//              they write dKs and dVs
-//   warp 8     TMA producer: K, V once; Q and dO per query tile, each as
-//              soon as the product that last reads it (dK, dV) is done
-//   warp 9     MMA issuer (one thread) and TMEM owner
-// TMEM columns: S^T/P^T [0,128), dP^T/dQ [128,256), dV [256,256+D), dK [256+D,256+2D).
+// Two kernels, each writing its gradient once (no atomics):
+//
+// attn_bwd_kv_kernel (dKs, dVs) - one CTA per 128-row key tile; it steps over
+//   64-query half tiles from the diagonal to the end.  For half step s the MMA
+//   warp computes S^T = K Q_h^T and dP^T = V dO_h^T into TMEM buffer s&1 while
+//   the compute warpgroups work on the other buffer; they write P^T and dS^T
+//   (hi/lo) back over the columns they read, and the MMA warp then adds
+//   dV += P^T dO_h and dK += dS^T Q_h with both A operands read from TMEM.
+//   Q_h, dO_h stream through a 4-slot ring.
+//
+// attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over
+//   64-key half tiles up to the diagonal: S = Q K_h^T and dP = dO V_h^T into
+//   TMEM buffer u&1, the compute warpgroups write dS (hi/lo) over the dP
+//   columns, and dQ += dS K_h reads it from TMEM.  K_h and V_h stream through
+//   4-slot rings, each slot released by the last product that reads it.
+//
+// Warp roles in both: warps 0-7 two compute warpgroups (thread (g, t) owns
+// TMEM lane t and columns [32g, 32g+32) of each 64-column half), warp 8 TMA
+// producer, warp 9 MMA issuer (one thread) and TMEM owner.
 #include <math.h>
 
 #include "lh_common.cuh"
@@ -31,78 +36,77 @@ namespace lh {
 
 bool make_seq_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int D, int box_rows);
 
-// [BH][rows][D] fp32 viewed as (D, rows, BH); box of 32 x box_rows x 1, 128-byte swizzle
-bool make_f32_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int D, int box_rows);
-
 namespace {
 using namespace sm100;
 
-constexpr int BM = 128;  // query rows per tile
-constexpr int BN = 128;  // key rows per CTA
 constexpr int kCompute = 256;
 constexpr int kThreads = kCompute + 64;
+constexpr int kRegion = 128 * 128;  // one [128 rows][64 bf16] SW128 region
+constexpr int kHalfRegion = 64 * 128;
 
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// P^T / dS (hi, lo) of 32 columns c0..c0+31 of one row as bf16 pairs over the
+// 32 TMEM columns they were read from: hi in the first 16, lo in the last 16.
+__device__ __forceinline__ void store_pair_chunk(uint32_t taddr, const uint32_t (&hi)[16], const uint32_t (&lo)[16]) {
+  tmem_st16(taddr, hi);
+  tmem_st16(taddr + 16, lo);
+}
+
+// ===========================================================================
+// dKs, dVs
+// ===========================================================================
 template <int D>
-struct BwdSmem {
-  static constexpr int kChunk = 128 * 128;
-  static constexpr int kTile = D / 64 * kChunk;
+struct KvSmem {
+  static constexpr int kTile = D / 64 * kRegion;         // K or V tile, 128 rows
+  static constexpr int kHalf = D / 64 * kHalfRegion;     // Q_h or dO_h, 64 rows
   static constexpr int oK = 0;
   static constexpr int oV = oK + kTile;
-  static constexpr int oQ = oV + kTile;
-  static constexpr int oO = oQ + kTile;          // dO
-  static constexpr int oHi = oO + kTile;         // dS^T, bf16 high part; later the fp32 dQ tile
-  static constexpr int oLo = oHi + 2 * kChunk;   // bf16 of the remainder
-  static constexpr int oVec = oLo + 2 * kChunk;  // LSE*log2e [128], Delta [128]
+  static constexpr int oRing = oV + kTile;               // 4 slots of (Q_h, dO_h)
+  static constexpr int kSlot = 2 * kHalf;
+  static constexpr int oVec = oRing + 4 * kSlot;         // [2][128] floats: LSE*log2e [64], Delta [64]
   static constexpr int oBar = oVec + 1024;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-// the 128 threads of compute warpgroup g
-__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    const __grid_constant__ CUtensorMap tmDQ,
-                    const float* __restrict__ LSE, const float* __restrict__ Delta,
-                    float* __restrict__ dK, float* __restrict__ dV, int* errw, int S, float scale_log2,
-                    float scale) {
-  using Lay = BwdSmem<D>;
+    attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOh,
+                       const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dK,
+                       float* __restrict__ dV, int* errw, int S, float scale_log2, float scale) {
+  using Lay = KvSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
-  uint64_t* bKV = bars + 0;      // K, V landed
-  uint64_t* bQ = bars + 1;       // Q_i landed
-  uint64_t* bQfree = bars + 2;   // dK product of tile i done: Q buffer free
-  uint64_t* bO = bars + 7;       // dO_i landed
-  uint64_t* bOfree = bars + 8;   // dV product of tile i done: dO buffer free
-  uint64_t* bSdP = bars + 3;     // S^T and dP^T of tile i in TMEM
-  uint64_t* bPS = bars + 4;      // P^T in TMEM and dS^T in shared memory (256 arrivals)
-  uint64_t* bDQ = bars + 5;      // dQ of tile i in TMEM (all products of tile i done)
-  uint64_t* bDQfree = bars + 6;  // dQ read out of TMEM (256 arrivals)
+  uint64_t* bKV = bars + 0;        // K, V landed
+  uint64_t* bLoad = bars + 1;      // [4] Q_h, dO_h of a ring slot landed
+  uint64_t* bSlotFree = bars + 5;  // [4] dV, dK products done with a slot
+  uint64_t* bF = bars + 9;         // [2] S^T, dP^T of a half step in TMEM buffer
+  uint64_t* bPS = bars + 11;       // [2] P^T, dS^T written back (256 arrivals)
+  uint64_t* bDone = bars + 13;     // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
-  float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);  // [0,128) LSE*log2e, [128,256) Delta
+  float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = (S + BM - 1) / BM;
+  const int n_qt = (S + 127) / 128;
   const int kt = (int)blockIdx.x;  // key tile; small kt = most query tiles, launched first
   const int bh = (int)blockIdx.y;
-  const int n_q = n_qt - kt;
+  const int NS = 2 * (n_qt - kt);  // half steps
 
   if (threadIdx.x == 0) {
     mbar_init(bKV, 1);
-    mbar_init(bQ, 1);
-    mbar_init(bQfree, 1);
-    mbar_init(bO, 1);
-    mbar_init(bOfree, 1);
-    mbar_init(bSdP, 1);
-    mbar_init(bPS, kCompute);
-    mbar_init(bDQ, 1);
-    mbar_init(bDQfree, kCompute);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bLoad[i], 1);
+      mbar_init(&bSlotFree[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bF[i], 1);
+      mbar_init(&bPS[i], kCompute);
+    }
+    mbar_init(bDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -111,210 +115,148 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
+  constexpr uint32_t tSP = 0, tDP = 128, tDV = 256, tDK = 256 + D;  // SP/DP: [2] x 64 columns
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmO);
-      mbar_expect_tx(bKV, 2 * BN * D * 2);
+      tma_prefetch_desc(&tmQh);
+      tma_prefetch_desc(&tmOh);
+      mbar_expect_tx(bKV, 2 * 128 * D * 2);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem + Lay::oK + c * Lay::kChunk, &tmK, bKV, c * 64, kt * BN, bh);
-        tma_load_3d(smem + Lay::oV + c * Lay::kChunk, &tmV, bKV, c * 64, kt * BN, bh);
+        tma_load_3d(smem + Lay::oK + c * kRegion, &tmK, bKV, c * 64, kt * 128, bh);
+        tma_load_3d(smem + Lay::oV + c * kRegion, &tmV, bKV, c * 64, kt * 128, bh);
       }
-      // Q is released by the dK product and dO by the dV product of the
-      // previous tile; each reloads as soon as its buffer is free
-      for (int it = 0; it < n_q; ++it) {
-        const int i = kt + it;
-        if (it >= 1 && !mbar_wait(bQfree, (it - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bQ, BM * D * 2);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oQ + c * Lay::kChunk, &tmQ, bQ, c * 64, i * BM, bh);
-        if (it >= 1 && !mbar_wait(bOfree, (it - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bO, BM * D * 2);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oO + c * Lay::kChunk, &tmO, bO, c * 64, i * BM, bh);
+      for (int s = 0; s < NS; ++s) {
+        const int slot = s & 3;
+        if (s >= 4 && !mbar_wait(&bSlotFree[slot], ((s >> 2) - 1) & 1, abort_flag)) break;
+        const int q0 = (kt + (s >> 1)) * 128 + (s & 1) * 64;
+        uint8_t* base = smem + Lay::oRing + slot * Lay::kSlot;
+        mbar_expect_tx(&bLoad[slot], 2 * 64 * D * 2);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + c * kHalfRegion, &tmQh, &bLoad[slot], c * 64, q0, bh);
+          tma_load_3d(base + Lay::kHalf + c * kHalfRegion, &tmOh, &bLoad[slot], c * 64, q0, bh);
+        }
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idSS = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idKM = idesc_bf16(128, D, false, true);  // A K-major, B MN-major
-      constexpr uint32_t idMM = idesc_bf16(128, D, true, true);   // A MN-major, B MN-major
-      const uint32_t sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
-      const uint32_t sQ = smem_u32(smem + Lay::oQ), sO = smem_u32(smem + Lay::oO);
-      const uint32_t sHi = smem_u32(smem + Lay::oHi), sLo = smem_u32(smem + Lay::oLo);
-      // base descriptors: an operand at byte offset off is base + (off >> 4)
-      const uint64_t kK = sdesc_sw128(sK, 16, 1024), kQ = sdesc_sw128(sQ, 16, 1024);
-      const uint64_t kV = sdesc_sw128(sV, 16, 1024), kO = sdesc_sw128(sO, 16, 1024);
-      const uint64_t kHi = sdesc_sw128(sHi, 16, 1024), kLo = sdesc_sw128(sLo, 16, 1024);
-      const uint64_t mO = sdesc_sw128(sO, Lay::kChunk, 1024), mQ = sdesc_sw128(sQ, Lay::kChunk, 1024);
-      const uint64_t mK = sdesc_sw128(sK, Lay::kChunk, 1024);
-      const uint64_t mHi = sdesc_sw128(sHi, Lay::kChunk, 1024), mLo = sdesc_sw128(sLo, Lay::kChunk, 1024);
-      bool ok = mbar_wait(bKV, 0, abort_flag);
-      for (int it = 0; ok && it < n_q; ++it) {
-        if (!mbar_wait(bQ, it & 1, abort_flag)) break;
+    {  // the whole warp; one elected lane issues each instruction
+      constexpr uint32_t idF = idesc_bf16(128, 64, false, false);  // S^T, dP^T: N = 64 queries
+      constexpr uint32_t idG = idesc_bf16(128, D, false, true);    // dV, dK: A from TMEM, B MN-major
+      const uint32_t sRing = smem_u32(smem + Lay::oRing);
+      const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
+      const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
+      const uint64_t kRing = sdesc_sw128(sRing, 16, 1024);
+      const uint64_t mRing = sdesc_sw128(sRing, kHalfRegion, 1024);
+      bool ok = mbar_wait_warp(bKV, 0, abort_flag);
+      // the loads of half step s landed (waited for before the products that
+      // precede its F in the issue order, so no wait sits between them)
+      auto wait_f = [&](int s) -> bool { return mbar_wait_warp(&bLoad[s & 3], (s >> 2) & 1, abort_flag); };
+      auto issue_f = [&](int s) {
+        const int slot = s & 3, b = s & 1;
         tc_fence_after();
-        // S^T = K Q^T  (M = keys, N = queries, K = d); the S^T columns held P^T of
-        // the previous tile, whose dV product was issued before this one
+        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
-          umma_bf16(tmem + tS, kK + off, kQ + off, idSS, kk > 0 ? 1u : 0u);
+          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // K, V tile (128 rows)
+          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // Q_h, dO_h (64 rows)
+          umma_bf16_w(tmem + tSP + b * 64, kK + at, kRing + qo + bt, idF, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + tDP + b * 64, kV + at, kRing + oo + bt, idF, kk > 0 ? 1u : 0u);
         }
-        // dP^T = V dO^T into the dQ columns, once dO has landed and the previous
-        // dQ has been read out
-        if (!mbar_wait(bO, it & 1, abort_flag)) break;
-        if (it >= 1 && !mbar_wait(bDQfree, (it - 1) & 1, abort_flag)) break;
+        umma_commit_w(&bF[b]);
+      };
+      if (ok && (ok = wait_f(0))) issue_f(0);
+      if (ok && NS > 1 && (ok = wait_f(1))) issue_f(1);
+      for (int s = 0; ok && s < NS; ++s) {
+        const int slot = s & 3, b = s & 1;
+        if (s + 2 < NS && !wait_f(s + 2)) { ok = false; break; }
+        if (!mbar_wait_warp(&bPS[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
-          umma_bf16(tmem + tDP, kV + off, kO + off, idSS, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; hi of chunk kk/2 at +(kk&1)*8, lo at +16
+          const uint32_t a = (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t bq = (kk * 2048) >> 4;
+          umma_bf16_tmem_a_w(tmem + tDV, tmem + tSP + b * 64 + a, mRing + oo + bq, idG, acc);
+          umma_bf16_tmem_a_w(tmem + tDV, tmem + tSP + b * 64 + a + 16, mRing + oo + bq, idG, 1u);
+          umma_bf16_tmem_a_w(tmem + tDK, tmem + tDP + b * 64 + a, mRing + qo + bq, idG, acc);
+          umma_bf16_tmem_a_w(tmem + tDK, tmem + tDP + b * 64 + a + 16, mRing + qo + bq, idG, 1u);
         }
-        umma_commit(bSdP);
-        if (!mbar_wait(bPS, it & 1, abort_flag)) break;
-        tc_fence_after();
-        // dK += dS^T Q: A = dS^T (hi, lo) K-major from shared memory; then Q is free
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t aoff = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
-          const uint64_t b = mQ + ((kk * 2048) >> 4);
-          umma_bf16(tmem + tDK, kHi + aoff, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16(tmem + tDK, kLo + aoff, b, idKM, 1u);
-        }
-        umma_commit(bQfree);
-        // dV += P^T dO: A = P^T (hi, lo) from TMEM, B = dO MN-major (K = queries); then dO is free
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint64_t b = mO + ((kk * 2048) >> 4);
-          umma_bf16_tmem_a(tmem + tDV, a, b, idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16_tmem_a(tmem + tDV, a + 16, b, idKM, 1u);
-        }
-        umma_commit(bOfree);
-        // dQ = dS K  (M = queries, K = keys, N = d): dS^T read M-major
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t off = (kk * 2048) >> 4;
-          umma_bf16(tmem + tDP, mHi + off, mK + off, idMM, kk > 0 ? 1u : 0u);
-          umma_bf16(tmem + tDP, mLo + off, mK + off, idMM, 1u);
-        }
-        umma_commit(bDQ);
+        umma_commit_w(&bSlotFree[slot]);
+        // the next half step that uses this TMEM buffer; its S^T, dP^T land
+        // after the products above have read P^T and dS^T (in-order issue)
+        if (s + 2 < NS) issue_f(s + 2);
       }
+      if (ok) umma_commit_w(bDone);
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
     const int ct = threadIdx.x;            // 0..255
-    const int g = warp >> 2;               // warpgroup: query columns [64g, 64g+64)
+    const int g = warp >> 2;               // query columns [32g, 32g+32) of each half
     const int t = (warp & 3) * 32 + lane;  // key row of the tile (TMEM lane)
-    const int kv_g = kt * BN + t;
+    const int kv_g = kt * 128 + t;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    uint8_t* sHib = smem + Lay::oHi;
-    uint8_t* sLob = smem + Lay::oLo;
     bool ok = true;
-    // LSE (ct < 128) or Delta (ct >= 128) of one query row of the tile at q0
-    auto vec_of = [&](int q0) -> float {
-      const int qg = q0 + (ct & 127);
-      if (ct < 128) return qg < S ? LSE[(int64_t)bh * S + qg] * 1.4426950408889634f : INFINITY;
-      return qg < S ? Delta[(int64_t)bh * S + qg] : 0.f;
+    // LSE (ct < 64) or Delta (64 <= ct < 128) of query row ct & 63 of half
+    // step s, loaded one half step ahead and converted when it is stored
+    auto vec_row = [&](int s) { return (kt + (s >> 1)) * 128 + (s & 1) * 64 + (ct & 63); };
+    auto vec_raw = [&](int s) -> float {
+      const int qg = vec_row(s);
+      return qg < S ? ldg_nc_f32((ct < 64 ? LSE : Delta) + (int64_t)bh * S + qg) : 0.f;
     };
-    float vec_next = vec_of(kt * BM);
-    for (int it = 0; it < n_q; ++it) {
-      const int q0 = (kt + it) * BM;
+    float vec_next = ct < 128 ? vec_raw(0) : 0.f;
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
+    for (int s = 0; s < NS; ++s) {
+      const int b = s & 1;
       const float vec_cur = vec_next;
-      if (it + 1 < n_q) vec_next = vec_of(q0 + BM);  // one tile ahead
-      compute_sync();  // every thread is done with the previous tile's LSE / Delta
-      sVec[ct] = vec_cur;
+      if (ct < 128 && s + 1 < NS) vec_next = vec_raw(s + 1);
+      if (ct < 64) sVec[b * 128 + ct] = vec_row(s) < S ? vec_cur * 1.4426950408889634f : INFINITY;
+      else if (ct < 128) sVec[b * 128 + ct] = vec_cur;
       compute_sync();
-      if (!mbar_wait(bSdP, it & 1, abort_flag)) { ok = false; break; }
-      __syncwarp();
+      const float* lse = sVec + b * 128;
+      const float* del = lse + 64;
+      const int q0 = (kt + (s >> 1)) * 128 + (s & 1) * 64;
+      const bool diag = (s >> 1) == 0;  // the diagonal query tile
+      // warp-uniform outcome for the collective TMEM accesses; after a failed
+      // wait the loop keeps its compute_sync count and skips the work
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bF[b], (s >> 1) & 1, abort_flag));
+      if (!ok) continue;
       tc_fence_after();
-      const bool diag = (it == 0);
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * g + cc;  // 32-column chunk of the tile
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tl + tS + c * 32, sr);
-        tmem_ld32(tl + tDP + c * 32, dr);
-        tmem_ld_wait();
-        uint32_t phi[16], plo[16], dhi[16], dlo[16];
-        const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tl + tSP + b * 64 + g * 32, sr);
+      tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
+      tmem_ld_wait();
+      uint32_t phi[16], plo[16], dhi[16], dlo[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int qi = c * 32 + e;
-          const float2 lse2 = *reinterpret_cast<const float2*>(sVec + qi);
-          const float2 del2 = *reinterpret_cast<const float2*>(sVec + 128 + qi);
-          float pa, pb;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-lse2.x, -lse2.y)),
-                    pa, pb);
-          pa = fast_exp2(pa);
-          pb = fast_exp2(pb);
-          if (diag) {
-            if (q0 + qi < kv_g) pa = 0.f;
-            if (q0 + qi + 1 < kv_g) pb = 0.f;
-          }
-          const uint64_t p2 = f2_pack(pa, pb);
-          const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(del2.x, del2.y));
-          float da, db;
-          f2_unpack(f2_mul(f2_mul(p2, sc2), diff2), da, db);
-          split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
-          split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+      for (int e = 0; e < 32; e += 2) {
+        const int qi = g * 32 + e;
+        const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
+        const float2 d2 = *reinterpret_cast<const float2*>(del + qi);
+        float pa, pb;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)), pa,
+                  pb);
+        pa = fast_exp2(pa);
+        pb = fast_exp2(pb);
+        if (diag) {
+          if (q0 + qi < kv_g) pa = 0.f;
+          if (q0 + qi + 1 < kv_g) pb = 0.f;
         }
-        // P^T over the S^T columns just read: hi in the first 16, lo in the last 16
-        tmem_st16(tl + tS + c * 32, phi);
-        tmem_st16(tl + tS + c * 32 + 16, plo);
-        if (cc == 0) {
-          // this group's previous dQ reduce must have read the regions it reuses
-          if (t == 0) bulk_wait_read_all();
-          group_sync(g);
-        }
-        // dS^T row t, query columns c*32..c*32+31: 4 chunks of 16 bytes in region c/2 = g
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = (c & 1) * 4 + q;
-          const int off = (c >> 1) * Lay::kChunk + t * 128 + ((ch ^ (t & 7)) << 4);
-          *reinterpret_cast<uint4*>(sHib + off) = make_uint4(dhi[4 * q], dhi[4 * q + 1], dhi[4 * q + 2], dhi[4 * q + 3]);
-          *reinterpret_cast<uint4*>(sLob + off) = make_uint4(dlo[4 * q], dlo[4 * q + 1], dlo[4 * q + 2], dlo[4 * q + 3]);
-        }
+        const uint64_t p2 = f2_pack(pa, pb);
+        const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(d2.x, d2.y));
+        float da, db;
+        f2_unpack(f2_mul(f2_mul(p2, sc2), diff2), da, db);
+        split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
+        split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
       }
+      store_pair_chunk(tl + tSP + b * 64 + g * 32, phi, plo);
+      store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
       tmem_st_wait();
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bPS);
-      // dQ of query row q0 + t, columns [D/2 g, D/2 (g+1)): TMEM -> shared memory,
-      // into the two regions (hi and lo, region g) that this group's dS writes
-      // use, then one TMA reduce-add per 32-column chunk into dQs, issued by
-      // the group; the dS buffers are free once the dQ product is done
-      if (!mbar_wait(bDQ, it & 1, abort_flag)) { ok = false; break; }
-      __syncwarp();
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = g * (D / 2) + c * 32;
-        uint32_t r[32];
-        tmem_ld32(tl + tDP + col, r);
-        tmem_ld_wait();
-        uint8_t* dst = smem + (c == 0 ? Lay::oHi : Lay::oLo) + g * (128 * 128) + t * 128;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(dst + ((k ^ (t & 7)) << 4)) = make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
-      }
-      tc_fence_before();
-      mbar_arrive(bDQfree);
-      fence_proxy_async_smem();
-      group_sync(g);
-      if (t == 0) {
-        for (int c = 0; c < D / 64; ++c)
-          tma_reduce_add_3d(&tmDQ, smem + (c == 0 ? Lay::oHi : Lay::oLo) + g * (128 * 128), g * (D / 2) + c * 32, q0, bh);
-        bulk_commit_group();
-      }
+      mbar_arrive(&bPS[b]);
     }
-    if (ok && !*abort_flag) {
-      // bDQ of the last tile has completed: dV and dK are final
-      __syncwarp();
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
@@ -337,7 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  if (threadIdx.x == 0 || threadIdx.x == 128) bulk_wait_all();  // every dQ reduce has landed
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
@@ -347,33 +288,255 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) report_error(errw, ERRW_TIMEOUT);
 }
 
+// ===========================================================================
+// dQs
+// ===========================================================================
+template <int D>
+struct QSmem {
+  static constexpr int kTile = D / 64 * kRegion;      // Q or dO tile, 128 rows
+  static constexpr int kHalf = D / 64 * kHalfRegion;  // K_h or V_h, 64 rows
+  static constexpr int oQ = 0;
+  static constexpr int oO = oQ + kTile;     // dO
+  static constexpr int oK = oO + kTile;     // 4 slots of K_h
+  static constexpr int oV = oK + 4 * kHalf; // 4 slots of V_h
+  static constexpr int oBar = oV + 4 * kHalf;
+  static constexpr int kBytes = oBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKh,
+                      const __grid_constant__ CUtensorMap tmVh, const __grid_constant__ CUtensorMap tmO,
+                      const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dQ,
+                      int* errw, int S, float scale_log2, float scale) {
+  using Lay = QSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
+  uint64_t* bQO = bars + 0;     // Q, dO landed
+  uint64_t* bK = bars + 1;      // [4] K_h of a slot landed
+  uint64_t* bV = bars + 5;      // [4] V_h of a slot landed
+  uint64_t* bKfree = bars + 9;  // [4] the dQ product is done with K_h
+  uint64_t* bVfree = bars + 13; // [4] the dP product is done with V_h
+  uint64_t* bF = bars + 17;     // [2] S, dP of a half step in TMEM buffer
+  uint64_t* bPS = bars + 19;    // [2] dS written back (256 arrivals)
+  uint64_t* bDone = bars + 21;  // every product done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = (S + 127) / 128;
+  const int qt = n_qt - 1 - (int)blockIdx.x;  // longest rows first
+  const int bh = (int)blockIdx.y;
+  const int NU = 2 * (qt + 1);  // 64-key half steps up to the diagonal
+
+  if (threadIdx.x == 0) {
+    mbar_init(bQO, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bK[i], 1);
+      mbar_init(&bV[i], 1);
+      mbar_init(&bKfree[i], 1);
+      mbar_init(&bVfree[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bF[i], 1);
+      mbar_init(&bPS[i], kCompute);
+    }
+    mbar_init(bDone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;  // S, dP: [2] x 64 columns
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    // K_h and V_h of half step u go to slot u & 3; V_h is released by the dP
+    // product of its half step, K_h by the dQ product, so each reloads as
+    // soon as its last reader is done
+    if (lane == 0) {
+      tma_prefetch_desc(&tmKh);
+      tma_prefetch_desc(&tmVh);
+      mbar_expect_tx(bQO, 2 * 128 * D * 2);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(smem + Lay::oQ + c * kRegion, &tmQ, bQO, c * 64, qt * 128, bh);
+        tma_load_3d(smem + Lay::oO + c * kRegion, &tmO, bQO, c * 64, qt * 128, bh);
+      }
+      for (int u = 0; u < NU; ++u) {
+        const int slot = u & 3, k0 = u * 64;
+        const uint32_t par = ((u >> 2) - 1) & 1;
+        if (u >= 4 && !mbar_wait(&bVfree[slot], par, abort_flag)) break;
+        mbar_expect_tx(&bV[slot], 64 * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oV + slot * Lay::kHalf + c * kHalfRegion, &tmVh, &bV[slot], c * 64, k0, bh);
+        if (u >= 4 && !mbar_wait(&bKfree[slot], par, abort_flag)) break;
+        mbar_expect_tx(&bK[slot], 64 * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oK + slot * Lay::kHalf + c * kHalfRegion, &tmKh, &bK[slot], c * 64, k0, bh);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    {  // the whole warp; one elected lane issues each instruction
+      constexpr uint32_t idF = idesc_bf16(128, 64, false, false);  // S, dP: N = 64 keys
+      constexpr uint32_t idG = idesc_bf16(128, D, false, true);    // dQ: A from TMEM, B MN-major
+      const uint64_t kQ = sdesc_sw128(smem_u32(smem + Lay::oQ), 16, 1024);
+      const uint64_t kO = sdesc_sw128(smem_u32(smem + Lay::oO), 16, 1024);
+      const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
+      const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
+      const uint64_t mK = sdesc_sw128(smem_u32(smem + Lay::oK), kHalfRegion, 1024);
+      bool ok = mbar_wait_warp(bQO, 0, abort_flag);
+      auto wait_f = [&](int u) -> bool {
+        return mbar_wait_warp(&bK[u & 3], (u >> 2) & 1, abort_flag) && mbar_wait_warp(&bV[u & 3], (u >> 2) & 1, abort_flag);
+      };
+      auto issue_f = [&](int u) {
+        const int slot = u & 3, b = u & 1;
+        tc_fence_after();
+        const uint32_t so = (slot * Lay::kHalf) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qoff = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;      // Q, dO (128 rows)
+          const uint32_t hoff = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // K_h, V_h (64 rows)
+          umma_bf16_w(tmem + tS + b * 64, kQ + qoff, kK + so + hoff, idF, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + tDP + b * 64, kO + qoff, kV + so + hoff, idF, kk > 0 ? 1u : 0u);
+        }
+        umma_commit_w(&bVfree[slot]);
+        umma_commit_w(&bF[b]);
+      };
+      if (ok && (ok = wait_f(0))) issue_f(0);
+      if (ok && NU > 1 && (ok = wait_f(1))) issue_f(1);
+      for (int u = 0; ok && u < NU; ++u) {
+        const int slot = u & 3, b = u & 1;
+        if (u + 2 < NU && !wait_f(u + 2)) { ok = false; break; }
+        if (!mbar_wait_warp(&bPS[b], (u >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t mk = mK + ((slot * Lay::kHalf) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 keys per step
+          const uint32_t a = tmem + tDP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint64_t bk = mk + ((kk * 2048) >> 4);
+          umma_bf16_tmem_a_w(tmem + tDQ, a, bk, idG, (u > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a_w(tmem + tDQ, a + 16, bk, idG, 1u);
+        }
+        umma_commit_w(&bKfree[slot]);
+        if (u + 2 < NU) issue_f(u + 2);
+      }
+      if (ok) umma_commit_w(bDone);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warpgroups
+    const int g = warp >> 2;               // key columns [32g, 32g+32) of each half
+    const int t = (warp & 3) * 32 + lane;  // query row of the tile (TMEM lane)
+    const int qg = qt * 128 + t;
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float lse = qg < S ? LSE[(int64_t)bh * S + qg] * 1.4426950408889634f : INFINITY;
+    const float del = qg < S ? Delta[(int64_t)bh * S + qg] : 0.f;
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
+    const uint64_t nl2 = f2_pack(-lse, -lse), d2 = f2_pack(del, del);
+    bool ok = true;
+    for (int u = 0; u < NU; ++u) {
+      const int b = u & 1;
+      const int k0 = (u >> 1) * 128 + (u & 1) * 64 + g * 32;  // first key of this thread's chunk
+      const bool diag = (u >> 1) == qt;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bF[b], (u >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tl + tS + b * 64 + g * 32, sr);
+      tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
+      tmem_ld_wait();
+      uint32_t dhi[16], dlo[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        float pa, pb;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nl2), pa, pb);
+        pa = fast_exp2(pa);
+        pb = fast_exp2(pb);
+        if (diag) {
+          if (k0 + e > qg) pa = 0.f;
+          if (k0 + e + 1 > qg) pb = 0.f;
+        }
+        const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), d2);
+        float da, db;
+        f2_unpack(f2_mul(f2_mul(f2_pack(pa, pb), sc2), diff2), da, db);
+        split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+      }
+      store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bPS[b]);
+    }
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = g * (D / 2) + c * 32;
+        uint32_t r[32];
+        tmem_ld32(tl + tDQ + col, r);
+        tmem_ld_wait();
+        if (qg < S) {
+          float4* dq4 = reinterpret_cast<float4*>(dQ + ((int64_t)bh * S + qg) * D + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dq4[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                                 __uint_as_float(r[4 * q + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report_error(errw, ERRW_TIMEOUT);
+}
+
+// TMA maps of the sequences: full 128-row boxes and 64-row half boxes
+struct SeqMaps {
+  CUtensorMap q, qh, kh, k, v, vh, o, oh;
+};
+
+template <int D>
+cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* lse, const float* delta, float* dqs,
+                         float* dks, float* dvs, int* errw, float scale_log2, float scale, cudaStream_t st) {
+  const unsigned n_qt = (unsigned)((S + 127) / 128);
+  int smem = KvSmem<D>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.qh, m.k, m.v, m.oh, lse, delta, dks, dvs,
+                                                                         errw, (int)S, scale_log2, scale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  smem = QSmem<D>::kAlloc;
+  e = cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_bwd_q_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.kh, m.vh, m.o, lse, delta, dqs, errw,
+                                                                        (int)S, scale_log2, scale);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
                             float* dvs, int* errw, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo, mdq;
-  if (!make_seq_map(&mq, qs, BH, S, d, BM) || !make_seq_map(&mk, ks, BH, S, d, BN) ||
-      !make_seq_map(&mv, vs, BH, S, d, BN) || !make_seq_map(&mo, dos, BH, S, d, BM) ||
-      !make_f32_map(&mdq, dqs, BH, S, d, BM))
+  SeqMaps m;
+  if (!make_seq_map(&m.q, qs, BH, S, d, 128) || !make_seq_map(&m.qh, qs, BH, S, d, 64) ||
+      !make_seq_map(&m.k, ks, BH, S, d, 128) || !make_seq_map(&m.kh, ks, BH, S, d, 64) ||
+      !make_seq_map(&m.v, vs, BH, S, d, 128) || !make_seq_map(&m.vh, vs, BH, S, d, 64) ||
+      !make_seq_map(&m.o, dos, BH, S, d, 128) || !make_seq_map(&m.oh, dos, BH, S, d, 64))
     return cudaErrorInvalidValue;
   const double scale = 1.0 / sqrt((double)d);
   const float scale_log2 = (float)(1.4426950408889634 * scale);
-  const dim3 grid((unsigned)((S + BN - 1) / BN), (unsigned)BH);
-  if (d == 128) {
-    const int smem = BwdSmem<128>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_bwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mdq, lse, delta, dks, dvs, errw, (int)S,
-                                                        scale_log2, (float)scale);
-  } else {
-    const int smem = BwdSmem<64>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_bwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, mo, mdq, lse, delta, dks, dvs, errw, (int)S,
-                                                       scale_log2, (float)scale);
-  }
-  return cudaGetLastError();
+  if (d == 128) return launch_bwd_d<128>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st);
+  return launch_bwd_d<64>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st);
 }
 
 }  // namespace lh

@@ -12,9 +12,10 @@
 //              it came from as a bf16 pair (per 32 keys: 16 columns of hi,
 //              16 of lo), where the P V product reads it
 //   warp 8     TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
-//   warp 9     MMA issuer (one thread): for each key tile, P_A V, then the next
-//              S_A = Q_A K^T, then P_B V and the next S_B, so the tensor core
-//              works on one tile while the other tile's softmax runs
+//   warp 9     MMA issuer (the converged warp; one elected lane issues):
+//              for each key tile, P_A V, then the next S_A = Q_A K^T, then
+//              P_B V and the next S_B, so the tensor core works on one tile
+//              while the other tile's softmax runs
 // TMEM columns: S_A/P_A [0,128), S_B/P_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 // The P pair keeps P V at fp32 accuracy; O is written in fp32.
 #include <cudaTypedefs.h>
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp; one elected lane issues each instruction
       constexpr uint32_t idQK = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idPV = idesc_bf16(BM, D, false, true);
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sK = smem_u32(smem + Lay::oK), sV = smem_u32(smem + Lay::oV);
@@ -126,11 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * Lay::kChunk + (kk & 3) * 32) >> 4;
-          umma_bf16(tmem + x * 128, qb + off, kb + off, idQK, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + x * 128, qb + off, kb + off, idQK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bS[x]);
+        umma_commit_w(&bS[x]);
       };
-      bool ok = mbar_wait(bQ, 0, abort_flag) && mbar_wait(&bK[0], 0, abort_flag);
+      bool ok = mbar_wait_warp(bQ, 0, abort_flag) && mbar_wait_warp(&bK[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -141,9 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool v_ready = false, k_next_ready = false;
         for (int x = 0; x < 2 && ok; ++x) {
           if (j > last[x]) continue;
-          if (!mbar_wait(&bP[x], j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bP[x], j & 1, abort_flag)) { ok = false; break; }
           if (!v_ready) {
-            if (!mbar_wait(&bV[st], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(&bV[st], (j >> 1) & 1, abort_flag)) { ok = false; break; }
             v_ready = true;
           }
           tc_fence_after();
@@ -153,20 +154,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t b = vb + ((kk * 2048) >> 4);
             const uint32_t a = pa + (kk >> 1) * 32 + (kk & 1) * 8;  // hi of keys 16kk..16kk+15
-            umma_bf16_tmem_a(tmem + 256 + x * D, a, b, idPV, (j > 0 || kk > 0) ? 1u : 0u);
-            umma_bf16_tmem_a(tmem + 256 + x * D, a + 16, b, idPV, 1u);
+            umma_bf16_tmem_a_w(tmem + 256 + x * D, a, b, idPV, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_tmem_a_w(tmem + 256 + x * D, a + 16, b, idPV, 1u);
           }
-          umma_commit(&bO[x]);
+          umma_commit_w(&bO[x]);
           if (j + 1 <= last[x]) {
             if (!k_next_ready) {
-              if (!mbar_wait(&bK[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait_warp(&bK[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
               k_next_ready = true;
               tc_fence_after();
             }
             issue_s(x, j + 1);  // after P V of this tile: the S columns hold P until then
           }
         }
-        if (ok) umma_commit(&bKVfree[st]);
+        if (ok) umma_commit_w(&bKVfree[st]);
       }
     }
   } else {

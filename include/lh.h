@@ -185,7 +185,7 @@ lh_status lh_attn_fwd(const lh_config *cfg, int64_t S, const void *qs, const voi
  * hi + lo pairs, so dQs, dKs, dVs keep fp32 accuracy for bf16 inputs.
  * In:  qs, ks, vs, lse from the forward; dos [BH][S][d] bf16 and
  *      delta [BH][S] fp32 (rowsum(dOs * Os)) from lh_scatter_back_adjoint.
- * Out: dqs, dks, dvs [BH][S][d] fp32 (dqs is zeroed and accumulated here).
+ * Out: dqs, dks, dvs [BH][S][d] fp32, each row written once (no accumulation).
  * ws: at least attn_bwd_ws_bytes (error word). */
 lh_status lh_attn_bwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs,
                       const float *lse, const void *dos, const float *delta, float *dqs, float *dks, float *dvs,
