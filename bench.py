@@ -38,6 +38,11 @@ METRIC = "Lighthouse attn fwd+bwd tokens/s/layer at N=512K on 1 B200; % of roofl
 UNIT = "tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+# the kernels each stage entry point launches (names as the ncu launch list shows them)
+STAGE_KERNELS = {"pool": ["pool_kernel"], "score_topk": ["score_pyramid_kernel", "topk_kernel"],
+                 "gather": ["gather_kernel"], "attn_fwd": ["attn_fwd_kernel"], "scatter_back": ["scatter_back_kernel"],
+                 "scatter_adjoint": ["scatter_adjoint_kernel"], "attn_bwd": ["attn_bwd_kv_kernel", "attn_bwd_q_kernel"],
+                 "pool_adjoint": ["pool_adjoint_kernel"]}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -145,8 +150,9 @@ def _vp(base: int, off: int = 0):
 
 
 def stage_calls(layer: lh.Layer, bufs: lh.Buffers, x: dict, y, grads):
-    """The eight stage entry points in lh_forward/lh_backward order, on the
-    same buffers, so each can be timed alone."""
+    """The eight stage entry points in lh_forward/lh_backward order, with the
+    arguments lh_forward uses (the pool and gather at the plan's first_level),
+    on the same buffers, so each kernel of the step can be timed alone."""
     I = bufs.info
     cfg = layer.cfg()
     c = bufs.ctx.data_ptr()
@@ -155,13 +161,16 @@ def stage_calls(layer: lh.Layer, bufs: lh.Buffers, x: dict, y, grads):
     dq, dk, dv = (g.data_ptr() for g in grads)
     st = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)  # noqa: E731
     S = ctypes.c_int64(I.S)
+    first = ctypes.c_int32(I.first_level)  # the levels lh_forward materialises
     call = _lib.call
     return [
-        ("pool", lambda: call("lh_pyramid_pool", ctypes.byref(cfg), _vp(q), _vp(k), _vp(v), _vp(w, I.ws_off_pyr_q),
-                              _vp(w, I.ws_off_pyr_k), _vp(w, I.ws_off_pyr_v), _vp(w, I.ws_off_norms), st())),
+        ("pool", lambda: call("lh_pyramid_pool_from", ctypes.byref(cfg), first, _vp(q), _vp(k), _vp(v),
+                              _vp(w, I.ws_off_pyr_q), _vp(w, I.ws_off_pyr_k), _vp(w, I.ws_off_pyr_v),
+                              _vp(w, I.ws_off_norms), st())),
         ("score_topk", lambda: call("lh_score_topk", ctypes.byref(cfg), _vp(w, I.ws_off_norms), _vp(w, I.ws_off_topk),
                                     _vp(c, I.ctx_off_sel), st())),
-        ("gather", lambda: call("lh_gather", ctypes.byref(cfg), _vp(q), _vp(k), _vp(v), _vp(w, I.ws_off_pyr_q),
+        ("gather", lambda: call("lh_gather_from", ctypes.byref(cfg), first, _vp(q), _vp(k), _vp(v),
+                                _vp(w, I.ws_off_pyr_q),
                                 _vp(w, I.ws_off_pyr_k), _vp(w, I.ws_off_pyr_v), _vp(c, I.ctx_off_sel),
                                 _vp(c, I.ctx_off_qs), _vp(c, I.ctx_off_ks), _vp(c, I.ctx_off_vs),
                                 _vp(c, I.ctx_off_seq_map), _vp(c, I.ctx_off_slot_of), st())),
@@ -186,10 +195,16 @@ def stage_work(layer: lh.Layer, info) -> dict:
     e = 2 if layer.dtype == "bf16" else 4
     BH, N, d, S = layer.BH, layer.N, layer.d, info.S
     U, E = info.upper_entries, info.pyr_entries
+    L, p, first = layer.L, layer.p, info.first_level
+    # pyramid rows the pool writes (levels >= first) and rows the gather reads:
+    # a kept entry of a level below first is the mean of its p^l level-0 rows
+    U_first = sum(info.level_len[lvl] for lvl in range(first, L)) if L > 1 else 0
+    kept = [p * info.kprime[lvl] for lvl in range(L - 1)] + [info.level_len[L - 1]] if L > 1 else [N]
+    read_rows = sum(n * (p ** lvl if 1 <= lvl < first else 1) for lvl, n in enumerate(kept))
     return {
-        "pool": ("hbm", 3 * BH * N * d * e + 3 * BH * U * d * e + 2 * BH * N * 4),
+        "pool": ("hbm", 3 * BH * N * d * e + 3 * BH * U_first * d * e + 2 * BH * N * 4),
         "score_topk": ("hbm", 2 * BH * N * 4 + 2 * BH * U * 4 + BH * info.sel_per_head * 4),
-        "gather": ("hbm", 3 * BH * S * d * (e + 2) + BH * S * 4 + BH * E * 4),
+        "gather": ("hbm", 3 * BH * read_rows * d * e + 3 * BH * S * d * 2 + BH * S * 4 + BH * E * 4),
         "attn_fwd": ("tensor", 2 * S * S * d * BH),
         "scatter_back": ("hbm", BH * N * d * e + BH * S * d * 2 + BH * E * 4),
         "scatter_adjoint": ("hbm", BH * N * d * e + 2 * BH * S * d * 2 + BH * S * 8),
@@ -377,7 +392,7 @@ def main():
                          "frac": ach / pk["bf16_tflops"]}
     top = max(stage_ms, key=stage_ms.get)
     ts = stages[top]
-    roofline = {"bound": ts["bound"], "kernel": top, "achieved": ts["achieved"],
+    roofline = {"bound": ts["bound"], "kernel": top, "kernels": STAGE_KERNELS[top], "achieved": ts["achieved"],
                 "peak": pk["hbm_gbs"] if ts["bound"] == "hbm" else pk["bf16_tflops"], "unit": ts["unit"],
                 "frac": ts["frac"], "traffic": measured_traffic(top, w.name), "peak_source": pk_src,
                 "share_of_step": stage_ms[top] / sum(stage_ms.values())}

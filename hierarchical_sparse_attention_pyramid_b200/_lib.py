@@ -39,7 +39,7 @@ class LhPlanInfo(ctypes.Structure):
                  ("level_off", c_int64 * MAX_LEVELS), ("upper_off", c_int64 * MAX_LEVELS),
                  ("upper_entries", c_int64), ("kprime", c_int32 * MAX_LEVELS), ("sel_off", c_int64 * MAX_LEVELS),
                  ("sel_per_head", c_int64)]
-                + [(n, c_size_t) for n in _SIZES])
+                + [(n, c_size_t) for n in _SIZES] + [("first_level", c_int32)])
 
 
 _P = c_void_p
@@ -48,9 +48,11 @@ _CFG = POINTER(LhConfig)
 SIGNATURES = {
     "lh_plan": [_CFG, POINTER(LhPlanInfo)],
     "lh_pyramid_pool": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lh_pyramid_pool_from": [_CFG, c_int32, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_score_topk": [_CFG, _P, _P, _P, _P],
     "lh_score_topk_static": [_CFG, _P, _P, _P],
     "lh_gather": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lh_gather_from": [_CFG, c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_fwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_bwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_scatter_back": [_CFG, _P, _P, _P, _P],

@@ -81,14 +81,21 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 
 # ------------------------------------------------------------------ stages
 
-def pyramid_pool(layer: Layer, q, k, v):
-    """-> pyr_q, pyr_k, pyr_v [BH, upper_entries, d] (levels >= 1), norms [2, BH, N] fp32."""
+def pyramid_pool(layer: Layer, q, k, v, first_level: int | None = None):
+    """-> pyr_q, pyr_k, pyr_v [BH, upper_entries, d] (levels >= 1), norms [2, BH, N] fp32.
+    With first_level (lh_pyramid_pool_from), levels below it are not written (rows left zero here)."""
     info = plan(layer)
     dev = q.device
     shp = (layer.BH, max(info.upper_entries, 1), layer.d)
-    pq, pk, pv = (_empty(shp, layer.torch_dtype, dev) for _ in range(3))
+    mk = torch.zeros if first_level is not None else _empty
+    pq, pk, pv = (mk(shp, dtype=layer.torch_dtype, device=dev) for _ in range(3))
     norms = _empty((2, layer.BH, layer.N), torch.float32, dev)
-    call("lh_pyramid_pool", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(norms), _stream())
+    if first_level is None:
+        call("lh_pyramid_pool", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(norms),
+             _stream())
+    else:
+        call("lh_pyramid_pool_from", ctypes.byref(layer.cfg()), ctypes.c_int32(first_level), _p(q), _p(k), _p(v),
+             _p(pq), _p(pk), _p(pv), _p(norms), _stream())
     return pq, pk, pv, norms
 
 
@@ -102,16 +109,21 @@ def score_topk(layer: Layer, norms, ws=None):
     return sel
 
 
-def gather(layer: Layer, q, k, v, pq, pk, pv, sel):
-    """-> qs, ks, vs [BH, S, d] bf16, seq_map [BH, S] int32, slot_of [BH, pyr_entries] int32."""
+def gather(layer: Layer, q, k, v, pq, pk, pv, sel, first_level: int | None = None):
+    """-> qs, ks, vs [BH, S, d] bf16, seq_map [BH, S] int32, slot_of [BH, pyr_entries] int32.
+    With first_level (lh_gather_from), kept entries of the levels below it are averaged from q, k, v."""
     info = plan(layer)
     dev = q.device
     S = info.S
     qs, ks, vs = (_empty((layer.BH, S, layer.d), torch.bfloat16, dev) for _ in range(3))
     seq_map = _empty((layer.BH, S), torch.int32, dev)
     slot_of = _empty((layer.BH, info.pyr_entries), torch.int32, dev)
-    call("lh_gather", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(sel),
-         _p(qs), _p(ks), _p(vs), _p(seq_map), _p(slot_of), _stream())
+    if first_level is None:
+        call("lh_gather", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(pq), _p(pk), _p(pv), _p(sel),
+             _p(qs), _p(ks), _p(vs), _p(seq_map), _p(slot_of), _stream())
+    else:
+        call("lh_gather_from", ctypes.byref(layer.cfg()), ctypes.c_int32(first_level), _p(q), _p(k), _p(v), _p(pq),
+             _p(pk), _p(pv), _p(sel), _p(qs), _p(ks), _p(vs), _p(seq_map), _p(slot_of), _stream())
     return qs, ks, vs, seq_map, slot_of
 
 

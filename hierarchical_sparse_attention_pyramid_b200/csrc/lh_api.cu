@@ -130,6 +130,16 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   const size_t bwd = off;
   info->ws_bytes = fwd > bwd ? fwd : bwd;
 
+  {
+    Dims tmp;
+    Dims* T = D ? D : &tmp;
+    T->L = L; T->log2p = log2p;
+    for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+      T->level_len[l] = info->level_len[l];
+      T->kprime[l] = info->kprime[l];
+    }
+    info->first_level = materialized_level(*T);
+  }
   if (D) {
     D->BH = BH; D->N = N; D->S = S;
     D->d = d; D->L = L; D->p = p; D->log2p = log2p; D->chunk = chunk;
@@ -193,6 +203,22 @@ lh_status lh_pyramid_pool(const lh_config* cfg, const void* q, const void* k, co
   return LH_OK;
 }
 
+lh_status lh_pyramid_pool_from(const lh_config* cfg, int32_t first_level, const void* q, const void* k,
+                               const void* v, void* pyr_q, void* pyr_k, void* pyr_v, float* norms,
+                               lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  if (first_level < 1 || first_level > (D.L > 1 ? D.L - 1 : 1))
+    return fail(LH_ERR_INVALID_ARG, "lh_pyramid_pool_from: first_level outside [1, max(1, L-1)]");
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v); LH_CHECK_PTR(norms);
+  if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); }
+  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, (cudaStream_t)stream, first_level),
+          "lh_pyramid_pool_from");
+  return LH_OK;
+}
+
 lh_status lh_score_topk(const lh_config* cfg, const float* norms, void* ws, int32_t* sel, lh_stream_t stream) {
   lh_plan_info info;
   Dims D;
@@ -218,6 +244,24 @@ lh_status lh_gather(const lh_config* cfg, const void* q, const void* k, const vo
   LH_CUDA(launch_gather(D, q, k, v, pyr_q, pyr_k, pyr_v, sel, qs, ks, vs, seq_map, slot_of, nullptr,
                         (cudaStream_t)stream),
           "lh_gather");
+  return LH_OK;
+}
+
+lh_status lh_gather_from(const lh_config* cfg, int32_t first_level, const void* q, const void* k, const void* v,
+                         const void* pyr_q, const void* pyr_k, const void* pyr_v, const int32_t* sel, void* qs,
+                         void* ks, void* vs, int32_t* seq_map, int32_t* slot_of, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  if (first_level < 1 || first_level > (D.L > 1 ? D.L - 1 : 1))
+    return fail(LH_ERR_INVALID_ARG, "lh_gather_from: first_level outside [1, max(1, L-1)]");
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v);
+  if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); LH_CHECK_PTR(sel); }
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(slot_of);
+  LH_CUDA(launch_gather(D, q, k, v, pyr_q, pyr_k, pyr_v, sel, qs, ks, vs, seq_map, slot_of, nullptr,
+                        (cudaStream_t)stream, first_level),
+          "lh_gather_from");
   return LH_OK;
 }
 
@@ -312,7 +356,7 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   void* vs = c + I.ctx_off_vs;
   float* os = reinterpret_cast<float*>(c + I.ctx_off_os);
   float* lse = reinterpret_cast<float*>(c + I.ctx_off_lse);
-  const int first = materialized_level(D);
+  const int first = I.first_level;
   LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st, first), "lh_forward: pool");
   LH_CUDA(launch_score_topk(D, norms, spyr, sel, errw, st), "lh_forward: score_topk");
   LH_CUDA(launch_gather(D, q, k, v, pq, pk, pv, sel, qs, ks, vs, seq_map, slot_of, errw, st, first),

@@ -108,6 +108,11 @@ typedef struct {
       ctx_off_lse;
   size_t ws_off_pyr_q, ws_off_pyr_k, ws_off_pyr_v, ws_off_norms, ws_off_topk;
   size_t ws_off_dos, ws_off_delta, ws_off_dqs, ws_off_dks, ws_off_dvs;
+  /* lowest pyramid level that lh_forward writes (1 <= first_level <= max(1, L-1)):
+   * a level l < L-1 is written whole only when N/p^l rows cost no more than
+   * reading back the p^(l+1) kprime[l] level-0 rows of its kept entries;
+   * the gather averages the kept entries of the levels below from level 0 */
+  int32_t first_level;
 } lh_plan_info;
 
 /* Validate cfg and fill *info (host only, no CUDA call).
@@ -126,6 +131,14 @@ lh_status lh_plan(const lh_config *cfg, lh_plan_info *info);
  * With L = 1 the pyramid buffers are not touched (may be NULL). */
 lh_status lh_pyramid_pool(const lh_config *cfg, const void *q, const void *k, const void *v, void *pyr_q,
                           void *pyr_k, void *pyr_v, float *norms, lh_stream_t stream);
+
+/* Stage 1 as lh_forward runs it: the same pooling and norms, but only levels
+ * first_level..L-1 are written (rows of levels 1..first_level-1 of the
+ * pyramid buffers are left untouched).  first_level in [1, max(1, L-1)];
+ * plan_info.first_level is the value lh_forward uses.  lh_pyramid_pool is
+ * this call with first_level = 1.  Same citations as lh_pyramid_pool. */
+lh_status lh_pyramid_pool_from(const lh_config *cfg, int32_t first_level, const void *q, const void *k, const void *v,
+                               void *pyr_q, void *pyr_k, void *pyr_v, float *norms, lh_stream_t stream);
 
 /* Stage 2 - max-pooled scores and stratified chunked top-k.
  * Cite: LH-summary "Technical details" (2) (coarser levels take max-pooled
@@ -168,6 +181,15 @@ lh_status lh_score_topk_static(const lh_config *cfg, const float *norms, int32_t
 lh_status lh_gather(const lh_config *cfg, const void *q, const void *k, const void *v, const void *pyr_q,
                     const void *pyr_k, const void *pyr_v, const int32_t *sel, void *qs, void *ks, void *vs,
                     int32_t *seq_map, int32_t *slot_of, lh_stream_t stream);
+
+/* Stage 3 as lh_forward runs it: identical outputs, but a kept entry of a
+ * level l < first_level is computed as the fp32 mean of its p^l level-0 rows
+ * of q, k, v (rounded once), so the pyramid buffers are read only for levels
+ * >= first_level (as written by lh_pyramid_pool_from with the same value).
+ * lh_gather is this call with first_level = 1. */
+lh_status lh_gather_from(const lh_config *cfg, int32_t first_level, const void *q, const void *k, const void *v,
+                         const void *pyr_q, const void *pyr_k, const void *pyr_v, const int32_t *sel, void *qs,
+                         void *ks, void *vs, int32_t *seq_map, int32_t *slot_of, lh_stream_t stream);
 
 /* Stage 4 - dense causal attention over the S-token sequence (tcgen05).
  * Cite: LH-summary "Technical details" (3) (stock attention over the gathered

@@ -53,6 +53,15 @@ def test_plan_matches_oracle_sizes(lib, name):
     assert info.ctx_bytes > 0 and info.ws_bytes > 0
     for f in ("ctx_off_sel", "ctx_off_qs", "ctx_off_lse", "ws_off_pyr_q", "ws_off_dqs"):
         assert getattr(info, f) % 256 == 0
+    # the lowest level lh_forward writes: the first level below the top whose
+    # N/p^l rows cost no more than the p^(l+1) k' level-0 rows its kept
+    # entries would read back, else the top level
+    want = max(1, w.L - 1)
+    for lvl, kp in enumerate(lo.budgets(w.N, w.p, w.L, w.k)):
+        if 1 <= lvl and w.N // w.p ** lvl <= w.p ** (lvl + 1) * kp:
+            want = lvl
+            break
+    assert info.first_level == want
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -88,6 +97,12 @@ def test_failure_paths_return_before_any_gpu_work(lib):
                           info.ws_bytes, None) == 3
     assert lib.lh_backward(ctypes.byref(cfg), fake, fake, info.ctx_bytes, fake, fake, fake, fake,
                            info.ws_bytes - 1, None) == 3
+    # first_level outside [1, L-1]
+    for first in (0, 3):
+        assert lib.lh_pyramid_pool_from(ctypes.byref(cfg), first, fake, fake, fake, fake, fake, fake, fake,
+                                        None) == 1
+        assert lib.lh_gather_from(ctypes.byref(cfg), first, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                                  fake, fake, fake, None) == 1
     # unsupported head dim in the attention stage
     bad = _lib.LhConfig(1, 1, 4096, 80, 3, 2, 256, 0, 0, 0)
     assert lib.lh_attn_fwd(ctypes.byref(bad), 100, fake, fake, fake, fake, fake, fake, None) == 2

@@ -97,6 +97,38 @@ def test_gather(name):
             pu.assert_close(pu.to_np(got[bh]), want, f"{name} {t}")
 
 
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_pool_from_and_gather_from(name):
+    """The stage calls lh_forward makes: the pool writes levels >= first_level
+    only (the rows below stay as they were), the norms are unchanged, and the
+    gather that averages the lower levels from level 0 matches the oracle, for
+    every admissible first_level (the plan's choice included)."""
+    w, x, heads = case(name)
+    L = layer_of(w)
+    info = lh.plan(L)
+    assert 1 <= info.first_level <= max(1, w.L - 1)
+    _, _, _, norms_full = lh.pyramid_pool(L, x["q"], x["k"], x["v"])
+    sel = lh.score_topk(L, norms_full) if w.L > 1 else torch.zeros(1, dtype=torch.int32, device="cuda")
+    for first in range(1, max(1, w.L - 1) + 1):
+        pq, pk, pv, norms = lh.pyramid_pool(L, x["q"], x["k"], x["v"], first_level=first)
+        qs, ks, vs, seq_map, slot_of = lh.gather(L, x["q"], x["k"], x["v"], pq, pk, pv, sel, first_level=first)
+        torch.cuda.synchronize()
+        assert torch.equal(norms, norms_full), f"{name} first_level {first}: norms differ"
+        for bh, o in enumerate(heads):
+            sv = o["saved"]
+            for lvl in range(1, w.L):
+                a, n = info.upper_off[lvl], info.level_len[lvl]
+                for got, want, t in ((pq, sv["pyr_q"], "q"), (pk, sv["pyr_k"], "k"), (pv, sv["pyr_v"], "v")):
+                    if lvl >= first:
+                        pu.assert_close(pu.to_np(got[bh, a:a + n]), want[lvl], f"{name} from {first} pyr_{t} {lvl}")
+                    else:
+                        assert not got[bh, a:a + n].any(), f"{name} from {first}: level {lvl} of pyr_{t} written"
+            np.testing.assert_array_equal(seq_map[bh].cpu().numpy().astype(np.int64), pu.oracle_seq_map(sv))
+            np.testing.assert_array_equal(slot_of[bh].cpu().numpy().astype(np.int64), pu.oracle_slot_of(sv))
+            for got, want, t in ((qs, sv["Qs"], "Qs"), (ks, sv["Ks"], "Ks"), (vs, sv["Vs"], "Vs")):
+                pu.assert_close(pu.to_np(got[bh]), want, f"{name} from {first} {t}")
+
+
 def _bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16)
 
