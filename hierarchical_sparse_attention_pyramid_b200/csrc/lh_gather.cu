@@ -259,7 +259,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32) scatter_adjoint_kernel(ScatterAdjArgs a) {
   constexpr int VE = (sizeof(T) == 2 && D == 128) ? 8 : 4;
   constexpr int LPR = D / VE, R = 32 / LPR;
-  constexpr int U = 4;
+  constexpr int U = 8;
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int64_t bh = wid / a.S;

@@ -14,8 +14,7 @@
 namespace lh {
 namespace {
 
-constexpr int kWarps = 8;   // warps per block
-constexpr int kUnroll = 8;  // row groups loaded ahead per warp
+constexpr int kWarps = 8;  // warps per block
 constexpr unsigned kFull = 0xffffffffu;
 
 struct PoolArgs {
@@ -65,7 +64,7 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[U], int lane) {
 template <typename T, int D, int NL>
 __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
   constexpr int VE = D / 32;
-  constexpr int U = sizeof(T) * VE >= 16 ? 8 : 16;  // rows loaded per batch
+  constexpr int U = 8;  // rows loaded per batch (two batches in flight)
   using Raw = typename RawVec<sizeof(T) * VE>::type;
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -264,9 +263,11 @@ cudaError_t pool_adj_dispatch_L(int L, const PoolAdjArgs& a, int64_t blocks, cud
   return cudaGetLastError();
 }
 
-int task_rows_for(const Dims& D) {
+// rows per warp task: a whole number of top-level blocks, and at least
+// min_rows so that the first loads' latency is paid once per long run
+int task_rows_for(const Dims& D, int min_rows) {
   const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
-  return (int)(ptop > 64 ? ptop : 64);
+  return (int)(ptop > min_rows ? ptop : min_rows);
 }
 
 }  // namespace
@@ -279,7 +280,7 @@ cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void*
   a.norms = norms;
   a.BH = D.BH; a.N = D.N; a.upper_entries = D.upper_entries;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) a.upper_off[l] = D.upper_off[l];
-  a.task_rows = task_rows_for(D);
+  a.task_rows = task_rows_for(D, 512);
   a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
   a.log2p = D.log2p;
   a.first_level = first_level;
@@ -300,7 +301,7 @@ cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dk
   a.slot_of = slot_of;
   a.BH = D.BH; a.N = D.N; a.S = D.S; a.pyr_entries = D.pyr_entries;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) a.level_off[l] = D.level_off[l];
-  a.task_rows = task_rows_for(D);
+  a.task_rows = task_rows_for(D, 64);
   a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
   a.log2p = D.log2p;
   const int64_t warps = 3 * D.BH * a.tasks_per_head;
