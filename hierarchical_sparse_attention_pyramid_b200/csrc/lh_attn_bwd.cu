@@ -18,11 +18,13 @@
 //   dV += P^T dO_h and dK += dS^T Q_h with both A operands read from TMEM.
 //   Q_h, dO_h stream through a 4-slot ring.
 //
-// attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over
-//   64-key half tiles up to the diagonal: S = Q K_h^T and dP = dO V_h^T into
-//   TMEM buffer u&1, the compute warpgroups write dS (hi/lo) over the dP
-//   columns, and dQ += dS K_h reads it from TMEM.  K_h and V_h stream through
-//   4-slot rings, each slot released by the last product that reads it.
+// attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over the
+//   128-key tiles up to the diagonal.  S = Q K_j^T runs two tiles ahead into a
+//   double-buffered TMEM region and dP = dO V_j^T one tile ahead; the compute
+//   warpgroups turn the scores into P as soon as they land, then write dS
+//   (hi/lo) over the dP columns, and dQ += dS K_j reads it from TMEM.  K
+//   streams through 3 stages (read by S(j) and, two tiles later, by dQ(j)),
+//   V through 2.
 //
 // Warp roles in both: warps 0-7 two compute warpgroups (thread (g, t) owns
 // TMEM lane t and columns [32g, 32g+32) of each 64-column half), warp 8 TMA
@@ -293,21 +295,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ===========================================================================
 template <int D>
 struct QSmem {
-  static constexpr int kTile = D / 64 * kRegion;      // Q or dO tile, 128 rows
-  static constexpr int kHalf = D / 64 * kHalfRegion;  // K_h or V_h, 64 rows
+  static constexpr int kTile = D / 64 * kRegion;  // one 128-row tile of Q, dO, K or V
   static constexpr int oQ = 0;
-  static constexpr int oO = oQ + kTile;     // dO
-  static constexpr int oK = oO + kTile;     // 4 slots of K_h
-  static constexpr int oV = oK + 4 * kHalf; // 4 slots of V_h
-  static constexpr int oBar = oV + 4 * kHalf;
+  static constexpr int oO = oQ + kTile;      // dO
+  static constexpr int oK = oO + kTile;      // 3 stages: K_j is read by S(j) two steps before dQ(j)
+  static constexpr int oV = oK + 3 * kTile;  // 2 stages
+  static constexpr int oBar = oV + 2 * kTile;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKh,
-                      const __grid_constant__ CUtensorMap tmVh, const __grid_constant__ CUtensorMap tmO,
+    attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dQ,
                       int* errw, int S, float scale_log2, float scale) {
   using Lay = QSmem<D>;
@@ -315,13 +316,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bQO = bars + 0;     // Q, dO landed
-  uint64_t* bK = bars + 1;      // [4] K_h of a slot landed
-  uint64_t* bV = bars + 5;      // [4] V_h of a slot landed
-  uint64_t* bKfree = bars + 9;  // [4] the dQ product is done with K_h
-  uint64_t* bVfree = bars + 13; // [4] the dP product is done with V_h
-  uint64_t* bF = bars + 17;     // [2] S, dP of a half step in TMEM buffer
-  uint64_t* bPS = bars + 19;    // [2] dS written back (256 arrivals)
-  uint64_t* bDone = bars + 21;  // every product done
+  uint64_t* bK = bars + 1;      // [3] K tile of a stage landed
+  uint64_t* bV = bars + 4;      // [2] V tile of a stage landed
+  uint64_t* bKfree = bars + 6;  // [3] the dQ product is done with a K stage
+  uint64_t* bVfree = bars + 9;  // [2] the dP product is done with a V stage
+  uint64_t* bS = bars + 11;     // [2] S of a key tile in TMEM buffer
+  uint64_t* bSfree = bars + 13; // [2] the scores of a buffer are in registers (256 arrivals)
+  uint64_t* bDP = bars + 15;    // dP of the current key tile in TMEM
+  uint64_t* bPS = bars + 16;    // dS written over dP (256 arrivals)
+  uint64_t* bDone = bars + 17;  // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
@@ -329,20 +332,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_qt = (S + 127) / 128;
   const int qt = n_qt - 1 - (int)blockIdx.x;  // longest rows first
   const int bh = (int)blockIdx.y;
-  const int NU = 2 * (qt + 1);  // 64-key half steps up to the diagonal
+  const int NJ = qt + 1;  // key tiles up to the diagonal
 
   if (threadIdx.x == 0) {
     mbar_init(bQO, 1);
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&bK[i], 1);
-      mbar_init(&bV[i], 1);
       mbar_init(&bKfree[i], 1);
-      mbar_init(&bVfree[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bF[i], 1);
-      mbar_init(&bPS[i], kCompute);
+      mbar_init(&bV[i], 1);
+      mbar_init(&bVfree[i], 1);
+      mbar_init(&bS[i], 1);
+      mbar_init(&bSfree[i], kCompute);
     }
+    mbar_init(bDP, 1);
+    mbar_init(bPS, kCompute);
     mbar_init(bDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -352,85 +357,106 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr uint32_t tS = 0, tDP = 128, tDQ = 256;  // S, dP: [2] x 64 columns
+  constexpr uint32_t tS = 0, tDP = 256, tDQ = 384;  // S: [2] x 128 columns; dP, then dS (hi/lo): 128
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
-    // K_h and V_h of half step u go to slot u & 3; V_h is released by the dP
-    // product of its half step, K_h by the dQ product, so each reloads as
-    // soon as its last reader is done
+    // K_j to stage j % 3 once the dQ product of key tile j-3 is done, V_j to
+    // stage j & 1 once the dP product of key tile j-2 is done
     if (lane == 0) {
-      tma_prefetch_desc(&tmKh);
-      tma_prefetch_desc(&tmVh);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
       mbar_expect_tx(bQO, 2 * 128 * D * 2);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_3d(smem + Lay::oQ + c * kRegion, &tmQ, bQO, c * 64, qt * 128, bh);
         tma_load_3d(smem + Lay::oO + c * kRegion, &tmO, bQO, c * 64, qt * 128, bh);
       }
-      for (int u = 0; u < NU; ++u) {
-        const int slot = u & 3, k0 = u * 64;
-        const uint32_t par = ((u >> 2) - 1) & 1;
-        if (u >= 4 && !mbar_wait(&bVfree[slot], par, abort_flag)) break;
-        mbar_expect_tx(&bV[slot], 64 * D * 2);
+      for (int j = 0; j < NJ; ++j) {
+        const int sk = j % 3, sv = j & 1;
+        if (j >= 3 && !mbar_wait(&bKfree[sk], ((j / 3) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&bK[sk], 128 * D * 2);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oV + slot * Lay::kHalf + c * kHalfRegion, &tmVh, &bV[slot], c * 64, k0, bh);
-        if (u >= 4 && !mbar_wait(&bKfree[slot], par, abort_flag)) break;
-        mbar_expect_tx(&bK[slot], 64 * D * 2);
+          tma_load_3d(smem + Lay::oK + sk * Lay::kTile + c * kRegion, &tmK, &bK[sk], c * 64, j * 128, bh);
+        if (j >= 2 && !mbar_wait(&bVfree[sv], ((j >> 1) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&bV[sv], 128 * D * 2);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + Lay::oK + slot * Lay::kHalf + c * kHalfRegion, &tmKh, &bK[slot], c * 64, k0, bh);
+          tma_load_3d(smem + Lay::oV + sv * Lay::kTile + c * kRegion, &tmV, &bV[sv], c * 64, j * 128, bh);
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Per key tile j: dQ += dS(j) K_j, then dP(j+1) = dO V_{j+1}^T (over the dS
+    // columns just read), then S(j+2) = Q K_{j+2}^T into the S buffer that
+    // tile j's scores have left, so the scores are two tiles ahead of the
+    // softmax-gradient pass and dP one tile ahead.
     {  // the whole warp; one elected lane issues each instruction
-      constexpr uint32_t idF = idesc_bf16(128, 64, false, false);  // S, dP: N = 64 keys
-      constexpr uint32_t idG = idesc_bf16(128, D, false, true);    // dQ: A from TMEM, B MN-major
+      constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S, dP: N = 128 keys
+      constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dQ: A from TMEM, B MN-major
       const uint64_t kQ = sdesc_sw128(smem_u32(smem + Lay::oQ), 16, 1024);
       const uint64_t kO = sdesc_sw128(smem_u32(smem + Lay::oO), 16, 1024);
       const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
       const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
-      const uint64_t mK = sdesc_sw128(smem_u32(smem + Lay::oK), kHalfRegion, 1024);
-      bool ok = mbar_wait_warp(bQO, 0, abort_flag);
-      auto wait_f = [&](int u) -> bool {
-        return mbar_wait_warp(&bK[u & 3], (u >> 2) & 1, abort_flag) && mbar_wait_warp(&bV[u & 3], (u >> 2) & 1, abort_flag);
-      };
-      auto issue_f = [&](int u) {
-        const int slot = u & 3, b = u & 1;
-        tc_fence_after();
-        const uint32_t so = (slot * Lay::kHalf) >> 4;
+      const uint64_t mK = sdesc_sw128(smem_u32(smem + Lay::oK), kRegion, 1024);
+      auto issue_s = [&](int j) {  // S(j) = Q K_j^T into buffer j & 1
+        const uint32_t ko = ((j % 3) * Lay::kTile) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qoff = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;      // Q, dO (128 rows)
-          const uint32_t hoff = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // K_h, V_h (64 rows)
-          umma_bf16_w(tmem + tS + b * 64, kQ + qoff, kK + so + hoff, idF, kk > 0 ? 1u : 0u);
-          umma_bf16_w(tmem + tDP + b * 64, kO + qoff, kV + so + hoff, idF, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + tS + (j & 1) * 128, kQ + off, kK + ko + off, idF, kk > 0 ? 1u : 0u);
         }
-        umma_commit_w(&bVfree[slot]);
-        umma_commit_w(&bF[b]);
+        umma_commit_w(&bS[j & 1]);
       };
-      if (ok && (ok = wait_f(0))) issue_f(0);
-      if (ok && NU > 1 && (ok = wait_f(1))) issue_f(1);
-      for (int u = 0; ok && u < NU; ++u) {
-        const int slot = u & 3, b = u & 1;
-        if (u + 2 < NU && !wait_f(u + 2)) { ok = false; break; }
-        if (!mbar_wait_warp(&bPS[b], (u >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t mk = mK + ((slot * Lay::kHalf) >> 4);
+      auto issue_dp = [&](int j) {  // dP(j) = dO V_j^T; then V_j is free
+        const uint32_t vo = ((j & 1) * Lay::kTile) >> 4;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 16 keys per step
-          const uint32_t a = tmem + tDP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + tDP, kO + off, kV + vo + off, idF, kk > 0 ? 1u : 0u);
+        }
+        umma_commit_w(bDP);
+        umma_commit_w(&bVfree[j & 1]);
+      };
+      bool ok = mbar_wait_warp(bQO, 0, abort_flag) && mbar_wait_warp(&bK[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        ok = mbar_wait_warp(&bV[0], 0, abort_flag);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dp(0);
+        if (NJ > 1 && (ok = mbar_wait_warp(&bK[1], 0, abort_flag))) {
+          tc_fence_after();
+          issue_s(1);
+        }
+      }
+      for (int j = 0; ok && j < NJ; ++j) {
+        // operands of the products after dQ(j), waited for first so that no
+        // wait sits between them
+        if (j + 1 < NJ && !mbar_wait_warp(&bV[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (j + 2 < NJ) {
+          if (!mbar_wait_warp(&bK[(j + 2) % 3], ((j + 2) / 3) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bSfree[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        if (!mbar_wait_warp(bPS, j & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t mk = mK + (((j % 3) * Lay::kTile) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step; hi of chunk kk/2 at +(kk&1)*8, lo at +16
+          const uint32_t a = tmem + tDP + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint64_t bk = mk + ((kk * 2048) >> 4);
-          umma_bf16_tmem_a_w(tmem + tDQ, a, bk, idG, (u > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a_w(tmem + tDQ, a, bk, idG, (j > 0 || kk > 0) ? 1u : 0u);
           umma_bf16_tmem_a_w(tmem + tDQ, a + 16, bk, idG, 1u);
         }
-        umma_commit_w(&bKfree[slot]);
-        if (u + 2 < NU) issue_f(u + 2);
+        umma_commit_w(&bKfree[j % 3]);
+        if (j + 1 < NJ) issue_dp(j + 1);  // after dQ(j) has read dS(j) (in-order issue)
+        if (j + 2 < NJ) issue_s(j + 2);
       }
       if (ok) umma_commit_w(bDone);
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
-    const int g = warp >> 2;               // key columns [32g, 32g+32) of each half
+    const int g = warp >> 2;               // keys [64g, 64g+64) of every key tile
     const int t = (warp & 3) * 32 + lane;  // query row of the tile (TMEM lane)
     const int qg = qt * 128 + t;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -439,37 +465,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
     const uint64_t nl2 = f2_pack(-lse, -lse), d2 = f2_pack(del, del);
     bool ok = true;
-    for (int u = 0; u < NU; ++u) {
-      const int b = u & 1;
-      const int k0 = (u >> 1) * 128 + (u & 1) * 64 + g * 32;  // first key of this thread's chunk
-      const bool diag = (u >> 1) == qt;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bF[b], (u >> 1) & 1, abort_flag));
+    for (int j = 0; j < NJ; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bS[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tl + tS + b * 64 + g * 32, sr);
-      tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
+      // P = 2^(s*scale*log2e - lse*log2e) of this thread's 64 keys; the S
+      // buffer is free once the scores are in registers
+      uint32_t r[2][32];
+      tmem_ld32(tl + tS + b * 128 + g * 64, r[0]);
+      tmem_ld32(tl + tS + b * 128 + g * 64 + 32, r[1]);
       tmem_ld_wait();
-      uint32_t dhi[16], dlo[16];
+      tc_fence_before();
+      mbar_arrive(&bSfree[b]);
+      // keys after the row are masked on the diagonal tile: limit = row there,
+      // past every key elsewhere
+      const int limit = j == qt ? t - g * 64 : 1 << 20;
+      float p[2][32];
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float pa, pb;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nl2), pa, pb);
-        pa = fast_exp2(pa);
-        pb = fast_exp2(pb);
-        if (diag) {
-          if (k0 + e > qg) pa = 0.f;
-          if (k0 + e + 1 > qg) pb = 0.f;
+      for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pa, pb;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][e]), __uint_as_float(r[ch][e + 1])), c2, nl2), pa, pb);
+          pa = fast_exp2(pa);
+          pb = fast_exp2(pb);
+          p[ch][e] = ch * 32 + e > limit ? 0.f : pa;
+          p[ch][e + 1] = ch * 32 + e + 1 > limit ? 0.f : pb;
         }
-        const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), d2);
-        float da, db;
-        f2_unpack(f2_mul(f2_mul(f2_pack(pa, pb), sc2), diff2), da, db);
-        split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+      ok = __all_sync(0xffffffffu, mbar_wait(bDP, j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // dS = P (dP - Delta) / sqrt(d) as a bf16 pair over the dP columns just
+      // read: per 32 keys, hi in the first 16 columns and lo in the last 16
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t dr[32];
+        tmem_ld32(tl + tDP + g * 64 + ch * 32, dr);
+        tmem_ld_wait();
+        uint32_t dhi[16], dlo[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), d2);
+          float da, db;
+          f2_unpack(f2_mul(f2_mul(f2_pack(p[ch][e], p[ch][e + 1]), sc2), diff2), da, db);
+          split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+        }
+        store_pair_chunk(tl + tDP + g * 64 + ch * 32, dhi, dlo);
       }
-      store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bPS[b]);
+      mbar_arrive(bPS);
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
       tc_fence_after();
@@ -500,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // TMA maps of the sequences: full 128-row boxes and 64-row half boxes
 struct SeqMaps {
-  CUtensorMap q, qh, kh, k, v, vh, o, oh;
+  CUtensorMap q, qh, k, v, o, oh;
 };
 
 template <int D>
@@ -517,7 +563,7 @@ cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* l
   smem = QSmem<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_q_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.kh, m.vh, m.o, lse, delta, dqs, errw,
+  attn_bwd_q_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dqs, errw,
                                                                         (int)S, scale_log2, scale);
   return cudaGetLastError();
 }
@@ -529,8 +575,7 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const 
                             float* dvs, int* errw, cudaStream_t st) {
   SeqMaps m;
   if (!make_seq_map(&m.q, qs, BH, S, d, 128) || !make_seq_map(&m.qh, qs, BH, S, d, 64) ||
-      !make_seq_map(&m.k, ks, BH, S, d, 128) || !make_seq_map(&m.kh, ks, BH, S, d, 64) ||
-      !make_seq_map(&m.v, vs, BH, S, d, 128) || !make_seq_map(&m.vh, vs, BH, S, d, 64) ||
+      !make_seq_map(&m.k, ks, BH, S, d, 128) || !make_seq_map(&m.v, vs, BH, S, d, 128) ||
       !make_seq_map(&m.o, dos, BH, S, d, 128) || !make_seq_map(&m.oh, dos, BH, S, d, 64))
     return cudaErrorInvalidValue;
   const double scale = 1.0 / sqrt((double)d);
