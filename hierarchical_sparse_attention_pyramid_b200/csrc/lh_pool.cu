@@ -9,10 +9,14 @@
 // Both kernels are HBM streams: one warp walks a contiguous run of rows of
 // one head and one of Q, K, V, so every load or store instruction of the warp
 // touches whole rows.
+#include <type_traits>
+
 #include "lh_common.cuh"
+#include "sm100.cuh"
 
 namespace lh {
 namespace {
+using namespace sm100;
 
 constexpr int kWarps = 8;  // warps per block
 constexpr unsigned kFull = 0xffffffffu;
@@ -81,11 +85,19 @@ __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
   float* norm_out = a.norms + ((int64_t)tensor * a.BH + bh) * a.N + row0;
   const int rid = scatter_row<U>(lane);
 
-  float acc[NL + 1][VE];
+  // bf16 rows are widened and summed as fp32 pairs (f32x2 arithmetic): one
+  // packed fma for the squares and one packed add per two channels
+  constexpr bool kPacked = std::is_same<T, __nv_bfloat16>::value && VE % 2 == 0;
+  constexpr int NP = kPacked ? VE / 2 : 1;
+  float acc[NL + 1][kPacked ? 1 : VE];
+  uint64_t acc2[NL + 1][NP];
 #pragma unroll
-  for (int l = 0; l <= NL; ++l)
+  for (int l = 0; l <= NL; ++l) {
 #pragma unroll
-    for (int i = 0; i < VE; ++i) acc[l][i] = 0.f;
+    for (int i = 0; i < (kPacked ? 1 : VE); ++i) acc[l][i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NP; ++i) acc2[l][i] = 0ull;
+  }
 
   auto load = [&](Raw (&x)[U], int r0) {
 #pragma unroll
@@ -98,32 +110,68 @@ __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
     float sq[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const T* e = reinterpret_cast<const T*>(&x[u]);
-      float v[VE];
+      if constexpr (kPacked) {
+        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&x[u]);  // channels 2i, 2i+1 in word i
+        uint64_t q2 = 0ull;
 #pragma unroll
-      for (int i = 0; i < VE; ++i) v[i] = Elem<T>::to_f(e[i]);
-      float q = 0.f;
+        for (int i = 0; i < NP; ++i) {
+          const uint64_t v2 = f2_pack(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xffff0000u));
+          q2 = f2_fma(v2, v2, q2);
+          if constexpr (NL > 1) acc2[1][i] = f2_add(acc2[1][i], v2);
+        }
+        float qa, qb;
+        f2_unpack(q2, qa, qb);
+        sq[u] = qa + qb;
+      } else {
+        const T* e = reinterpret_cast<const T*>(&x[u]);
+        float v[VE];
 #pragma unroll
-      for (int i = 0; i < VE; ++i) q = fmaf(v[i], v[i], q);
-      sq[u] = q;
+        for (int i = 0; i < VE; ++i) v[i] = Elem<T>::to_f(e[i]);
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < VE; ++i) q = fmaf(v[i], v[i], q);
+        sq[u] = q;
+        if constexpr (NL > 1) {
+#pragma unroll
+          for (int i = 0; i < VE; ++i) acc[1][i] += v[i];
+        }
+      }
       if constexpr (NL > 1) {
-#pragma unroll
-        for (int i = 0; i < VE; ++i) acc[1][i] += v[i];
         const int done = r0 + u + 1;  // rows of this task consumed
         if (done <= rows && (done & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
           for (int l = 1; l < NL; ++l) {
             if ((done & ((1 << (l * log2p)) - 1)) != 0) break;
             const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
-            float m[VE];
-#pragma unroll
-            for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
             const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
-            if (l >= a.first_level) store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
+            if constexpr (kPacked) {
+              const uint64_t inv2 = f2_pack(inv, inv);
+              if (l >= a.first_level) {
+                Raw o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-            for (int i = 0; i < VE; ++i) {
-              acc[l + 1][i] += acc[l][i];
-              acc[l][i] = 0.f;
+                for (int i = 0; i < NP; ++i) {
+                  float ma, mb;
+                  f2_unpack(f2_mul(acc2[l][i], inv2), ma, mb);
+                  ow[i] = pack_bf16x2(ma, mb);
+                }
+                *reinterpret_cast<Raw*>(dst + (a.upper_off[l] + e_idx) * D) = o;
+              }
+#pragma unroll
+              for (int i = 0; i < NP; ++i) {
+                acc2[l + 1][i] = f2_add(acc2[l + 1][i], acc2[l][i]);
+                acc2[l][i] = 0ull;
+              }
+            } else {
+              float m[VE];
+#pragma unroll
+              for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
+              if (l >= a.first_level) store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
+#pragma unroll
+              for (int i = 0; i < VE; ++i) {
+                acc[l + 1][i] += acc[l][i];
+                acc[l][i] = 0.f;
+              }
             }
           }
         }
