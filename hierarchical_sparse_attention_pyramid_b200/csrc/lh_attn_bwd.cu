@@ -85,11 +85,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bKV = bars + 0;        // K, V landed
   uint64_t* bLoad = bars + 1;      // [4] Q_h, dO_h of a ring slot landed
   uint64_t* bSlotFree = bars + 5;  // [4] dV, dK products done with a slot
-  uint64_t* bF = bars + 9;         // [2] S^T, dP^T of a half step in TMEM buffer
-  uint64_t* bPS = bars + 11;       // [2] P^T, dS^T written back (256 arrivals)
-  uint64_t* bDone = bars + 13;     // every product done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
+  uint64_t* bS = bars + 9;         // [2] S^T of a half step in TMEM buffer
+  uint64_t* bDP = bars + 11;       // [2] dP^T of a half step in TMEM buffer
+  uint64_t* bP = bars + 13;        // [2] P^T written back (256 arrivals)
+  uint64_t* bDS = bars + 15;       // [2] dS^T written back (256 arrivals)
+  uint64_t* bDone = bars + 17;     // every product done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
   float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,8 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bSlotFree[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bF[i], 1);
-      mbar_init(&bPS[i], kCompute);
+      mbar_init(&bS[i], 1);
+      mbar_init(&bDP[i], 1);
+      mbar_init(&bP[i], kCompute);
+      mbar_init(&bDS[i], kCompute);
     }
     mbar_init(bDone, 1);
     *abort_flag = 0;
@@ -155,36 +159,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the loads of half step s landed (waited for before the products that
       // precede its F in the issue order, so no wait sits between them)
       auto wait_f = [&](int s) -> bool { return mbar_wait_warp(&bLoad[s & 3], (s >> 2) & 1, abort_flag); };
+      // S^T = K Q_h^T, then dP^T = V dO_h^T, of half step s into TMEM buffer s & 1,
+      // each with its own completion so the P^T pass can start on S^T alone
       auto issue_f = [&](int s) {
         const int slot = s & 3, b = s & 1;
         tc_fence_after();
         const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // K, V tile (128 rows)
-          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // Q_h, dO_h (64 rows)
+          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // K tile (128 rows)
+          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // Q_h (64 rows)
           umma_bf16_w(tmem + tSP + b * 64, kK + at, kRing + qo + bt, idF, kk > 0 ? 1u : 0u);
+        }
+        umma_commit_w(&bS[b]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // V tile
+          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // dO_h
           umma_bf16_w(tmem + tDP + b * 64, kV + at, kRing + oo + bt, idF, kk > 0 ? 1u : 0u);
         }
-        umma_commit_w(&bF[b]);
+        umma_commit_w(&bDP[b]);
       };
       if (ok && (ok = wait_f(0))) issue_f(0);
       if (ok && NS > 1 && (ok = wait_f(1))) issue_f(1);
       for (int s = 0; ok && s < NS; ++s) {
         const int slot = s & 3, b = s & 1;
         if (s + 2 < NS && !wait_f(s + 2)) { ok = false; break; }
-        if (!mbar_wait_warp(&bPS[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
+        // dV += P^T dO_h as soon as P^T is back (16 queries per step; hi of
+        // chunk kk/2 at +(kk&1)*8, lo at +16), then dK += dS^T Q_h
+        if (!mbar_wait_warp(&bP[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step; hi of chunk kk/2 at +(kk&1)*8, lo at +16
-          const uint32_t a = (kk >> 1) * 32 + (kk & 1) * 8;
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a = tmem + tSP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t bq = (kk * 2048) >> 4;
-          umma_bf16_tmem_a_w(tmem + tDV, tmem + tSP + b * 64 + a, mRing + oo + bq, idG, acc);
-          umma_bf16_tmem_a_w(tmem + tDV, tmem + tSP + b * 64 + a + 16, mRing + oo + bq, idG, 1u);
-          umma_bf16_tmem_a_w(tmem + tDK, tmem + tDP + b * 64 + a, mRing + qo + bq, idG, acc);
-          umma_bf16_tmem_a_w(tmem + tDK, tmem + tDP + b * 64 + a + 16, mRing + qo + bq, idG, 1u);
+          const uint64_t bo = mRing + oo + ((kk * 2048) >> 4);
+          umma_bf16_tmem_a_w(tmem + tDV, a, bo, idG, acc);
+          umma_bf16_tmem_a_w(tmem + tDV, a + 16, bo, idG, 1u);
+        }
+        if (!mbar_wait_warp(&bDS[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t a = tmem + tDP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t bq = mRing + qo + ((kk * 2048) >> 4);
+          umma_bf16_tmem_a_w(tmem + tDK, a, bq, idG, acc);
+          umma_bf16_tmem_a_w(tmem + tDK, a + 16, bq, idG, 1u);
         }
         umma_commit_w(&bSlotFree[slot]);
         // the next half step that uses this TMEM buffer; its S^T, dP^T land
@@ -209,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return qg < S ? ldg_nc_f32((ct < 64 ? LSE : Delta) + (int64_t)bh * S + qg) : 0.f;
     };
     float vec_next = ct < 128 ? vec_raw(0) : 0.f;
-    const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     for (int s = 0; s < NS; ++s) {
       const int b = s & 1;
       const float vec_cur = vec_next;
@@ -223,40 +245,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag = (s >> 1) == 0;  // the diagonal query tile
       // warp-uniform outcome for the collective TMEM accesses; after a failed
       // wait the loop keeps its compute_sync count and skips the work
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bF[b], (s >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bS[b], (s >> 1) & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tl + tSP + b * 64 + g * 32, sr);
-      tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
-      tmem_ld_wait();
-      uint32_t phi[16], plo[16], dhi[16], dlo[16];
+      // P^T as a bf16 pair over the S^T columns just read (hi in the first 16
+      // columns of the 32-query chunk, lo in the last 16); the dV product
+      // starts on it while dP^T is still being computed
+      float p[32];
+      {
+        uint32_t sr[32];
+        tmem_ld32(tl + tSP + b * 64 + g * 32, sr);
+        tmem_ld_wait();
+        uint32_t phi[16], plo[16];
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int qi = g * 32 + e;
-        const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
-        const float2 d2 = *reinterpret_cast<const float2*>(del + qi);
-        float pa, pb;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)), pa,
-                  pb);
-        pa = fast_exp2(pa);
-        pb = fast_exp2(pb);
-        if (diag) {
-          if (q0 + qi < kv_g) pa = 0.f;
-          if (q0 + qi + 1 < kv_g) pb = 0.f;
+        for (int e = 0; e < 32; e += 2) {
+          const int qi = g * 32 + e;
+          const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
+          float pa, pb;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)),
+                    pa, pb);
+          pa = fast_exp2(pa);
+          pb = fast_exp2(pb);
+          if (diag) {
+            if (q0 + qi < kv_g) pa = 0.f;
+            if (q0 + qi + 1 < kv_g) pb = 0.f;
+          }
+          p[e] = pa;
+          p[e + 1] = pb;
+          split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
         }
-        const uint64_t p2 = f2_pack(pa, pb);
-        const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(d2.x, d2.y));
-        float da, db;
-        f2_unpack(f2_mul(f2_mul(p2, sc2), diff2), da, db);
-        split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
-        split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+        store_pair_chunk(tl + tSP + b * 64 + g * 32, phi, plo);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bP[b]);
       }
-      store_pair_chunk(tl + tSP + b * 64 + g * 32, phi, plo);
-      store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bPS[b]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bDP[b], (s >> 1) & 1, abort_flag));
+      if (!ok) continue;
+      tc_fence_after();
+      // dS^T = P^T (dP^T - Delta) / sqrt(d) as a bf16 pair over the dP^T columns
+      {
+        uint32_t dr[32];
+        tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
+        tmem_ld_wait();
+        uint32_t dhi[16], dlo[16];
+        const uint64_t sc2 = f2_pack(scale, scale);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float2 d2 = *reinterpret_cast<const float2*>(del + g * 32 + e);
+          const uint64_t diff2 =
+              f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(d2.x, d2.y));
+          float da, db;
+          f2_unpack(f2_mul(f2_mul(f2_pack(p[e], p[e + 1]), sc2), diff2), da, db);
+          split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
+        }
+        store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bDS[b]);
+      }
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
       tc_fence_after();
