@@ -54,7 +54,6 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_plan: d must be 64 or 128");
   if (p < 2 || (p & (p - 1)) != 0) return fail(LH_ERR_UNSUPPORTED, "lh_plan: p must be a power of two >= 2");
   if (L > 8) return fail(LH_ERR_UNSUPPORTED, "lh_plan: L must be <= 8");
-  if (chunk > 4096) return fail(LH_ERR_UNSUPPORTED, "lh_plan: chunk must be <= 4096");
   if (N >= ((int64_t)1 << 28)) return fail(LH_ERR_UNSUPPORTED, "lh_plan: N must be < 2^28");
   if (B * H > (int64_t)65535 * 65535 || H > 65535) return fail(LH_ERR_UNSUPPORTED, "lh_plan: too many heads");
   const int log2p = ilog2(p);

@@ -79,6 +79,7 @@ struct TopkArgs {
   int32_t chunks[LH_MAX_LEVELS];
   int32_t chunk_prefix[LH_MAX_LEVELS + 1];
   int L;
+  int smem_keys;  // chunks up to this size are staged in shared memory
 };
 
 // exclusive scan of one int per thread over the block; returns the block total in *total
@@ -134,7 +135,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     for (int i = threadIdx.x; i < size; i += kTopkThreads) out[i] = (int32_t)(start + i);
     return;
   }
-  for (int i = threadIdx.x; i < size; i += kTopkThreads) keys[i] = __float_as_uint(src[i]);
+  // a chunk that fits the dynamic shared memory is staged there; a larger one
+  // (a global top-k over a whole level) is read from the score pyramid in
+  // every pass, where it stays L2-resident
+  const bool staged = size <= a.smem_keys;
+  const uint32_t* K = staged ? keys : reinterpret_cast<const uint32_t*>(src);
+  if (staged)
+    for (int i = threadIdx.x; i < size; i += kTopkThreads) keys[i] = __float_as_uint(src[i]);
   __syncthreads();
 
   // radix select of the q-th largest key, 8 bits per pass from the top
@@ -144,7 +151,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     if (threadIdx.x < 256) hist[threadIdx.x] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < size; i += kTopkThreads) {
-      const uint32_t k = keys[i];
+      const uint32_t k = K[i];
       if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -187,14 +194,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
   const int seg = (size + kTopkThreads - 1) / kTopkThreads;
   const int i0 = min(size, (int)threadIdx.x * seg), i1 = min(size, i0 + seg);
   int n_eq = 0;
-  for (int i = i0; i < i1; ++i) n_eq += keys[i] == tau;
+  for (int i = i0; i < i1; ++i) n_eq += K[i] == tau;
   int tot;
   int eq_rank = block_exclusive_scan(n_eq, warp_sums, &tot);
   int n_sel = 0;
   {
     int r = eq_rank;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
+      const uint32_t k = K[i];
       if (k > tau) ++n_sel;
       else if (k == tau) { n_sel += r < need_eq; ++r; }
     }
@@ -203,7 +210,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
   {
     int r = eq_rank;
     for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
+      const uint32_t k = K[i];
       bool take = false;
       if (k > tau) take = true;
       else if (k == tau) { take = r < need_eq; ++r; }
@@ -259,7 +266,9 @@ cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, in
     const int64_t sz = M / C + (M % C ? 1 : 0);
     if (sz > max_size) max_size = sz;
   }
-  const size_t smem = (size_t)max_size * sizeof(uint32_t);
+  constexpr int64_t kSmemKeys = 48 * 1024;  // 192 KB of staged keys
+  t.smem_keys = (int)kSmemKeys;
+  const size_t smem = (size_t)(max_size < kSmemKeys ? max_size : kSmemKeys) * sizeof(uint32_t);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

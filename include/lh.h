@@ -19,7 +19,7 @@
  *    dK, dV are [B][H][N][d] in cfg->dtype.  The gathered sequence tensors
  *    Qs, Ks, Vs, dOs are [BH][S][d] bf16; Os, dQs, dKs, dVs are [BH][S][d]
  *    fp32; LSE and Delta are [BH][S] fp32.
- *  - Support: d in {64, 128}; p a power of two >= 2; 1 <= L <= 16;
+ *  - Support: d in {64, 128}; p a power of two >= 2; 1 <= L <= 8;
  *    N divisible by p^(L-1); N < 2^28; k >= 1; B*H <= 65535 * 65535.
  *    dtype LH_FP32 pools and scores in fp32 and casts the gathered sequence
  *    to bf16 for the tensor cores.
@@ -150,7 +150,10 @@ lh_status lh_pyramid_pool_from(const lh_config *cfg, int32_t first_level, const 
  *      kprime[l] parent indices at level l+1 in ascending order.  The M
  *      candidates of a level are split into C = max(1, M / chunk) contiguous
  *      chunks (the first M mod C one longer); chunk c keeps its
- *      floor(k'/C) + [c < k' mod C] highest fp32 scores, ties to the lower index. */
+ *      floor(k'/C) + [c < k' mod C] highest fp32 scores, ties to the lower index.
+ *      A chunk of at least M candidates makes C = 1: an exact global top-k per
+ *      level (chunks above 48K candidates are read from the score pyramid in
+ *      every radix pass instead of being staged in shared memory). */
 lh_status lh_score_topk(const lh_config *cfg, const float *norms, void *ws, int32_t *sel, lh_stream_t stream);
 
 /* Stage 2 without workspace, for callers that cannot allocate device memory

@@ -70,7 +70,7 @@ def test_plan_matches_oracle_sizes(lib, name):
     (dict(N=1000, L=5), 2),     # N not divisible by p^(L-1)
     (dict(L=9), 2),             # more levels than the kernels take
     (dict(k=0), 1),             # invalid budget
-    (dict(chunk=8192), 2),      # chunk above the shared-memory bound
+    (dict(chunk=-5), 1),        # negative chunk
     (dict(dtype=7), 1),         # bad enum
 ])
 def test_plan_rejects(lib, kw, status):

@@ -81,6 +81,26 @@ def test_score_topk_bit_exact(name):
         np.testing.assert_array_equal(sel[bh].cpu().numpy().astype(np.int64), pu.oracle_sel_flat(w, o["saved"]))
 
 
+@pytest.mark.parametrize("N,L,p,k", [(131072, 3, 2, 512), (65536, 4, 4, 100)])
+def test_score_topk_global_chunk_bit_exact(N, L, p, k):
+    """An exact global top-k per level (one chunk of every candidate): the
+    65536-candidate level is read from the score pyramid in every radix pass,
+    the smaller ones are staged in shared memory; indices must match the
+    oracle's sort exactly (selection only, after gap repair)."""
+    w = Workload("global_topk", 1, 2, N, 64, L, p, k, "bf16", "qk_sum", "iid", 17, chunk=1 << 20)
+    L_ = layer_of(w)
+    heads = [pu.head_case(w, bh) for bh in range(w.H)]
+    q = torch.stack([h["q"] for h in heads]).cuda()
+    kk = torch.stack([h["k"] for h in heads]).cuda()
+    _, _, _, norms = lh.pyramid_pool(L_, q, kk, kk)
+    sel = lh.score_topk(L_, norms)
+    torch.cuda.synchronize()
+    for bh, h in enumerate(heads):
+        want, _ = lo.select(pu.to_np(h["q"]), pu.to_np(h["k"]), w.p, w.L, w.k, w.chunk, w.scorer)
+        np.testing.assert_array_equal(sel[bh].cpu().numpy().astype(np.int64),
+                                      np.concatenate([np.asarray(x, np.int64) for x in want]))
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_gather(name):
     w, x, heads = case(name)
