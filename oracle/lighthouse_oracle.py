@@ -83,15 +83,35 @@ def pyramid_entry_count(N: int, p: int, L: int) -> int:
     return sum(level_lengths(N, p, L))
 
 
-def budgets(N: int, p: int, L: int, k: int) -> list[int]:
-    """k'_l = min(k, M_l), M_l = N / p^(l+1) candidates for level l (reading R3 / C4)."""
+# The three readings of what a level keeps (reading C2).  "parents" (R3, the
+# default): k'_l parents at level l+1, chosen by their max-pooled scores among
+# all N/p^(l+1) entries, each bringing its p children.  "direct": p*k'_l
+# entries of level l chosen by their own scores among all N/p^l.  "nested"
+# (coarse to fine): as "parents", but the candidate parents at level l+1 are
+# only the entries kept there (the whole top level for l = L-2).
+SELECTIONS = ("parents", "direct", "nested")
+
+
+def budgets(N: int, p: int, L: int, k: int, selection: str = "parents") -> list[int]:
+    """k'_l for l = 0..L-2: min(k, candidates).  parents / direct: N/p^(l+1)
+    candidates (reading R3 / C4); nested: the p k'_(l+1) kept entries of level
+    l+1, or the N/p^(L-1) top entries for l = L-2."""
     check_shape(N, p, L)
-    return [min(k, N // p ** (l + 1)) for l in range(L - 1)]
+    if selection not in SELECTIONS:
+        raise ValueError(f"unknown selection {selection!r}")
+    if selection != "nested":
+        return [min(k, N // p ** (l + 1)) for l in range(L - 1)]
+    out = [0] * (L - 1)
+    cand = N // p ** (L - 1)
+    for lvl in range(L - 2, -1, -1):
+        out[lvl] = min(k, cand)
+        cand = p * out[lvl]
+    return out
 
 
-def gathered_length(N: int, p: int, L: int, k: int) -> int:
-    """S = N/p^(L-1) + sum_l p*k'_l  (LH-post Key formulas, with k' = min(k, M))."""
-    return N // p ** (L - 1) + sum(p * kp for kp in budgets(N, p, L, k))
+def gathered_length(N: int, p: int, L: int, k: int, selection: str = "parents") -> int:
+    """S = N/p^(L-1) + sum_l p*k'_l  (LH-post Key formulas, with k' = min(k, candidates))."""
+    return N // p ** (L - 1) + sum(p * kp for kp in budgets(N, p, L, k, selection))
 
 
 # ----------------------------------------------------------------------------
@@ -172,22 +192,41 @@ def stratified_topk(scores: np.ndarray, k: int, T: int = DEFAULT_CHUNK) -> np.nd
     return np.concatenate(kept) if kept else np.zeros(0, np.int64)
 
 
-def select(Q, K, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum"):
-    """Selection for one head.  Returns (sel, spyr): sel[l] are the kept parent
-    indices at level l+1 (ascending) for l = 0..L-2; spyr is the score pyramid."""
+def select(Q, K, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum",
+           selection: str = "parents"):
+    """Selection for one head.  Returns (sel, spyr); spyr is the score pyramid.
+    parents / nested: sel[l] are the kept parent indices at level l+1
+    (ascending) for l = 0..L-2; direct: sel[l] are the kept level-l entries."""
+    N = np.asarray(Q).shape[0]
     spyr = score_pyramid(level0_scores(Q, K, scorer), p, L)
-    sel = [stratified_topk(spyr[l + 1], k, T) for l in range(L - 1)]
+    kp = budgets(N, p, L, k, selection)
+    if selection == "parents":
+        sel = [stratified_topk(spyr[l + 1], kp[l], T) for l in range(L - 1)]
+    elif selection == "direct":
+        sel = [stratified_topk(spyr[l], p * kp[l], T) for l in range(L - 1)]
+    else:
+        # top down: the candidates of level l+1 are its kept entries, chunked
+        # and ranked by position in that ascending list (ties: lower index)
+        sel = [None] * (L - 1)
+        kept = np.arange(N // p ** (L - 1), dtype=np.int64)
+        for lvl in range(L - 2, -1, -1):
+            pos = stratified_topk(spyr[lvl + 1][kept], kp[lvl], T)
+            sel[lvl] = kept[pos]
+            kept = (sel[lvl][:, None] * p + np.arange(p)[None, :]).reshape(-1)
     return sel, spyr
 
 
-def selected_entries(sel, N: int, p: int, L: int) -> list[np.ndarray]:
-    """Entries kept at every level: the p children of each kept parent for
-    l < L-1, and the whole top level (LH-post Key formulas: the first term of S
-    is the top level, kept entirely)."""
+def selected_entries(sel, N: int, p: int, L: int, selection: str = "parents") -> list[np.ndarray]:
+    """Entries kept at every level: for l < L-1 the p children of each kept
+    parent (parents, nested) or the kept entries themselves (direct); and the
+    whole top level (LH-post Key formulas: the first term of S is the top
+    level, kept entirely)."""
     out = []
     for l in range(L - 1):
-        parents = np.asarray(sel[l], np.int64)
-        out.append((parents[:, None] * p + np.arange(p)[None, :]).reshape(-1))
+        kept = np.asarray(sel[l], np.int64)
+        if selection != "direct":
+            kept = (kept[:, None] * p + np.arange(p)[None, :]).reshape(-1)
+        out.append(kept)
     out.append(np.arange(N // p ** (L - 1), dtype=np.int64))
     return out
 
@@ -287,22 +326,22 @@ def scatter_back(Os, seq_level, seq_index, N: int, p: int, L: int) -> np.ndarray
 # ----------------------------------------------------------------------------
 
 def forward_head(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum",
-                 sel=None, attn_dtype="bf16"):
+                 sel=None, attn_dtype="bf16", selection: str = "parents"):
     """One head of the layer.  Returns (Y, saved) with everything the backward
     and the parity tests need.  ``sel`` freezes the selection (used by the
     causality and finite-difference checks); by default it is computed.
     ``attn_dtype`` = "bf16" rounds the attention inputs (reading R11); None
-    keeps them exact."""
+    keeps them exact.  ``selection`` is the reading of C2 (see SELECTIONS)."""
     Q = np.asarray(Q, np.float64)
     K = np.asarray(K, np.float64)
     V = np.asarray(V, np.float64)
     N = Q.shape[0]
     pq, pk, pv = (pyramid_pool(X, p, L) for X in (Q, K, V))
     if sel is None:
-        sel, spyr = select(Q, K, p, L, k, T, scorer)
+        sel, spyr = select(Q, K, p, L, k, T, scorer, selection)
     else:
         spyr = None
-    seq_level, seq_index = causal_order(selected_entries(sel, N, p, L), p)
+    seq_level, seq_index = causal_order(selected_entries(sel, N, p, L, selection), p)
     Qs, Ks, Vs = gather(pq, seq_level, seq_index), gather(pk, seq_level, seq_index), gather(pv, seq_level, seq_index)
     if attn_dtype == "bf16":
         Qs, Ks, Vs = round_bf16(Qs), round_bf16(Ks), round_bf16(Vs)
@@ -310,7 +349,7 @@ def forward_head(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer
         raise ValueError(f"unknown attn_dtype {attn_dtype!r}")
     Os, lse = causal_attention(Qs, Ks, Vs)
     Y = scatter_back(Os, seq_level, seq_index, N, p, L)
-    saved = dict(N=N, p=p, L=L, k=k, T=T, scorer=scorer, attn_dtype=attn_dtype, sel=sel, spyr=spyr,
+    saved = dict(N=N, p=p, L=L, k=k, T=T, scorer=scorer, attn_dtype=attn_dtype, selection=selection, sel=sel, spyr=spyr,
                  pyr_q=pq, pyr_k=pk, pyr_v=pv,
                  seq_level=seq_level, seq_index=seq_index,
                  slot_of=slot_table(seq_level, seq_index, N, p, L),
@@ -397,10 +436,11 @@ def backward_head(dY, saved):
 # several heads: [BH, N, d], selection per head (reading R9)
 # ----------------------------------------------------------------------------
 
-def forward(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum", attn_dtype="bf16"):
+def forward(Q, K, V, p: int, L: int, k: int, T: int = DEFAULT_CHUNK, scorer: str = "qk_sum", attn_dtype="bf16",
+            selection: str = "parents"):
     Ys, saves = [], []
     for h in range(Q.shape[0]):
-        Y, sv = forward_head(Q[h], K[h], V[h], p, L, k, T, scorer, attn_dtype=attn_dtype)
+        Y, sv = forward_head(Q[h], K[h], V[h], p, L, k, T, scorer, attn_dtype=attn_dtype, selection=selection)
         Ys.append(Y)
         saves.append(sv)
     return np.stack(Ys), saves

@@ -99,7 +99,7 @@ def m_backward_no_rowsum(Qs, Ks, Vs, dOs):
     return scale * dZ @ Ks, scale * dZ.T @ Qs, P.T @ dOs
 
 
-def m_budget_no_min(N, p, L, k):
+def m_budget_no_min(N, p, L, k, selection="parents"):
     return [k for _ in range(L - 1)]
 
 

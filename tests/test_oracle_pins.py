@@ -159,6 +159,80 @@ def test_selection_invariants():
         assert np.all(groups % p == np.arange(p)) and np.all(groups[:, 0] // p == sel[l])
 
 
+# ---------------------------------------------------- the other readings of C2
+
+def test_budgets_nested_follow_the_kept_counts():
+    # by hand: N=64, p=2, L=4, k=3 -> top level has 8 entries; level 2 keeps
+    # min(3, 8)=3 parents -> 6 candidates at level 2; level 1 keeps min(3, 6)=3
+    # -> 6 candidates at level 1; level 0 keeps min(3, 6)=3
+    assert lo.budgets(64, 2, 4, 3, "nested") == [3, 3, 3]
+    # budgets above the candidates: N=16 -> 2 top entries, k'_2 = min(5, 2) = 2,
+    # then 4 candidates at level 2 (k'_1 = 4), then 8 at level 1 (k'_0 = 5)
+    assert lo.budgets(16, 2, 4, 5, "nested") == [5, 4, 2]
+    assert lo.gathered_length(16, 2, 4, 5, "nested") == 2 + 2 * (5 + 4 + 2)
+    assert lo.budgets(64, 2, 4, 3, "direct") == lo.budgets(64, 2, 4, 3)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_direct_selection_bruteforce(seed):
+    """direct: level l keeps the p*k'_l entries of level l with the largest own
+    scores (per stratification chunk), by exhaustive search."""
+    r = rng(300 + seed)
+    N, p, L = 16, 2, 3
+    k = int(r.integers(1, 4))
+    T = int(r.integers(2, 9))
+    Q = r.integers(-2, 3, (N, 2)).astype(np.float64)  # small integer vectors: many equal norms
+    K = r.integers(-2, 3, (N, 2)).astype(np.float64)
+    sel, spyr = lo.select(Q, K, p, L, k, T, selection="direct")
+    kp = lo.budgets(N, p, L, k, "direct")
+    for lvl in range(L - 1):
+        np.testing.assert_array_equal(sel[lvl], brute_topk(spyr[lvl], p * kp[lvl], T))
+    ent = lo.selected_entries(sel, N, p, L, "direct")
+    assert sum(len(e) for e in ent) == lo.gathered_length(N, p, L, k, "direct")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_nested_selection_bruteforce(seed):
+    """nested: going down from the whole top level, level l keeps the p children
+    of the k'_l best of the entries kept at level l+1 (per stratification chunk
+    of that ascending list), by exhaustive search."""
+    r = rng(400 + seed)
+    N, p, L = 32, 2, 4
+    k = int(r.integers(1, 4))
+    T = int(r.integers(2, 9))
+    Q = r.integers(-2, 3, (N, 2)).astype(np.float64)
+    K = r.integers(-2, 3, (N, 2)).astype(np.float64)
+    sel, spyr = lo.select(Q, K, p, L, k, T, selection="nested")
+    kp = lo.budgets(N, p, L, k, "nested")
+    kept = np.arange(N // p ** (L - 1))
+    for lvl in range(L - 2, -1, -1):
+        cand = kept
+        want = cand[brute_topk(spyr[lvl + 1][cand], kp[lvl], T)]
+        np.testing.assert_array_equal(sel[lvl], want)
+        assert set(sel[lvl].tolist()) <= set(cand.tolist())
+        kept = np.sort(np.concatenate([sel[lvl] * p + c for c in range(p)]))
+    ent = lo.selected_entries(sel, N, p, L, "nested")
+    assert sum(len(e) for e in ent) == lo.gathered_length(N, p, L, k, "nested")
+
+
+def test_readings_agree_when_everything_fits_and_nested_is_parents_at_L2():
+    r = rng(9)
+    N, p, L = 256, 4, 4
+    Q, K = r.standard_normal((N, 8)), r.standard_normal((N, 8))
+    ents = {}
+    for sel_mode in lo.SELECTIONS:
+        sel, _ = lo.select(Q, K, p, L, 10_000, T=64, selection=sel_mode)
+        ents[sel_mode] = lo.selected_entries(sel, N, p, L, sel_mode)
+    for l in range(L):
+        np.testing.assert_array_equal(ents["parents"][l], np.arange(N // p ** l))
+        np.testing.assert_array_equal(ents["direct"][l], ents["parents"][l])
+        np.testing.assert_array_equal(ents["nested"][l], ents["parents"][l])
+    # with two levels the nested candidates are the whole top level
+    a, _ = lo.select(Q, K, p, 2, 7, T=16, selection="parents")
+    b, _ = lo.select(Q, K, p, 2, 7, T=16, selection="nested")
+    np.testing.assert_array_equal(a[0], b[0])
+
+
 # ---------------------------------------------------------------- gather order
 
 def test_causal_order_invariants():
