@@ -268,7 +268,8 @@ def oracle_sample(w: synth.Workload, heads: int = 1, max_seconds: float = 60.0) 
         x = synth.head_inputs(w, h)
         arr = {n: t.double().numpy() for n, t in x.items()}
         t0 = time.perf_counter()
-        Y, sv = lo.forward_head(arr["q"], arr["k"], arr["v"], w.p, w.L, w.k, w.chunk, w.scorer)
+        Y, sv = lo.forward_head(arr["q"], arr["k"], arr["v"], w.p, w.L, w.k, w.chunk, w.scorer,
+                                selection=w.selection)
         lo.backward_head(arr["dy"], sv)
         times.append(time.perf_counter() - t0)
         if sum(times) > max_seconds:
@@ -280,6 +281,8 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
+    if args.selection != "parents":
+        w = w.with_(selection=args.selection)
     # one head per step; the oracle keeps no state between steps, so warm-up
     # steps only load the code paths
     for _ in range(min(args.warmup, 1)):
@@ -307,7 +310,8 @@ def run_reference(args, world, rank):
 def workload_config(w: synth.Workload) -> dict:
     info = lh.plan(lh.Layer.of(w))
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "L": w.L, "p": w.p, "k": w.k,
-            "chunk": w.chunk, "scorer": w.scorer, "S": int(info.S), "parallelism": "replicas (one layer per GPU)",
+            "chunk": w.chunk, "scorer": w.scorer, "selection": w.selection, "S": int(info.S),
+            "parallelism": "replicas (one layer per GPU)",
             "l2": "inputs larger than L2 (Q,K,V,dY %.1f GB per GPU)" % (4 * w.B * w.H * w.N * w.d * 2 / 1e9)}
 
 
@@ -325,6 +329,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead (a smaller cut for profiling)")
+    ap.add_argument("--selection", default="parents", choices=["parents", "direct", "nested"],
+                    help="what a level keeps (the default reading, or one of the two others)")
     args = ap.parse_args()
 
     world, rank, local = dist_setup()
@@ -339,6 +345,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.heads:
         w = w.with_(H=args.heads)
+    if args.selection != "parents":
+        w = w.with_(selection=args.selection)
     layer = lh.Layer.of(w)
     x = synth.cuda_inputs(w, dev, seed=w.seed + 16 * rank)
     bufs = lh.Buffers(layer, dev)

@@ -19,11 +19,13 @@ STATUS_NAMES = {0: "LH_OK", 1: "LH_ERR_INVALID_ARG", 2: "LH_ERR_UNSUPPORTED", 3:
                 4: "LH_ERR_CUDA", 5: "LH_ERR_TIMEOUT", 6: "LH_ERR_DEVICE"}
 DTYPES = {"bf16": 0, "fp32": 1}
 SCORERS = {"qk_sum": 0, "k": 1, "q": 2}
+SELECTIONS = {"parents": 0, "direct": 1, "nested": 2}
 
 
 class LhConfig(ctypes.Structure):
     _fields_ = [("B", c_int64), ("H", c_int64), ("N", c_int64), ("d", c_int32), ("L", c_int32), ("p", c_int32),
-                ("k", c_int32), ("chunk", c_int32), ("dtype", c_int32), ("scorer", c_int32)]
+                ("k", c_int32), ("chunk", c_int32), ("dtype", c_int32), ("scorer", c_int32),
+                ("selection", c_int32)]
 
 
 _SIZES = ["pyr_bytes", "norms_bytes", "topk_ws_bytes", "sel_bytes", "seq_bytes", "os_bytes", "seq_map_bytes", "slot_of_bytes",

@@ -32,10 +32,11 @@ class Layer:
     chunk: int = 2048
     dtype: str = "bf16"
     scorer: str = "qk_sum"
+    selection: str = "parents"
 
     def cfg(self) -> LhConfig:
         return LhConfig(self.B, self.H, self.N, self.d, self.L, self.p, self.k, self.chunk,
-                        _lib.DTYPES[self.dtype], _lib.SCORERS[self.scorer])
+                        _lib.DTYPES[self.dtype], _lib.SCORERS[self.scorer], _lib.SELECTIONS[self.selection])
 
     @property
     def torch_dtype(self):
@@ -48,7 +49,8 @@ class Layer:
     @staticmethod
     def of(w) -> "Layer":
         """From a synth.Workload (or anything with the same fields)."""
-        return Layer(w.B, w.H, w.N, w.d, w.L, w.p, w.k, w.chunk, w.dtype, w.scorer)
+        return Layer(w.B, w.H, w.N, w.d, w.L, w.p, w.k, w.chunk, w.dtype, w.scorer,
+                     getattr(w, "selection", "parents"))
 
 
 def plan(layer: Layer) -> LhPlanInfo:

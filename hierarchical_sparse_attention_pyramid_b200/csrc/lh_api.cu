@@ -51,6 +51,8 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
     return fail(LH_ERR_INVALID_ARG, "lh_plan: sizes must be positive");
   if (cfg->dtype != LH_BF16 && cfg->dtype != LH_FP32) return fail(LH_ERR_INVALID_ARG, "lh_plan: bad dtype");
   if (cfg->scorer < LH_SCORE_QK_SUM || cfg->scorer > LH_SCORE_Q) return fail(LH_ERR_INVALID_ARG, "lh_plan: bad scorer");
+  if (cfg->selection < LH_SELECT_PARENTS || cfg->selection > LH_SELECT_NESTED)
+    return fail(LH_ERR_INVALID_ARG, "lh_plan: bad selection");
   if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_plan: d must be 64 or 128");
   if (p < 2 || (p & (p - 1)) != 0) return fail(LH_ERR_UNSUPPORTED, "lh_plan: p must be a power of two >= 2");
   if (L > 8) return fail(LH_ERR_UNSUPPORTED, "lh_plan: L must be <= 8");
@@ -72,12 +74,35 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
       upper += info->level_len[l];
     }
   }
+  // k'_l = min(k, candidates): N/p^(l+1) (parents, direct), or the kept
+  // entries of level l+1 (nested: the whole top level for l = L-2)
+  const int sel_mode = cfg->selection;
+  if (sel_mode == LH_SELECT_NESTED) {
+    int64_t cand = info->level_len[L - 1];
+    for (int l = L - 2; l >= 0; --l) {
+      info->kprime[l] = (int32_t)(k < cand ? k : cand);
+      cand = (int64_t)p * info->kprime[l];
+    }
+  } else {
+    for (int l = 0; l + 1 < L; ++l) {
+      const int64_t M = info->level_len[l + 1];
+      info->kprime[l] = (int32_t)(k < M ? k : M);
+    }
+  }
+  if (sel_mode == LH_SELECT_NESTED) {
+    // the nested top-k stages every chunk of a level's candidates in shared memory
+    for (int l = 0; l + 1 < L; ++l) {
+      const int64_t M = l + 1 == L - 1 ? info->level_len[L - 1] : (int64_t)p * info->kprime[l + 1];
+      const int64_t C = M / chunk > 1 ? M / chunk : 1;
+      if ((M + C - 1) / C > 48 * 1024)
+        return fail(LH_ERR_UNSUPPORTED, "lh_plan: nested selection needs chunks of at most 49152 candidates");
+    }
+  }
+  // sel holds k'_l parents per level, or the p k'_l kept entries (direct)
   int64_t S = info->level_len[L - 1];
   for (int l = 0; l + 1 < L; ++l) {
-    const int64_t M = info->level_len[l + 1];
-    info->kprime[l] = (int32_t)(k < M ? k : M);
     info->sel_off[l] = selsum;
-    selsum += info->kprime[l];
+    selsum += sel_mode == LH_SELECT_DIRECT ? (int64_t)p * info->kprime[l] : info->kprime[l];
     S += (int64_t)p * info->kprime[l];
   }
   if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_plan: S too large");
@@ -89,7 +114,10 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   const size_t e = cfg->dtype == LH_BF16 ? 2 : 4;
   info->pyr_bytes = (size_t)BH * upper * d * e;
   info->norms_bytes = (size_t)2 * BH * N * 4;
-  info->topk_ws_bytes = LH_ERR_WORD_BYTES + align_up((size_t)BH * upper * 4);
+  // score pyramid (levels >= 1), plus the level-0 scores when level 0 is
+  // selected directly
+  info->topk_ws_bytes = LH_ERR_WORD_BYTES + align_up((size_t)BH * upper * 4) +
+                        (sel_mode == LH_SELECT_DIRECT ? align_up((size_t)BH * N * 4) : 0);
   info->sel_bytes = (size_t)BH * selsum * 4;
   info->seq_bytes = (size_t)BH * S * d * 2;
   info->os_bytes = (size_t)BH * S * d * 4;
@@ -142,7 +170,7 @@ lh_status plan_impl(const lh_config* cfg, lh_plan_info* info, Dims* D) {
   if (D) {
     D->BH = BH; D->N = N; D->S = S;
     D->d = d; D->L = L; D->p = p; D->log2p = log2p; D->chunk = chunk;
-    D->dtype = cfg->dtype; D->scorer = cfg->scorer;
+    D->dtype = cfg->dtype; D->scorer = cfg->scorer; D->selection = cfg->selection;
     for (int l = 0; l < LH_MAX_LEVELS; ++l) {
       D->level_len[l] = info->level_len[l];
       D->level_off[l] = info->level_off[l];

@@ -17,6 +17,7 @@ struct Dims {
   int d, L, p, log2p, chunk;
   int dtype;   // LH_BF16 / LH_FP32
   int scorer;  // lh_scorer
+  int selection;  // lh_selection
   int64_t level_len[LH_MAX_LEVELS];
   int64_t level_off[LH_MAX_LEVELS];  // into slot_of rows
   int64_t upper_off[LH_MAX_LEVELS];  // into pyramid rows (levels >= 1)

@@ -10,7 +10,8 @@
 // Entry (l, i) covers tokens [i p^l, (i+1) p^l); its key is
 // (e = (i+1) p^l - 1, -l) and its range is R(l,i) = [e, e + p^l).  The slot of
 // an entry is the number of kept entries with a smaller key, counted level by
-// level with binary searches over the sorted parent lists, so no sort runs.
+// level with binary searches over the sorted parent lists (or, when levels are
+// selected directly, the sorted lists of kept entries), so no sort runs.
 #include "lh_common.cuh"
 
 namespace lh {
@@ -35,6 +36,7 @@ struct GatherArgs {
   int64_t cnt_off[LH_MAX_LEVELS + 1];  // first sequence entry id of each level's kept list
   int32_t kprime[LH_MAX_LEVELS];
   int L, log2p, first_level;
+  int direct;  // sel lists the kept entries themselves (not parents)
 };
 
 // kept entries of level lv with index < X
@@ -42,6 +44,15 @@ __device__ __forceinline__ int64_t kept_below(const GatherArgs& a, const int32_t
   if (X <= 0) return 0;
   if (lv == a.L - 1) return min(X, a.level_len[lv]);
   const int32_t* s = sel_h + a.sel_off[lv];
+  if (a.direct) {  // lower_bound of X in the sorted kept list
+    int lo = 0, hi = a.kprime[lv] << a.log2p;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((int64_t)s[mid] < X) lo = mid + 1;
+      else hi = mid;
+    }
+    return lo;
+  }
   const int n = a.kprime[lv];
   const int64_t m = X >> a.log2p, r = X & ((1 << a.log2p) - 1);
   int lo = 0, hi = n;  // lower_bound of m
@@ -67,7 +78,9 @@ __global__ void __launch_bounds__(kWarps * 32) gather_kernel(GatherArgs a) {
   while (l + 1 < a.L && id >= a.cnt_off[l + 1]) ++l;
   const int64_t j = id - a.cnt_off[l];
   int64_t i;
-  if (l < a.L - 1) i = ((int64_t)sel_h[a.sel_off[l] + (j >> a.log2p)] << a.log2p) + (j & ((1 << a.log2p) - 1));
+  if (l < a.L - 1)
+    i = a.direct ? (int64_t)sel_h[a.sel_off[l] + j]
+                 : ((int64_t)sel_h[a.sel_off[l] + (j >> a.log2p)] << a.log2p) + (j & ((1 << a.log2p) - 1));
   else i = j;
   const int64_t e = ((i + 1) << (l * a.log2p)) - 1;
   // one level per lane: kept entries whose key is below (e, -l)
@@ -360,6 +373,7 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
   a.L = D.L;
   a.log2p = D.log2p;
   a.first_level = first_level;
+  a.direct = D.selection == LH_SELECT_DIRECT;
   cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * D.pyr_entries * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (D.BH * D.S + kWarps - 1) / kWarps;

@@ -62,7 +62,8 @@ extern "C" lh_status lh_score_topk_static(const lh_config* cfg, const float* nor
     set_error_message("lh_score_topk_static: norms or sel is NULL or not 16-byte aligned");
     return LH_ERR_INVALID_ARG;
   }
-  const size_t need = (size_t)D.BH * D.upper_entries * sizeof(float);
+  // the score pyramid, and (direct selection) the level-0 scores after it
+  const size_t need = info.topk_ws_bytes - LH_ERR_WORD_BYTES;
   if (need > kStaticScratchBytes) {
     set_error_message("lh_score_topk_static: the score pyramid needs %zu bytes but the static scratch holds %zu; "
                       "use lh_score_topk with a caller-provided ws",

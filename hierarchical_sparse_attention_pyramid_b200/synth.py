@@ -49,6 +49,7 @@ class Workload:
     structure: str      # "iid", "lognormal_token" or "outlier_tokens"
     seed: int
     chunk: int = 2048
+    selection: str = "parents"  # "parents", "direct" or "nested"
 
     @property
     def torch_dtype(self):

@@ -64,6 +64,15 @@ typedef enum {
   LH_SCORE_Q = 2       /* ||Q_t|| */
 } lh_scorer;
 
+/* What a level below the top keeps (the pages fix only the count p*k per
+ * level: LH-post "Key formulas"; these are the three readings of it). */
+typedef enum {
+  LH_SELECT_PARENTS = 0, /* k' parents at level l+1 by max-pooled score, each with its p children (default) */
+  LH_SELECT_DIRECT = 1,  /* p*k' entries of level l by their own score */
+  LH_SELECT_NESTED = 2   /* as PARENTS, parents only among the entries kept at level l+1 (the whole
+                            top level for l = L-2); k' = min(k, candidates) */
+} lh_selection;
+
 typedef struct {
   int64_t B, H, N; /* batch, heads, sequence length */
   int32_t d;       /* head dimension */
@@ -73,6 +82,7 @@ typedef struct {
   int32_t chunk;   /* top-k stratification chunk T (candidates); 0 = 2048 */
   int32_t dtype;   /* lh_dtype of Q, K, V, Y, dY, dQ, dK, dV */
   int32_t scorer;  /* lh_scorer */
+  int32_t selection; /* lh_selection */
 } lh_config;
 
 #define LH_MAX_LEVELS 16

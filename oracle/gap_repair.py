@@ -19,16 +19,38 @@ import torch
 from . import lighthouse_oracle as lo
 
 
-def near_ties(Q, K, p, L, k, T=lo.DEFAULT_CHUNK, scorer="qk_sum", rel_gap=1e-5):
-    """Level-0 tokens to push down: one per chunk whose q-th/(q+1)-th gap is small."""
+def _decisions(Q, K, p, L, k, T, scorer, selection):
+    """Every top-k the selection makes: (level of the candidates, their level
+    indices in ascending order, their scores, the budget over them)."""
+    N = Q.shape[0]
     s0 = lo.level0_scores(Q, K, scorer)
     spyr = lo.score_pyramid(s0, p, L)
+    kp = lo.budgets(N, p, L, k, selection)
+    out = []
+    if selection == "parents":
+        for l in range(L - 1):
+            out.append((l + 1, np.arange(spyr[l + 1].shape[0]), spyr[l + 1], kp[l]))
+    elif selection == "direct":
+        for l in range(L - 1):
+            out.append((l, np.arange(spyr[l].shape[0]), spyr[l], p * kp[l]))
+    else:
+        kept = np.arange(N // p ** (L - 1))
+        for l in range(L - 2, -1, -1):
+            sc = spyr[l + 1][kept]
+            out.append((l + 1, kept, sc, kp[l]))
+            sel = kept[lo.stratified_topk(sc, kp[l], T)]
+            kept = (sel[:, None] * p + np.arange(p)[None, :]).reshape(-1)
+    return s0, out
+
+
+def near_ties(Q, K, p, L, k, T=lo.DEFAULT_CHUNK, scorer="qk_sum", rel_gap=1e-5, selection="parents"):
+    """Level-0 tokens to push down: one per chunk whose q-th/(q+1)-th gap is small."""
+    s0, decisions = _decisions(Q, K, p, L, k, T, scorer, selection)
     tokens = []
-    for l in range(L - 1):
-        scores = spyr[l + 1]
+    for lvl, cand, scores, budget in decisions:
         M = scores.shape[0]
         sizes = lo.chunk_sizes(M, T)
-        qs = lo.quotas(min(k, M), len(sizes))
+        qs = lo.quotas(min(budget, M), len(sizes))
         start = 0
         for size, q in zip(sizes, qs):
             if 0 < q < size:
@@ -37,8 +59,8 @@ def near_ties(Q, K, p, L, k, T=lo.DEFAULT_CHUNK, scorer="qk_sum", rel_gap=1e-5):
                 a = scores[start + order[q - 1]]
                 b = scores[start + order[q]]
                 if a <= 0 or (a - b) / a < rel_gap:
-                    m = start + int(order[q])
-                    block = p ** (l + 1)
+                    m = int(cand[start + int(order[q])])
+                    block = p ** lvl
                     t0 = m * block
                     tokens.append(t0 + int(np.argmax(s0[t0:t0 + block])))
             start += size
@@ -46,14 +68,14 @@ def near_ties(Q, K, p, L, k, T=lo.DEFAULT_CHUNK, scorer="qk_sum", rel_gap=1e-5):
 
 
 def repair_head(Q: torch.Tensor, K: torch.Tensor, p, L, k, T=lo.DEFAULT_CHUNK, scorer="qk_sum",
-                rel_gap=1e-5, max_rounds=16, factor=0.98):
+                rel_gap=1e-5, max_rounds=16, factor=0.98, selection="parents"):
     """Repair one head's [N, d] Q and K (CPU tensors, any float dtype).
     Returns (Q, K, rows_repaired)."""
     Q = Q.clone()
     K = K.clone()
     repaired = 0
     for _ in range(max_rounds):
-        toks = near_ties(Q.double().numpy(), K.double().numpy(), p, L, k, T, scorer, rel_gap)
+        toks = near_ties(Q.double().numpy(), K.double().numpy(), p, L, k, T, scorer, rel_gap, selection)
         if not toks:
             return Q, K, repaired
         t = torch.tensor(toks, dtype=torch.long)

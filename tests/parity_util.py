@@ -46,7 +46,8 @@ def head_case(w: synth.Workload, bh: int):
     """CPU inputs of one head with the top-k near-ties removed (dtype of w)."""
     h = synth.head_inputs(w, bh)
     if w.L > 1:
-        h["q"], h["k"], n = gap_repair.repair_head(h["q"], h["k"], w.p, w.L, w.k, w.chunk, w.scorer)
+        h["q"], h["k"], n = gap_repair.repair_head(h["q"], h["k"], w.p, w.L, w.k, w.chunk, w.scorer,
+                                                   selection=getattr(w, "selection", "parents"))
         h["repaired"] = n
     return h
 
@@ -59,7 +60,8 @@ def all_heads_case(w: synth.Workload):
 
 def oracle_head(w: synth.Workload, q, k, v, dy=None):
     """fp64 oracle of one head from [N, d] tensors."""
-    Y, sv = lo.forward_head(to_np(q), to_np(k), to_np(v), w.p, w.L, w.k, w.chunk, w.scorer)
+    Y, sv = lo.forward_head(to_np(q), to_np(k), to_np(v), w.p, w.L, w.k, w.chunk, w.scorer,
+                            selection=getattr(w, "selection", "parents"))
     out = dict(Y=Y, saved=sv)
     if dy is not None:
         dQ, dK, dV, ex = lo.backward_head(to_np(dy), sv)

@@ -10,7 +10,7 @@ import subprocess
 import pytest
 
 from hierarchical_sparse_attention_pyramid_b200 import _lib, plan, Layer
-from hierarchical_sparse_attention_pyramid_b200.synth import WORKLOADS
+from hierarchical_sparse_attention_pyramid_b200.synth import WORKLOADS, Workload
 from oracle import lighthouse_oracle as lo
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -64,6 +64,17 @@ def test_plan_matches_oracle_sizes(lib, name):
     assert info.first_level == want
 
 
+@pytest.mark.parametrize("selection", ["direct", "nested"])
+def test_plan_of_the_other_readings(lib, selection):
+    for N, p, L, k in ((8192, 2, 4, 48), (8192, 2, 5, 40), (1 << 16, 4, 5, 300), (4096, 2, 3, 5000)):
+        w = Workload("r", 1, 2, N, 64, L, p, k, "bf16", "qk_sum", "iid", 0, selection=selection)
+        info = plan(Layer.of(w))
+        kp = lo.budgets(N, p, L, k, selection)
+        assert list(info.kprime)[: L - 1] == kp
+        assert info.S == lo.gathered_length(N, p, L, k, selection)
+        assert info.sel_per_head == sum(kp) * (p if selection == "direct" else 1)
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), 2),            # unsupported head dim
     (dict(p=3), 2),             # p not a power of two
@@ -72,9 +83,10 @@ def test_plan_matches_oracle_sizes(lib, name):
     (dict(k=0), 1),             # invalid budget
     (dict(chunk=-5), 1),        # negative chunk
     (dict(dtype=7), 1),         # bad enum
+    (dict(selection=3), 1),     # bad enum
 ])
 def test_plan_rejects(lib, kw, status):
-    base = dict(B=1, H=2, N=4096, d=128, L=3, p=2, k=16, chunk=0, dtype=0, scorer=0)
+    base = dict(B=1, H=2, N=4096, d=128, L=3, p=2, k=16, chunk=0, dtype=0, scorer=0, selection=0)
     base.update(kw)
     cfg = _lib.LhConfig(**base)
     info = _lib.LhPlanInfo()

@@ -25,6 +25,11 @@ SMALL = {
         Workload("keep_all_kscore", 2, 1, 512, 64, 3, 2, 1000, "bf16", "k", "iid", 14),
         Workload("dense_L1", 1, 2, 700, 64, 1, 2, 1, "bf16", "qk_sum", "iid", 15),
         Workload("qscore_fp32_d128", 1, 1, 2048, 128, 4, 2, 20, "fp32", "q", "iid", 16, chunk=128),
+        # the two other readings of what a level keeps
+        Workload("direct_sel", 1, 2, 8192, 128, 4, 2, 48, "bf16", "qk_sum", "iid", 18, chunk=512,
+                 selection="direct"),
+        Workload("nested_sel", 1, 2, 8192, 64, 5, 2, 40, "bf16", "k", "lognormal_token", 19, chunk=32,
+                 selection="nested"),
     )
 }
 
