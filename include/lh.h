@@ -156,11 +156,14 @@ lh_status lh_pyramid_pool_from(const lh_config *cfg, int32_t first_level, const 
  * stratified: every interval contributes a fixed number).
  * In:  norms from lh_pyramid_pool; ws of topk_ws_bytes (score pyramid scratch,
  *      preceded by the error word).
- * Out: sel [BH][sel_per_head] int32: for level l < L-1, at sel_off[l],
- *      kprime[l] parent indices at level l+1 in ascending order.  The M
- *      candidates of a level are split into C = max(1, M / chunk) contiguous
- *      chunks (the first M mod C one longer); chunk c keeps its
- *      floor(k'/C) + [c < k' mod C] highest fp32 scores, ties to the lower index.
+ * Out: sel [BH][sel_per_head] int32: for level l < L-1, at sel_off[l], in
+ *      ascending order, kprime[l] parent indices at level l+1 (PARENTS,
+ *      NESTED) or p * kprime[l] entry indices at level l (DIRECT).  The M
+ *      candidates of a level (all N/p^(l+1) entries of level l+1; all N/p^l of
+ *      level l for DIRECT; the kept entries of level l+1 in ascending order for
+ *      NESTED) are split into C = max(1, M / chunk) contiguous chunks (the
+ *      first M mod C one longer); chunk c keeps its floor(b/C) + [c < b mod C]
+ *      highest fp32 scores of the budget b, ties to the lower index.
  *      A chunk of at least M candidates makes C = 1: an exact global top-k per
  *      level (chunks above 48K candidates are read from the score pyramid in
  *      every radix pass instead of being staged in shared memory). */
@@ -184,8 +187,9 @@ lh_status lh_score_topk_static(const lh_config *cfg, const float *norms, int32_t
 /* Stage 3 - gather the kept entries into one causally ordered sequence.
  * Cite: LH-post "How it works" (3) (kept entries sorted into causal order
  * form a contiguous sequence of length S); LH-summary "Technical details" (3).
- * Kept entries: the p children (l, m*p + c) of every parent m in sel level l,
- * and every entry of the top level L-1.  Entry (l, i) has key
+ * Kept entries: the p children (l, m*p + c) of every parent m in sel level l
+ * (or, with LH_SELECT_DIRECT, the entries listed in sel level l), and every
+ * entry of the top level L-1.  Entry (l, i) has key
  * (e = (i+1) p^l - 1, -l); slots are the ranks of the keys.
  * In:  q, k, v (level 0) and pyr_q/k/v (levels >= 1), sel.
  * Out: qs, ks, vs [BH][S][d] bf16; seq_map [BH][S] int32 = (l << 28) | i;
