@@ -8,3 +8,4 @@ seeded synthetic inputs.
 from .api import (Buffers, Layer, LighthouseAttentionFn, attn_bwd, attn_fwd, backward, check_error, forward,  # noqa: F401
                   gather, lighthouse_attention, plan, pool_adjoint, pyramid_pool, scatter_back,
                   scatter_back_adjoint, score_topk)
+from . import pisa  # noqa: F401

@@ -44,8 +44,20 @@ class LhPlanInfo(ctypes.Structure):
                 + [(n, c_size_t) for n in _SIZES] + [("first_level", c_int32)])
 
 
+class LhPisaConfig(ctypes.Structure):
+    _fields_ = [("B", c_int64), ("H", c_int64), ("N", c_int64), ("d", c_int32), ("p", c_int32), ("L", c_int32),
+                ("block", c_int32), ("group", c_int32), ("topk", c_int32)]
+
+
+class LhPisaInfo(ctypes.Structure):
+    _fields_ = [("n_groups", c_int64), ("blocks", c_int64 * MAX_LEVELS), ("level_off", c_int64 * MAX_LEVELS),
+                ("upper_entries", c_int64), ("pyr_bytes", c_size_t), ("kept_elems", c_size_t),
+                ("max_candidates", c_int32)]
+
+
 _P = c_void_p
 _CFG = POINTER(LhConfig)
+_PCFG = POINTER(LhPisaConfig)
 # name -> argument types (all return lh_status unless listed in _RESTYPES)
 SIGNATURES = {
     "lh_plan": [_CFG, POINTER(LhPlanInfo)],
@@ -62,6 +74,9 @@ SIGNATURES = {
     "lh_pool_adjoint": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_forward": [_CFG, _P, _P, _P, _P, _P, c_size_t, _P, c_size_t, _P],
     "lh_backward": [_CFG, _P, _P, c_size_t, _P, _P, _P, _P, c_size_t, _P],
+    "lh_pisa_plan": [_PCFG, POINTER(LhPisaInfo)],
+    "lh_pisa_pool_keys": [_PCFG, _P, _P, _P],
+    "lh_pisa_select": [_PCFG, _P, _P, _P, _P, _P, _P, _P],
     "lh_check_error": [_P, _P],
     "lh_clear_error": [_P, _P],
     "lh_status_string": [c_int],

@@ -23,6 +23,11 @@ Workloads (names give what they are):
   outlier_1m          B=1 H=8  N=1048576 d=128 L=6 p=4 k=1536 bf16 iid, 1% of the
                       positions (uniform, shared by all heads) have Q, K, V rows x4
 dY is iid N(0,1) in the input dtype for every workload.
+
+PISA block selection workloads (PISA_WORKLOADS) take Q and K from the same
+generators: pisa_small_8k (H=2, N=8192), pisa_128k and pisa_256k (H=16),
+all d=128, p=4, blocks of 64, groups of 128, K=8, L = 3, 4, 5, LogNormal(0,0.5)
+per token.
 """
 
 from __future__ import annotations
@@ -67,6 +72,47 @@ WORKLOADS = {
         Workload("kscore_128k", 1, 16, 131072, 128, 3, 2, 1536, "bf16", "k", "iid", 2),
         Workload("sparse64_512k", 1, 16, 524288, 128, 5, 4, 384, "bf16", "qk_sum", "iid", 3),
         Workload("outlier_1m", 1, 8, 1048576, 128, 6, 4, 1536, "bf16", "qk_sum", "outlier_tokens", 4),
+    )
+}
+
+
+@dataclass(frozen=True)
+class PisaWorkload:
+    """PISA block selection inputs: q, k [B, H, N, d] bf16 drawn by the same
+    generators as the Lighthouse workloads (head_inputs / cuda_inputs)."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    p: int
+    L: int
+    block: int
+    group: int
+    topk: int
+    structure: str
+    seed: int
+    dtype: str = "bf16"
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16
+
+    def with_(self, **kw) -> "PisaWorkload":
+        return replace(self, **kw)
+
+
+# The review of PISA times block selection at 64K, 128K and 256K tokens
+# (section 3, Figure 3) without model sizes; these take d = 128, blocks of 64,
+# groups of 128 queries, K = 8 kept blocks per level and p = 4, with L chosen
+# so the coarsest level has no more blocks than a finer level scores (p K = 32).
+# Per-token LogNormal(0, 0.5) scales on the rows give the block scores spread.
+PISA_WORKLOADS = {
+    w.name: w
+    for w in (
+        PisaWorkload("pisa_small_8k", 1, 2, 8192, 128, 4, 3, 64, 128, 8, "lognormal_token", 20),
+        PisaWorkload("pisa_128k", 1, 16, 131072, 128, 4, 4, 64, 128, 8, "lognormal_token", 21),
+        PisaWorkload("pisa_256k", 1, 16, 262144, 128, 4, 5, 64, 128, 8, "lognormal_token", 22),
     )
 }
 

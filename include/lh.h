@@ -266,6 +266,71 @@ lh_status lh_forward(const lh_config *cfg, const void *q, const void *k, const v
 lh_status lh_backward(const lh_config *cfg, const void *dy, const void *ctx, size_t ctx_bytes, void *dq,
                       void *dk, void *dv, void *ws, size_t ws_bytes, lh_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * PISA block selection (a second workload on the same pyramid idea).
+ * Cite: the blog.secrett2633.cloud review "[논문리뷰] Block Sparse Attention
+ * with Log-Linear Complexity" (PISA-review), section 1 (block sparse
+ * attention selects key blocks per query; LSE scores the candidate blocks)
+ * and section 3 (keys pooled fine-to-coarse; selection starts at the
+ * coarsest level, keeps the top K by LSE and expands them into sub-blocks
+ * level by level down to the finest; O(N log N)).
+ *
+ * Readings of what the page leaves open:
+ *  - level l entry j is the mean of keys [j p^l, (j+1) p^l) (level 0 = the
+ *    keys), stored in bf16 rounded to nearest even from the exact mean;
+ *  - a block is `block` (C) consecutive entries of one level; block b of
+ *    level l has sub-blocks p b .. p b + p - 1 at level l-1;
+ *  - `group` (G) consecutive queries share one selection;
+ *  - the score of block b of level l for group g is
+ *      ln sum_{i in g} sum_{j in b, (j+1) p^l - 1 <= i} exp(q_i . k^(l)_j / sqrt(d)),
+ *    -inf when no pair is visible;
+ *  - the coarsest level's candidates are all its blocks; a level keeps
+ *    min(topk, candidates) blocks, higher score first, equal scores (-inf
+ *    included) to the lower block index.
+ * Support: bf16 Q and K [B][H][N][d]; d in {64, 128}; block in {64, 128};
+ * group = 128; p a power of two >= 2; 1 <= L <= 8; N divisible by
+ * block * p^(L-1) and < 2^28; blocks[L-1] <= 512 and p * topk <= 512;
+ * B*H <= 65535.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int64_t B, H, N; /* batch, heads, sequence length */
+  int32_t d;       /* head dimension */
+  int32_t p;       /* pooling factor between levels */
+  int32_t L;       /* levels of the key pyramid (level 0 = the keys) */
+  int32_t block;   /* C: entries per block, every level */
+  int32_t group;   /* G: queries per selection */
+  int32_t topk;    /* K: blocks kept per level */
+} lh_pisa_config;
+
+typedef struct {
+  int64_t n_groups;                   /* N / group */
+  int64_t blocks[LH_MAX_LEVELS];      /* N / (block p^l) */
+  int64_t level_off[LH_MAX_LEVELS];   /* first row of level l >= 1 in the key pyramid */
+  int64_t upper_entries;              /* sum over l >= 1 of N / p^l */
+  size_t pyr_bytes;                   /* key pyramid [BH][upper_entries][d] bf16 */
+  size_t kept_elems;                  /* BH * n_groups * L * topk */
+  int32_t max_candidates;             /* most candidates one level scores */
+} lh_pisa_info;
+
+/* Validate cfg and fill *info (host only, no CUDA call). */
+lh_status lh_pisa_plan(const lh_pisa_config *cfg, lh_pisa_info *info);
+
+/* The key pyramid.  In: k [BH][N][d] bf16.  Out: kpyr [BH][upper_entries][d]
+ * bf16, level l >= 1 from row level_off[l]; each entry is summed exactly (fp64)
+ * from the level-0 keys and rounded once.  L = 1: nothing is written (kpyr
+ * may be NULL). */
+lh_status lh_pisa_pool_keys(const lh_pisa_config *cfg, const void *k, void *kpyr, lh_stream_t stream);
+
+/* The coarse-to-fine selection.  In: q, k [BH][N][d] bf16; kpyr from
+ * lh_pisa_pool_keys (unused when L = 1); ws: at least LH_ERR_WORD_BYTES (the
+ * error word; a bounded wait that runs out sets it).
+ * Out: kept_idx [BH][n_groups][L][topk] int32 and kept_score (same shape,
+ * fp32, natural log): for every group and level the kept blocks in
+ * ascending block order with their scores, padded with -1 / -inf when a
+ * level has fewer than topk candidates.  Level 0 is the selection. */
+lh_status lh_pisa_select(const lh_pisa_config *cfg, const void *q, const void *k, const void *kpyr,
+                         int32_t *kept_idx, float *kept_score, void *ws, lh_stream_t stream);
+
 /* Synchronise `stream`, read the error word at the start of ws, clear it and
  * return LH_OK, LH_ERR_TIMEOUT or LH_ERR_DEVICE (or LH_ERR_CUDA). */
 lh_status lh_check_error(void *ws, lh_stream_t stream);

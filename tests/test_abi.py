@@ -124,3 +124,54 @@ def test_status_strings(lib):
     for s in range(7):
         assert lib.lh_status_string(s).decode()
     assert lib.lh_status_string(99).decode() == "unknown status"
+
+
+# ---------------------------------------------------------------- PISA selection
+
+def _pisa_cfg(**kw):
+    base = dict(B=1, H=2, N=8192, d=128, p=4, L=3, block=64, group=128, topk=8)
+    base.update(kw)
+    return _lib.LhPisaConfig(**base)
+
+
+@pytest.mark.parametrize("name", ["pisa_small_8k", "pisa_128k", "pisa_256k"])
+def test_pisa_plan_matches_oracle_sizes(lib, name):
+    from hierarchical_sparse_attention_pyramid_b200.synth import PISA_WORKLOADS
+    from oracle import pisa_oracle as po
+    w = PISA_WORKLOADS[name]
+    info = _lib.LhPisaInfo()
+    cfg = _pisa_cfg(B=w.B, H=w.H, N=w.N, d=w.d, p=w.p, L=w.L, block=w.block, group=w.group, topk=w.topk)
+    assert lib.lh_pisa_plan(ctypes.byref(cfg), ctypes.byref(info)) == 0
+    assert list(info.blocks)[: w.L] == po.level_blocks(w.N, w.p, w.L, w.block)
+    assert info.n_groups == w.N // w.group
+    assert info.upper_entries == sum(w.N // w.p ** l for l in range(1, w.L))
+    assert info.pyr_bytes == w.B * w.H * info.upper_entries * w.d * 2
+    assert info.kept_elems == w.B * w.H * info.n_groups * w.L * w.topk
+    assert info.max_candidates == max(po.level_blocks(w.N, w.p, w.L, w.block)[-1], w.p * w.topk)
+    off = 0
+    for lv in range(1, w.L):
+        assert info.level_off[lv] == off
+        off += w.N // w.p ** lv
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(block=32), 2), (dict(group=64), 2), (dict(p=3), 2), (dict(L=9), 2),
+    (dict(N=8192 + 128), 2),            # not a whole number of coarsest blocks
+    (dict(N=65536, L=1), 2),            # 1024 coarsest blocks > 512
+    (dict(topk=200), 2),                # p * topk > 512
+    (dict(topk=0), 1), (dict(N=0), 1), (dict(B=0), 1),
+])
+def test_pisa_plan_rejects(lib, kw, status):
+    info = _lib.LhPisaInfo()
+    assert lib.lh_pisa_plan(ctypes.byref(_pisa_cfg(**kw)), ctypes.byref(info)) == status
+    assert lib.lh_last_error_message().decode().startswith("lh_pisa_plan")
+
+
+def test_pisa_calls_reject_bad_pointers_before_any_launch(lib):
+    cfg = _pisa_cfg()
+    buf = ctypes.create_string_buffer(64)
+    odd = ctypes.c_void_p(ctypes.addressof(buf) + 1)
+    assert lib.lh_pisa_pool_keys(ctypes.byref(cfg), None, None, None) == 1
+    assert lib.lh_pisa_pool_keys(ctypes.byref(cfg), odd, odd, None) == 1
+    assert lib.lh_pisa_select(ctypes.byref(cfg), None, None, None, None, None, None, None) == 1
+    assert lib.lh_pisa_plan(None, None) == 1
