@@ -11,6 +11,10 @@ one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the layer) on the host cores, one head per step, on rank 0 only.
+
+--workload pisa_128k (or pisa_small_8k, pisa_256k) times the second workload
+instead: one step = lh_pisa_pool_keys + lh_pisa_select over all heads (PISA
+block selection), same timing rules, its own metric.
 """
 
 from __future__ import annotations
@@ -31,7 +35,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from hierarchical_sparse_attention_pyramid_b200 import _lib, synth  # noqa: E402
+from hierarchical_sparse_attention_pyramid_b200 import _lib, pisa, synth  # noqa: E402
 from hierarchical_sparse_attention_pyramid_b200 import api as lh  # noqa: E402
 
 METRIC = "Lighthouse attn fwd+bwd tokens/s/layer at N=512K on 1 B200; % of roofline"
@@ -315,6 +319,217 @@ def workload_config(w: synth.Workload) -> dict:
             "l2": "inputs larger than L2 (Q,K,V,dY %.1f GB per GPU)" % (4 * w.B * w.H * w.N * w.d * 2 / 1e9)}
 
 
+# ------------------------------------------------------------------ PISA block selection
+
+PISA_METRIC = "PISA block selection tokens/s (key pyramid + coarse-to-fine LSE top-K, all heads) on 1 B200"
+# ex2 results per clock per SM: 4 per SM sub-partition (the special-function
+# unit rate of sm_100), 4 sub-partitions
+MUFU_EX2_PER_CLK_SM = 16
+SMS = 148
+
+
+def pisa_of(w) -> pisa.Pisa:
+    return pisa.Pisa(w.B, w.H, w.N, w.d, w.p, w.L, w.block, w.group, w.topk)
+
+
+def pisa_config(w) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L, "block": w.block,
+            "group": w.group, "topk": w.topk, "structure": w.structure,
+            "parallelism": "replicas (one selection per GPU)",
+            "l2": ("inputs larger than L2" if 2 * w.B * w.H * w.N * w.d * 2 > 126e6 else "inputs smaller than L2")
+                  + " (Q, K %.2f GB per GPU); key blocks are re-read from L2 by design" % (2 * w.B * w.H * w.N * w.d * 2 / 1e9)}
+
+
+def pisa_scored_candidates(w, idx) -> int:
+    """Candidate blocks the selection kernel scores (loads and multiplies):
+    every visible block of the coarsest level, then every visible sub-block of
+    the blocks kept one level up, summed over groups, levels and heads."""
+    G, C, p, L = w.group, w.block, w.p, w.L
+    n_groups = w.N // G
+    last = (torch.arange(n_groups, device=idx.device, dtype=torch.int64) + 1) * G - 1   # [n_groups]
+    n_top = w.N // (C * p ** (L - 1))
+    b = torch.arange(n_top, device=idx.device, dtype=torch.int64)
+    total = int((((b[None, :] * C + 1) * p ** (L - 1) - 1) <= last[:, None]).sum()) * w.B * w.H
+    for lv in range(L - 2, -1, -1):
+        kept = idx[:, :, lv + 1, :].long()                                   # [BH, n_groups, K]
+        sub = kept[..., None] * p + torch.arange(p, device=idx.device)      # [BH, n_groups, K, p]
+        vis = (kept[..., None] >= 0) & (((sub * C + 1) * p ** lv - 1) <= last[None, :, None, None])
+        total += int(vis.sum())
+    return total
+
+
+def pisa_oracle_sample(w, max_seconds: float = 20.0) -> dict:
+    """fp64 oracle on a bounded sample: head 0's key pyramid plus as many of
+    its groups (spread over the sequence) as fit in max_seconds; returns
+    seconds per group (the pyramid's time spread over the head's groups)."""
+    from oracle import pisa_oracle as po
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    h = synth.head_inputs(w, 0)
+    Q, K = h["q"].double().numpy(), h["k"].double().numpy()
+    n_groups = w.N // w.group
+    t0 = time.perf_counter()
+    levels = po.key_pyramid(K, w.p, w.L)
+    t_pyr = time.perf_counter() - t0
+    order = np.random.default_rng(0).permutation(n_groups)
+    t_sel, done = 0.0, 0
+    for g in order:
+        t0 = time.perf_counter()
+        po.select_group(Q, levels, int(g), w.group, w.block, w.p, w.L, w.topk)
+        t_sel += time.perf_counter() - t0
+        done += 1
+        if t_pyr + t_sel > max_seconds:
+            break
+    per_group = t_sel / done + t_pyr / n_groups
+    return {"sec_per_group": per_group, "groups": done, "cores": cores,
+            "sample": f"head 0: key pyramid + {done} of {n_groups} groups (random order), fp64, scaled to "
+                      f"{w.B * w.H} heads x {n_groups} groups"}
+
+
+def run_pisa_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = synth.PISA_WORKLOADS[args.workload]
+    total_groups = w.B * w.H * (w.N // w.group)
+    budget = max(5.0, 150.0 / max(1, args.steps + min(args.warmup, 1)))
+    secs, cores, sample = [], None, ""
+    for _ in range(min(args.warmup, 1)):
+        pisa_oracle_sample(w, 2.0)
+    for _ in range(args.steps):
+        r = pisa_oracle_sample(w, budget)
+        secs.append(r["sec_per_group"] * total_groups)
+        cores, sample = r["cores"], r["sample"]
+    sec = float(np.mean(secs))
+    value = w.B * w.N / sec
+    print(json.dumps({
+        "impl": "reference", "metric": PISA_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": pisa_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def run_pisa(args, world, rank, local):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.PISA_WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
+    sel = pisa_of(w)
+    info = pisa.plan(sel)
+    x = synth.cuda_inputs(w, dev, seed=w.seed + 16 * rank)
+    q, k = x["q"], x["k"]
+    del x
+    kpyr = torch.empty((sel.BH, max(info.upper_entries, 1), w.d), dtype=torch.bfloat16, device=dev)
+    shp = (sel.BH, info.n_groups, w.L, w.topk)
+    out = (torch.empty(shp, dtype=torch.int32, device=dev), torch.empty(shp, dtype=torch.float32, device=dev))
+    ws = torch.zeros(_lib.ERR_WORD_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        pisa.pool_keys(sel, k, kpyr)
+        pisa.select(sel, q, k, kpyr, out, ws)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    barrier(world)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    value = world * w.B * w.N / (ms / 1e3)
+
+    # each kernel alone (same buffers), CUDA events on the launching stream
+    stage_ms = time_stages([("pool_keys", lambda: pisa.pool_keys(sel, k, kpyr)),
+                            ("select", lambda: pisa.select(sel, q, k, kpyr, out, ws))], max(3, min(args.steps, 10)))
+    pk, pk_src = peaks()
+    scored = pisa_scored_candidates(w, out[0])
+    exps = scored * w.group * w.block
+    sm_mhz = pk.get("sm_max_mhz", 1965.0)
+    mufu_peak = SMS * MUFU_EX2_PER_CLK_SM * sm_mhz * 1e6 / 1e12   # T ex2 / s
+    t_sel = stage_ms["select"] / 1e3
+    mma_flops = 2.0 * exps * w.d
+    roofline = {"bound": "alu", "kernel": "select", "kernels": ["pisa_select_kernel"],
+                "achieved": exps / t_sel / 1e12, "peak": mufu_peak, "unit": "T ex2/s",
+                "frac": exps / t_sel / 1e12 / mufu_peak, "traffic": None, "peak_source":
+                f"derived: {SMS} SMs x {MUFU_EX2_PER_CLK_SM} ex2/clk x {sm_mhz:.0f} MHz",
+                "scored_blocks": scored, "exp_per_block": w.group * w.block,
+                "tensor": {"achieved_tflops": mma_flops / t_sel / 1e12, "peak": pk["bf16_tflops"],
+                           "frac": mma_flops / t_sel / 1e12 / pk["bf16_tflops"]},
+                "share_of_step": stage_ms["select"] / sum(stage_ms.values())}
+    pool_bytes = sel.BH * w.N * w.d * 2 + sel.BH * info.upper_entries * w.d * 2
+    stages = {"pool_keys": {"ms": stage_ms["pool_keys"], "bound": "hbm",
+                            "achieved": pool_bytes / (stage_ms["pool_keys"] / 1e3) / 1e9, "unit": "GB/s",
+                            "frac": pool_bytes / (stage_ms["pool_keys"] / 1e3) / 1e9 / pk["hbm_gbs"]},
+              "select": {"ms": stage_ms["select"], "bound": "alu", "frac": roofline["frac"]}}
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk = q.cpu().pin_memory(), k.cpu().pin_memory()
+        hi = torch.empty(shp, dtype=torch.int32).pin_memory()
+        hs = torch.empty(shp, dtype=torch.float32).pin_memory()
+        dq, dk = torch.empty_like(q), torch.empty_like(k)
+        h2d = 2 * q.numel() * 2
+        d2h = hi.numel() * 4 + hs.numel() * 4
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            pisa.pool_keys(sel, dk, kpyr)
+            pisa.select(sel, dq, dk, kpyr, out, ws)
+            hi.copy_(out[0], non_blocking=True)
+            hs.copy_(out[1], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        k_e = max(2, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(k_e):
+            e2e_step()
+        b.record(st)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e = max_over_ranks(a.elapsed_time(b) / k_e, world, dev)
+        e2e = {"value": world * w.B * w.N / (ms_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ms_e, "steps": k_e}
+
+    cpu = None
+    if not args.no_cpu and rank == 0 and world == 1:
+        r = pisa_oracle_sample(w, 20.0)
+        sec = r["sec_per_group"] * sel.BH * info.n_groups
+        cpu = {"value": w.B * w.N / sec, "unit": UNIT, "cores": r["cores"], "kind": "oracle", "sample": r["sample"]}
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": PISA_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": pisa_config(w), "clocks": clocks,
+            "e2e": e2e, "gpu_launches": 2 * args.steps, "roofline": roofline, "stages": stages,
+            "cpu_baseline": cpu}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -322,7 +537,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="sparse64_512k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="sparse64_512k", choices=sorted(synth.WORKLOADS) + sorted(synth.PISA_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -334,6 +549,12 @@ def main():
     args = ap.parse_args()
 
     world, rank, local = dist_setup()
+    if args.workload in synth.PISA_WORKLOADS:
+        if args.impl == "reference":
+            run_pisa_reference(args, world, rank)
+        else:
+            run_pisa(args, world, rank, local)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

@@ -12,13 +12,16 @@
 //
 // pisa_select_kernel - one CTA per (query group of 128 rows, head).  The group
 //   makes one selection.  Warp roles:
-//     warp 0      TMA producer: the group's Q tile once, then the key block of
-//                 every candidate into a 4-stage ring
-//     warp 1      MMA issuer: S = Q K_b^T (128 x C, fp32) per candidate into
-//                 one of 256/C TMEM buffers
-//     warps 2-5   scorers, thread = query row: the row's masked max and sum
-//                 of 2^(s - max) over the block, reduced over the warp's 32
-//                 rows into one log2 partial per candidate; at the end of a
+//     warp 0      TMA producer: the group's Q tile once, then the visible
+//                 candidates' key blocks, 128 key rows (one unit: two blocks
+//                 of 64 or one of 128) per stage of a 2-stage ring
+//     warp 1      MMA issuer: S = Q K_unit^T (128 x 128, fp32) per unit into
+//                 one of two TMEM buffers
+//     warps 2-9   scorers, thread = (query row, column half): the row's
+//                 max and sum of 2^(s - max) over its half of the block
+//                 (masked only where the warp sees a causal edge), reduced
+//                 over the warp's 32 rows into one log2 partial per
+//                 candidate; at the end of a
 //                 level they combine the four partials into each candidate's
 //                 score, rank the candidates, write the kept blocks and build
 //                 the next level's candidate list (the kept blocks' p
@@ -29,6 +32,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
+
+#include <type_traits>
 
 #include "lh_common.cuh"
 #include "sm100.cuh"
@@ -41,8 +46,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kG = 128;          // queries per group: the MMA's M
-constexpr int kMaxCand = 512;    // candidates of one level held in shared memory
-constexpr int kThreads = 192;    // producer, MMA issuer, 4 scorer warps
+constexpr int kMaxCand = 256;    // candidates of one level held in shared memory
+constexpr int kScorers = 256;    // 8 scorer warps
+constexpr int kThreads = 64 + kScorers;  // producer, MMA issuer, scorers
 constexpr int kMaxLevels = 8;
 
 struct PisaArgs {
@@ -54,24 +60,34 @@ struct PisaArgs {
   int* errw;
 };
 
+// A "unit" is 128 key rows: two blocks of 64 (scored by one MMA of N = 128)
+// or one block of 128.
 template <int D, int C>
 struct PisaSmem {
-  static constexpr int NST = C == 64 ? 4 : 2;  // key stages
-  static constexpr int NBUF = 256 / C;         // TMEM score buffers (256 columns)
+  static constexpr int BPU = 128 / C;          // blocks per unit
+  static constexpr int NST = 2;                // key stages, one unit each
+  static constexpr int NBUF = 2;               // TMEM score buffers, 128 columns each
   static constexpr int kQChunk = kG * 128;     // [128 rows][64 bf16]
-  static constexpr int kKChunk = C * 128;      // [C rows][64 bf16]
+  static constexpr int kKChunk = 128 * 128;    // [128 key rows][64 bf16]
   static constexpr int kQ = D / 64 * kQChunk;
   static constexpr int kKStage = D / 64 * kKChunk;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
   static constexpr int oCand = oK + NST * kKStage;          // int [2][kMaxCand]
   static constexpr int oScore = oCand + 2 * kMaxCand * 4;   // float [kMaxCand]
-  static constexpr int oPart = oScore + kMaxCand * 4;       // float [4][kMaxCand], then int flags [kMaxCand]
-  static constexpr int oMisc = oPart + 4 * kMaxCand * 4;    // int counts [2], tmem slot, abort flag
+  static constexpr int oPart = oScore + kMaxCand * 4;       // float [8][kMaxCand], then int flags [kMaxCand]
+  static constexpr int oMisc = oPart + 8 * kMaxCand * 4;    // int counts [2], tmem slot, abort flag
   static constexpr int oBar = oMisc + 64;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
+
+// maximum over the warp (redux.sync on sm_100a)
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 
 // is block b of level l seen by any query of the group?  (its first entry's
 // last averaged token (bC+1) p^l - 1 is at or before the group's last query)
@@ -84,16 +100,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     pisa_select_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK0,
                        const __grid_constant__ CUtensorMap tmKU, const PisaArgs a) {
   using Lay = PisaSmem<D, C>;
-  constexpr int NST = Lay::NST, NBUF = Lay::NBUF;
+  constexpr int NST = Lay::NST, NBUF = Lay::NBUF, BPU = Lay::BPU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bQ = bars + 0;
-  uint64_t* bLevel = bars + 1;             // a level's candidate list is ready (128 arrivals)
+  uint64_t* bLevel = bars + 1;             // a level's candidate list is ready (one arrival per scorer)
   uint64_t* bK = bars + 2;                 // [NST] key block landed
   uint64_t* bKfree = bars + 2 + NST;       // [NST] its MMA is done
   uint64_t* bS = bars + 2 + 2 * NST;       // [NBUF] scores in TMEM
-  uint64_t* bSfree = bars + 2 + 2 * NST + NBUF;  // [NBUF] scores read (128 arrivals)
+  uint64_t* bSfree = bars + 2 + 2 * NST + NBUF;  // [NBUF] scores read (one arrival per scorer)
   int32_t* cand = reinterpret_cast<int32_t*>(smem + Lay::oCand);
   float* score = reinterpret_cast<float*>(smem + Lay::oScore);
   float* part = reinterpret_cast<float*>(smem + Lay::oPart);
@@ -110,14 +126,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(bQ, 1);
-    mbar_init(bLevel, 128);
+    mbar_init(bLevel, kScorers);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bK[s], 1);
       mbar_init(&bKfree[s], 1);
     }
     for (int s = 0; s < NBUF; ++s) {
       mbar_init(&bS[s], 1);
-      mbar_init(&bSfree[s], 128);
+      mbar_init(&bSfree[s], kScorers);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -137,29 +153,34 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_expect_tx(bQ, kG * D * 2);
       for (int ch = 0; ch < D / 64; ++ch)
         tma_load_3d(smem + Lay::oQ + ch * Lay::kQChunk, &tmQ, bQ, ch * 64, first_query, bh);
-      uint32_t u = 0;
+      uint32_t u = 0;  // units loaded so far
       bool ok = true;
       for (int li = 0; ok && li < L; ++li) {
         const int l = L - 1 - li, buf = li & 1;
         if (!mbar_wait(bLevel, li & 1, abort_flag)) break;
         const int n = count[buf];
-        for (int c = 0; c < n; ++c) {
-          const int b = cand[buf * kMaxCand + c];
-          if (!block_visible(b, l, log2p, C, last_query)) continue;
+        const int* cl = cand + buf * kMaxCand;
+        int nv = 0;  // visible candidates: a prefix of the ascending list
+        while (nv < n && block_visible(cl[nv], l, log2p, C, last_query)) ++nv;
+        const CUtensorMap* map = l == 0 ? &tmK0 : &tmKU;
+        const int row0 = l == 0 ? 0 : a.level_off[l];
+        for (int c = 0; c < nv; c += BPU) {
+          const int nb = nv - c < BPU ? nv - c : BPU;
           const int st = (int)(u % NST);
           if (u >= (uint32_t)NST && !mbar_wait(&bKfree[st], ((u / NST) - 1) & 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&bK[st], C * D * 2);
-          const CUtensorMap* map = l == 0 ? &tmK0 : &tmKU;
-          const int row = (l == 0 ? 0 : a.level_off[l]) + b * C;
-          for (int ch = 0; ch < D / 64; ++ch)
-            tma_load_3d(smem + Lay::oK + st * Lay::kKStage + ch * Lay::kKChunk, map, &bK[st], ch * 64, row, bh);
+          mbar_expect_tx(&bK[st], nb * C * D * 2);
+          for (int j = 0; j < nb; ++j)
+            for (int ch = 0; ch < D / 64; ++ch)
+              tma_load_3d(smem + Lay::oK + st * Lay::kKStage + ch * Lay::kKChunk + j * C * 128, map, &bK[st],
+                          ch * 64, row0 + cl[c + j] * C, bh);
           ++u;
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idS = idesc_bf16(kG, C, false, false);
+    constexpr uint32_t idFull = idesc_bf16(kG, 128, false, false);
+    constexpr uint32_t idHalf = idesc_bf16(kG, C, false, false);  // a unit holding one block of 64
     const uint64_t dQ = sdesc_sw128(smem_u32(smem + Lay::oQ), 16, 1024);
     const uint64_t dK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
     bool ok = mbar_wait_warp(bQ, 0, abort_flag);
@@ -168,9 +189,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int l = L - 1 - li, buf = li & 1;
       if (!mbar_wait_warp(bLevel, li & 1, abort_flag)) break;
       const int n = count[buf];
-      for (int c = 0; c < n; ++c) {
-        const int b = cand[buf * kMaxCand + c];
-        if (!block_visible(b, l, log2p, C, last_query)) continue;
+      const int* cl = cand + buf * kMaxCand;
+      int nv = 0;
+      while (nv < n && block_visible(cl[nv], l, log2p, C, last_query)) ++nv;
+      for (int c = 0; c < nv; c += BPU) {
+        const uint32_t id = nv - c >= BPU ? idFull : idHalf;
         const int st = (int)(u % NST), sb = (int)(u % NBUF);
         if (!mbar_wait_warp(&bK[st], (u / NST) & 1, abort_flag)) { ok = false; break; }
         if (u >= (uint32_t)NBUF && !mbar_wait_warp(&bSfree[sb], ((u / NBUF) - 1) & 1, abort_flag)) {
@@ -183,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = ((kk >> 2) * Lay::kQChunk + (kk & 3) * 32) >> 4;
           const uint32_t ok_ = ((kk >> 2) * Lay::kKChunk + (kk & 3) * 32) >> 4;
-          umma_bf16_w(tmem + sb * C, dQ + oq, kb + ok_, idS, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + sb * 128, dQ + oq, kb + ok_, id, kk > 0 ? 1u : 0u);
         }
         umma_commit_w(&bKfree[st]);
         umma_commit_w(&bS[sb]);
@@ -192,18 +215,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else {
     // ------------------------------------------------------------ scorers
-    const int t = threadIdx.x - 64;              // 0..127
+    // Thread (h, row): query row `row` of the group (TMEM lane row) and
+    // columns [h C/2, h C/2 + C/2) of each candidate's score tile.  Each warp
+    // reduces its 32 rows into one log2-sum-exp2 partial per candidate; the
+    // eight partials are combined at the end of the level.
+    const int t = threadIdx.x - 64;              // 0..255
     const int q = warp & 3;                      // TMEM lane quarter of this warp
+    const int h = (warp - 2) >> 2;               // column half
+    const int wp = h * 4 + q;                    // partial slot of this warp
     const int row = q * 32 + lane;               // query row of the group
     const int i = first_query + row;
-    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    constexpr int HC = C / 2;                    // columns per thread
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + h * HC;
     const float ln2 = 0.69314718055994530942f;
+    const float sl2 = a.scale_log2;
     const int64_t out0 = ((int64_t)bh * a.n_groups + g) * L * a.K;
-    auto sync_scorers = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+    auto sync_scorers = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
 
     // the coarsest level's candidates: all its blocks
     const int n_top = (a.N >> ((L - 1) * log2p)) / C;
-    for (int c = t; c < n_top; c += 128) cand[c] = c;
+    for (int c = t; c < n_top; c += kScorers) cand[c] = c;
     if (t == 0) count[0] = n_top;
     sync_scorers();
     mbar_arrive(bLevel);
@@ -214,72 +245,139 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int l = L - 1 - li, buf = li & 1;
       const int n = count[buf];
       const int* cl = cand + buf * kMaxCand;
-      for (int c = 0; ok && c < n; ++c) {
-        const int b = cl[c];
-        if (!block_visible(b, l, log2p, C, last_query)) {
-          if (lane == 0) part[q * kMaxCand + c] = -INFINITY;
-          continue;
-        }
+      // the list is ascending and visibility falls with the block index, so
+      // the visible candidates are a prefix of it
+      int nv = 0;
+      while (nv < n && block_visible(cl[nv], l, log2p, C, last_query)) ++nv;
+      if (lane == 0)
+        for (int c = nv; c < n; ++c) part[wp * kMaxCand + c] = -INFINITY;
+      const int lbase = ((i + 1) >> (l * log2p)) - 1 - h * HC;
+      // one unit at a time: both blocks of a unit of two are scored
+      // together, so their exponentials and warp reductions interleave
+      auto score_blocks = [&](auto nb_tag, int c0) {
+        constexpr int NB = decltype(nb_tag)::value;  // blocks of this unit
+        uint32_t r[NB][HC / 32][32];
         const int sb = (int)(u % NBUF);
         ok = __all_sync(0xffffffffu, mbar_wait(&bS[sb], (u / NBUF) & 1, abort_flag));
-        if (!ok) break;
+        if (!ok) return;
         tc_fence_after();
-        uint32_t r[C / 32][32];
 #pragma unroll
-        for (int h = 0; h < C / 32; ++h) tmem_ld32(tl + sb * C + h * 32, r[h]);
+        for (int j = 0; j < NB; ++j)
+#pragma unroll
+          for (int x = 0; x < HC / 32; ++x) tmem_ld32(tl + sb * 128 + j * C + x * 32, r[j][x]);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&bSfree[sb]);
         ++u;
-        // last column this row sees: entry j = bC + col is visible while
-        // (j+1) p^l - 1 <= i
-        const int lim = ((i + 1) >> (l * log2p)) - 1 - b * C;
-        float mx = -INFINITY;
+        // last column of this thread's half the row sees, per candidate:
+        // entry j = bC + col is visible while (j+1) p^l - 1 <= i
+        int lim[NB];
+        bool all_vis = true;
 #pragma unroll
-        for (int h = 0; h < C / 32; ++h)
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (h * 32 + x <= lim) mx = fmaxf(mx, __uint_as_float(r[h][x]));
-        float m_row = -INFINITY, s_row = 0.f;
-        if (mx != -INFINITY) {
-          m_row = mx * a.scale_log2;
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int h = 0; h < C / 32; ++h)
-#pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float e0 = fast_exp2(fmaf(__uint_as_float(r[h][x]), a.scale_log2, -m_row));
-              const float e1 = fast_exp2(fmaf(__uint_as_float(r[h][x + 1]), a.scale_log2, -m_row));
-              s0 += h * 32 + x <= lim ? e0 : 0.f;
-              s1 += h * 32 + x + 1 <= lim ? e1 : 0.f;
-            }
-          s_row = s0 + s1;
+        for (int j = 0; j < NB; ++j) {
+          lim[j] = lbase - cl[c0 + j] * C;
+          all_vis = all_vis && lim[j] >= HC - 1;
         }
-        // the warp's 32 rows: one log2-sum-exp2 partial
-        float M = m_row;
+        float m_row[NB], s_row[NB];
+        if (__all_sync(0xffffffffu, all_vis)) {
+          // every column visible to every row of the warp: no masks
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float S = M == -INFINITY || m_row == -INFINITY ? 0.f : s_row * fast_exp2(m_row - M);
+          for (int j = 0; j < NB; ++j) {
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-        if (lane == 0) part[q * kMaxCand + c] = S > 0.f ? M + __log2f(S) : -INFINITY;
-      }
+            for (int x = 0; x < HC / 32; ++x)
+#pragma unroll
+              for (int y = 0; y < 32; y += 8)
+#pragma unroll
+                for (int z = 0; z < 4; ++z)
+                  mx[z] = max3f(mx[z], __uint_as_float(r[j][x][y + 2 * z]), __uint_as_float(r[j][x][y + 2 * z + 1]));
+            m_row[j] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+          }
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            const uint64_t c2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_row[j], -m_row[j]);
+            uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int x = 0; x < HC / 32; ++x)
+#pragma unroll
+              for (int y = 0; y < 32; y += 4) {
+                float e0, e1, e2, e3;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(r[j][x][y]), __uint_as_float(r[j][x][y + 1])), c2, nm2), e0, e1);
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(r[j][x][y + 2]), __uint_as_float(r[j][x][y + 3])), c2, nm2), e2,
+                          e3);
+                acc0 = f2_add(acc0, f2_pack(fast_exp2(e0), fast_exp2(e1)));
+                acc1 = f2_add(acc1, f2_pack(fast_exp2(e2), fast_exp2(e3)));
+              }
+            float s0, s1;
+            f2_unpack(f2_add(acc0, acc1), s0, s1);
+            s_row[j] = s0 + s1;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int x = 0; x < HC / 32; ++x)
+#pragma unroll
+              for (int y = 0; y < 32; ++y)
+                if (x * 32 + y <= lim[j]) mx = fmaxf(mx, __uint_as_float(r[j][x][y]));
+            m_row[j] = -INFINITY;
+            s_row[j] = 0.f;
+            if (mx != -INFINITY) {
+              m_row[j] = mx * sl2;
+              float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+              for (int x = 0; x < HC / 32; ++x)
+#pragma unroll
+                for (int y = 0; y < 32; y += 2) {
+                  const float e0 = fast_exp2(fmaf(__uint_as_float(r[j][x][y]), sl2, -m_row[j]));
+                  const float e1 = fast_exp2(fmaf(__uint_as_float(r[j][x][y + 1]), sl2, -m_row[j]));
+                  s0 += x * 32 + y <= lim[j] ? e0 : 0.f;
+                  s1 += x * 32 + y + 1 <= lim[j] ? e1 : 0.f;
+                }
+              s_row[j] = s0 + s1;
+            }
+          }
+        }
+        // the warp's 32 rows: one log2-sum-exp2 partial per candidate
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          const float M = warp_max_f32(m_row[j]);
+          float S = M == -INFINITY || m_row[j] == -INFINITY ? 0.f : s_row[j] * fast_exp2(m_row[j] - M);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+          if (lane == 0) part[wp * kMaxCand + c0 + j] = S > 0.f ? M + __log2f(S) : -INFINITY;
+        }
+      };
+      int c = 0;
+      if constexpr (Lay::BPU == 2)
+        for (; ok && c + 1 < nv; c += 2) score_blocks(std::integral_constant<int, 2>{}, c);
+      for (; ok && c < nv; ++c) score_blocks(std::integral_constant<int, 1>{}, c);
       // level end: scores, ranks, kept blocks, next candidates.  Every scorer
       // thread runs all L levels and reaches each barrier, also after an
       // abort (its waits then fail at once and the level's lists hold
       // placeholders of bounded size), so no warp waits at a barrier alone.
       sync_scorers();
-      for (int c = t; c < n; c += 128) {
-        const float p0 = part[c], p1 = part[kMaxCand + c], p2 = part[2 * kMaxCand + c], p3 = part[3 * kMaxCand + c];
-        const float M = fmaxf(fmaxf(p0, p1), fmaxf(p2, p3));
+      for (int c = t; c < n; c += kScorers) {
+        float pv[8];
+        float M = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          pv[x] = part[x * kMaxCand + c];
+          M = fmaxf(M, pv[x]);
+        }
         float sc = -INFINITY;
-        if (M != -INFINITY)
-          sc = (M + __log2f(fast_exp2(p0 - M) + fast_exp2(p1 - M) + fast_exp2(p2 - M) + fast_exp2(p3 - M))) * ln2;
+        if (M != -INFINITY) {
+          float S = 0.f;
+#pragma unroll
+          for (int x = 0; x < 8; ++x) S += fast_exp2(pv[x] - M);
+          sc = (M + __log2f(S)) * ln2;
+        }
         score[c] = sc;
       }
       sync_scorers();
       const int kk = n < a.K ? n : a.K;
-      for (int c = t; c < n; c += 128) {
+      for (int c = t; c < n; c += kScorers) {
         const float s = score[c];
         int rank = 0;
         for (int c2 = 0; c2 < n; ++c2) {
@@ -292,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int nbuf = buf ^ 1;
       int32_t* nl = cand + nbuf * kMaxCand;
       const int p = 1 << log2p;
-      for (int c = t; c < n; c += 128) {
+      for (int c = t; c < n; c += kScorers) {
         if (!flag[c]) continue;
         int pos = 0;
         for (int c2 = 0; c2 < c; ++c2) pos += flag[c2];
@@ -301,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (l > 0)
           for (int x = 0; x < p; ++x) nl[pos * p + x] = cl[c] * p + x;
       }
-      for (int pos = kk + t; pos < a.K; pos += 128) {
+      for (int pos = kk + t; pos < a.K; pos += kScorers) {
         a.kept_idx[out0 + (int64_t)l * a.K + pos] = -1;
         a.kept_score[out0 + (int64_t)l * a.K + pos] = -INFINITY;
       }
@@ -438,9 +536,9 @@ lh_status pisa_plan_impl(const lh_pisa_config* cfg, lh_pisa_info* info) {
   if (N % top_span != 0) return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: N must be divisible by block * p^(L-1)");
   if (N % G != 0) return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: N must be divisible by the group size");
   const int64_t n_top = N / top_span;
-  if (n_top > kMaxCand) return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: the coarsest level has more than 512 blocks");
+  if (n_top > kMaxCand) return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: the coarsest level has more than 256 blocks");
   if ((int64_t)p * K > kMaxCand && L > 1)
-    return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: p * topk must be <= 512");
+    return fail(LH_ERR_UNSUPPORTED, "lh_pisa_plan: p * topk must be <= 256");
   int64_t upper = 0;
   for (int l = 0; l < L; ++l) {
     info->blocks[l] = (N >> (l * log2p)) / C;

@@ -289,7 +289,7 @@ lh_status lh_backward(const lh_config *cfg, const void *dy, const void *ctx, siz
  *    included) to the lower block index.
  * Support: bf16 Q and K [B][H][N][d]; d in {64, 128}; block in {64, 128};
  * group = 128; p a power of two >= 2; 1 <= L <= 8; N divisible by
- * block * p^(L-1) and < 2^28; blocks[L-1] <= 512 and p * topk <= 512;
+ * block * p^(L-1) and < 2^28; blocks[L-1] <= 256 and p * topk <= 256;
  * B*H <= 65535.
  * ------------------------------------------------------------------------- */
 typedef struct {
