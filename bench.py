@@ -235,7 +235,8 @@ def time_stages(calls, iters: int) -> dict:
 def source_sha(kernel: str) -> str:
     files = {"pool": "lh_pool.cu", "pool_adjoint": "lh_pool.cu", "score_topk": "lh_select.cu",
              "gather": "lh_gather.cu", "scatter_back": "lh_gather.cu", "scatter_adjoint": "lh_gather.cu",
-             "attn_fwd": "lh_attn_fwd.cu", "attn_bwd": "lh_attn_bwd.cu"}
+             "attn_fwd": "lh_attn_fwd.cu", "attn_bwd": "lh_attn_bwd.cu", "select": "lh_pisa.cu",
+             "pool_keys": "lh_pisa.cu"}
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_sparse_attention_pyramid_b200", "csrc")
     for f in (files[kernel], "lh_common.cuh", "sm100.cuh"):
@@ -468,7 +469,7 @@ def run_pisa(args, world, rank, local):
     mma_flops = 2.0 * exps * w.d
     roofline = {"bound": "alu", "kernel": "select", "kernels": ["pisa_select_kernel"],
                 "achieved": exps / t_sel / 1e12, "peak": mufu_peak, "unit": "T ex2/s",
-                "frac": exps / t_sel / 1e12 / mufu_peak, "traffic": None, "peak_source":
+                "frac": exps / t_sel / 1e12 / mufu_peak, "traffic": measured_traffic("select", w.name), "peak_source":
                 f"derived: {SMS} SMs x {MUFU_EX2_PER_CLK_SM} ex2/clk x {sm_mhz:.0f} MHz",
                 "scored_blocks": scored, "exp_per_block": w.group * w.block,
                 "tensor": {"achieved_tflops": mma_flops / t_sel / 1e12, "peak": pk["bf16_tflops"],

@@ -421,25 +421,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 // key pyramid
 // ---------------------------------------------------------------------------
 
-// x rounded to the nearest bf16 value, ties to even, straight from binary64
-// (IEEE 754 round-to-nearest-even applied to the 7 stored fraction bits).
-// Magnitudes below the normal bf16 range become a signed zero.
+// x rounded to the nearest bf16 value, ties to even, as if straight from
+// binary64: x is first rounded to fp32 with round-to-odd (truncate, then set
+// the last bit when anything was cut off), then to bf16 with round-to-nearest-
+// even.  Rounding to odd at a precision at least two bits above the target's
+// makes the second rounding the correct one (Boldo and Melquiond, "Emulation
+// of FMA and correctly rounded sums: proved algorithms using rounding to
+// odd", IEEE Trans. Computers 57(4), 2008); fp32 keeps 24 bits, bf16 8.
 __device__ __forceinline__ uint16_t bf16_from_double_rne(double x) {
-  const uint64_t u = (uint64_t)__double_as_longlong(x);
-  const uint32_t sign = (uint32_t)(u >> 63) << 15;
-  int e = (int)((u >> 52) & 0x7FF);
-  const uint64_t frac = u & ((1ull << 52) - 1);
-  uint64_t keep = frac >> 45;
-  const uint64_t rest = frac & ((1ull << 45) - 1), half = 1ull << 44;
-  if (rest > half || (rest == half && (keep & 1))) ++keep;
-  if (keep == 128) {
-    keep = 0;
-    ++e;
-  }
-  const int fe = e - 1023 + 127;
-  if (e == 0 || fe <= 0) return (uint16_t)sign;
-  if (fe >= 255) return (uint16_t)(sign | 0x7F80u);
-  return (uint16_t)(sign | ((uint32_t)fe << 7) | (uint32_t)keep);
+  float r = __double2float_rz(x);
+  if ((double)r != x) r = __uint_as_float(__float_as_uint(r) | 1u);
+  return __bfloat16_as_ushort(__float2bfloat16_rn(r));
 }
 
 struct PoolKArgs {
@@ -450,24 +442,24 @@ struct PoolKArgs {
   int64_t level_off[kMaxLevels];
 };
 
-template <int D>
+template <int D, int NL>
 __global__ void __launch_bounds__(256) pisa_pool_kernel(PoolKArgs a) {
   constexpr int VE = D / 32;  // columns per lane
   using Raw = typename RawVec<2 * VE>::type;
   const int lane = threadIdx.x & 31;
-  const int span_log = (a.L - 1) * a.log2p;
+  const int span_log = (NL - 1) * a.log2p;
   const int64_t spans = a.N >> span_log;
   const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (w >= a.BH * spans) return;
   const int64_t bh = w / spans, s = w % spans;
   const int span = 1 << span_log;
   const __nv_bfloat16* src = a.k + ((bh * a.N + (s << span_log)) * D) + lane * VE;
-  double acc[kMaxLevels][VE];
+  double acc[NL][VE];  // acc[l]: running sum of the level-l entry being built (l >= 1)
 #pragma unroll
-  for (int l = 0; l < kMaxLevels; ++l)
+  for (int l = 0; l < NL; ++l)
 #pragma unroll
     for (int v = 0; v < VE; ++v) acc[l][v] = 0.0;
-  constexpr int U = 8;
+  constexpr int U = 16;  // rows in flight per lane
   for (int r0 = 0; r0 < span; r0 += U) {
     Raw raw[U];
 #pragma unroll
@@ -481,8 +473,8 @@ __global__ void __launch_bounds__(256) pisa_pool_kernel(PoolKArgs a) {
       for (int v = 0; v < VE; ++v) acc[1][v] += (double)__bfloat162float(e[v]);
       const int done = r0 + x + 1;  // rows of the span summed so far
 #pragma unroll
-      for (int l = 1; l < kMaxLevels; ++l) {
-        if (l >= a.L || (done & ((1 << (l * a.log2p)) - 1)) != 0) break;
+      for (int l = 1; l < NL; ++l) {
+        if ((done & ((1 << (l * a.log2p)) - 1)) != 0) break;
         // level l entry complete: mean = sum * 2^-(l log2 p), exact
         const double inv = ldexp(1.0, -l * a.log2p);
         const int64_t entry = ((s << span_log) + done) >> (l * a.log2p);
@@ -492,7 +484,7 @@ __global__ void __launch_bounds__(256) pisa_pool_kernel(PoolKArgs a) {
         Raw packed;
         memcpy(&packed, o, sizeof(packed));
         *reinterpret_cast<Raw*>(a.pyr + (bh * a.upper + a.level_off[l] + entry - 1) * D + lane * VE) = packed;
-        if (l + 1 < kMaxLevels) {
+        if (l + 1 < NL) {
 #pragma unroll
           for (int v = 0; v < VE; ++v) acc[l + 1][v] += acc[l][v];
         }
@@ -501,6 +493,18 @@ __global__ void __launch_bounds__(256) pisa_pool_kernel(PoolKArgs a) {
       }
     }
   }
+}
+
+template <int D>
+cudaError_t launch_pool_keys_t(const PoolKArgs& a, unsigned blocks, cudaStream_t st) {
+  switch (a.L) {
+#define LH_CASE(n) \
+  case n: pisa_pool_kernel<D, n><<<blocks, 256, 0, st>>>(a); break;
+    LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 lh_status fail(lh_status s, const char* what) {
@@ -591,11 +595,8 @@ lh_status lh_pisa_pool_keys(const lh_pisa_config* cfg, const void* k, void* kpyr
   for (int l = 0; l < kMaxLevels; ++l) a.level_off[l] = info.level_off[l];
   const int64_t warps = a.BH * (a.N >> ((a.L - 1) * a.log2p));
   const unsigned blocks = (unsigned)((warps + 7) / 8);
-  if (cfg->d == 128)
-    pisa_pool_kernel<128><<<blocks, 256, 0, (cudaStream_t)stream>>>(a);
-  else
-    pisa_pool_kernel<64><<<blocks, 256, 0, (cudaStream_t)stream>>>(a);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = cfg->d == 128 ? launch_pool_keys_t<128>(a, blocks, (cudaStream_t)stream)
+                                      : launch_pool_keys_t<64>(a, blocks, (cudaStream_t)stream);
   if (e != cudaSuccess) {
     set_error_message("lh_pisa_pool_keys: %s", cudaGetErrorString(e));
     return LH_ERR_CUDA;
