@@ -86,7 +86,8 @@ def check_group(Qh, levels, w, g, idx, sco):
         want = sc[pos]
         got = sco[lv, :kk].astype(np.float64)
         both_inf = np.isneginf(want) & np.isneginf(got)
-        diff = np.abs(np.where(both_inf, 0.0, got - want))
+        with np.errstate(invalid="ignore"):
+            diff = np.abs(np.where(both_inf, 0.0, got - want))
         assert np.all(diff <= EPS), (g, lv, got, want)
         o_kept, _ = po.top_blocks(cands, sc, K)
         if not np.array_equal(o_kept, kept):
