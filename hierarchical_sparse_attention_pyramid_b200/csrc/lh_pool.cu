@@ -185,15 +185,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
   };
 
   // two batches in flight: the loads of the next batch are issued before the
-  // current one is processed
-  Raw xa[U], xb[U];
-  load(xa, 0);
-  for (int r0 = 0; r0 < rows; r0 += 2 * U) {
-    if (r0 + U < rows) load(xb, r0 + U);
-    process(xa, r0);
-    if (r0 + U >= rows) break;
-    if (r0 + 2 * U < rows) load(xa, r0 + 2 * U);
-    process(xb, r0 + U);
+  // current one is processed (one copy of the processing code, so the loop
+  // body stays small in the instruction cache)
+  Raw cur[U], nxt[U];
+  load(cur, 0);
+  for (int r0 = 0; r0 < rows; r0 += U) {
+    if (r0 + U < rows) load(nxt, r0 + U);
+    process(cur, r0);
+#pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
   }
 }
 
