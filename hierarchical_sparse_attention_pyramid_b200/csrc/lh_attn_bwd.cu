@@ -11,12 +11,14 @@
 // Two kernels, each writing its gradient once (no atomics):
 //
 // attn_bwd_kv_kernel (dKs, dVs) - one CTA per 128-row key tile; it steps over
-//   64-query half tiles from the diagonal to the end.  For half step s the MMA
-//   warp computes S^T = K Q_h^T and dP^T = V dO_h^T into TMEM buffer s&1 while
-//   the compute warpgroups work on the other buffer; they write P^T and dS^T
-//   (hi/lo) back over the columns they read, and the MMA warp then adds
-//   dV += P^T dO_h and dK += dS^T Q_h with both A operands read from TMEM.
-//   Q_h, dO_h stream through a 4-slot ring.
+//   128-query tiles from the diagonal to the end.  For step j the MMA warp
+//   computes S^T = K Q_j^T and dP^T = V dO_j^T (N = 128) into TMEM; the
+//   compute warpgroups write P^T and dS^T (hi/lo) back over the columns they
+//   read, and the MMA warp adds dV += P^T dO_j and dK += dS^T Q_j with both A
+//   operands read from TMEM.  The next step's S^T is issued right after dV(j)
+//   and its dP^T right after dK(j), so the tensor core works on one step's
+//   products while the compute warps turn the other's scores around.  Q_j,
+//   dO_j stream through a 2-slot ring.
 //
 // attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over the
 //   128-key tiles up to the diagonal.  S = Q K_j^T runs two tiles ahead into a
@@ -27,8 +29,10 @@
 //   V through 2.
 //
 // Warp roles in both: warps 0-7 two compute warpgroups (thread (g, t) owns
-// TMEM lane t and columns [32g, 32g+32) of each 64-column half), warp 8 TMA
-// producer, warp 9 MMA issuer (one thread) and TMEM owner.
+// TMEM lane t and 64 columns of each step: [64g, 64g+64) in the dK/dV kernel,
+// the columns [32g, 32g+32) of each 64-column half in the dQ kernel), warp 8
+// TMA producer, warp 9 MMA issuer (a converged warp; one elected lane issues)
+// and TMEM owner.
 #include <math.h>
 
 #include "lh_common.cuh"
@@ -44,7 +48,6 @@ using namespace sm100;
 constexpr int kCompute = 256;
 constexpr int kThreads = kCompute + 64;
 constexpr int kRegion = 128 * 128;  // one [128 rows][64 bf16] SW128 region
-constexpr int kHalfRegion = 64 * 128;
 
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -60,22 +63,21 @@ __device__ __forceinline__ void store_pair_chunk(uint32_t taddr, const uint32_t 
 // ===========================================================================
 template <int D>
 struct KvSmem {
-  static constexpr int kTile = D / 64 * kRegion;         // K or V tile, 128 rows
-  static constexpr int kHalf = D / 64 * kHalfRegion;     // Q_h or dO_h, 64 rows
+  static constexpr int kTile = D / 64 * kRegion;         // one 128-row tile: K, V, Q_j or dO_j
   static constexpr int oK = 0;
   static constexpr int oV = oK + kTile;
-  static constexpr int oRing = oV + kTile;               // 4 slots of (Q_h, dO_h)
-  static constexpr int kSlot = 2 * kHalf;
-  static constexpr int oVec = oRing + 4 * kSlot;         // [2][128] floats: LSE*log2e [64], Delta [64]
-  static constexpr int oBar = oVec + 1024;
+  static constexpr int oRing = oV + kTile;               // 2 slots of (Q_j, dO_j)
+  static constexpr int kSlot = 2 * kTile;
+  static constexpr int oVec = oRing + 2 * kSlot;         // [2][256] floats: LSE*log2e [128], Delta [128]
+  static constexpr int oBar = oVec + 2048;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOh,
+    attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dK,
                        float* __restrict__ dV, int* errw, int S, float scale_log2, float scale) {
   using Lay = KvSmem<D>;
@@ -83,13 +85,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bKV = bars + 0;        // K, V landed
-  uint64_t* bLoad = bars + 1;      // [4] Q_h, dO_h of a ring slot landed
-  uint64_t* bSlotFree = bars + 5;  // [4] dV, dK products done with a slot
-  uint64_t* bS = bars + 9;         // [2] S^T of a half step in TMEM buffer
-  uint64_t* bDP = bars + 11;       // [2] dP^T of a half step in TMEM buffer
-  uint64_t* bP = bars + 13;        // [2] P^T written back (256 arrivals)
-  uint64_t* bDS = bars + 15;       // [2] dS^T written back (256 arrivals)
-  uint64_t* bDone = bars + 17;     // every product done
+  uint64_t* bLoad = bars + 1;      // [2] Q_j, dO_j of a ring slot landed
+  uint64_t* bSlotFree = bars + 3;  // [2] dV, dK products done with a slot
+  uint64_t* bS = bars + 5;         // S^T of the step in TMEM
+  uint64_t* bDP = bars + 6;        // dP^T of the step in TMEM
+  uint64_t* bP = bars + 7;         // P^T written back (256 arrivals)
+  uint64_t* bDS = bars + 8;        // dS^T written back (256 arrivals)
+  uint64_t* bDone = bars + 9;      // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
   float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);
@@ -98,20 +100,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_qt = (S + 127) / 128;
   const int kt = (int)blockIdx.x;  // key tile; small kt = most query tiles, launched first
   const int bh = (int)blockIdx.y;
-  const int NS = 2 * (n_qt - kt);  // half steps
+  const int NJ = n_qt - kt;        // 128-query steps, from the diagonal tile on
 
   if (threadIdx.x == 0) {
     mbar_init(bKV, 1);
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bLoad[i], 1);
       mbar_init(&bSlotFree[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bS[i], 1);
-      mbar_init(&bDP[i], 1);
-      mbar_init(&bP[i], kCompute);
-      mbar_init(&bDS[i], kCompute);
-    }
+    mbar_init(bS, 1);
+    mbar_init(bDP, 1);
+    mbar_init(bP, kCompute);
+    mbar_init(bDS, kCompute);
     mbar_init(bDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -121,145 +121,150 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr uint32_t tSP = 0, tDP = 128, tDV = 256, tDK = 256 + D;  // SP/DP: [2] x 64 columns
+  constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQh);
-      tma_prefetch_desc(&tmOh);
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmO);
       mbar_expect_tx(bKV, 2 * 128 * D * 2);
       for (int c = 0; c < D / 64; ++c) {
         tma_load_3d(smem + Lay::oK + c * kRegion, &tmK, bKV, c * 64, kt * 128, bh);
         tma_load_3d(smem + Lay::oV + c * kRegion, &tmV, bKV, c * 64, kt * 128, bh);
       }
-      for (int s = 0; s < NS; ++s) {
-        const int slot = s & 3;
-        if (s >= 4 && !mbar_wait(&bSlotFree[slot], ((s >> 2) - 1) & 1, abort_flag)) break;
-        const int q0 = (kt + (s >> 1)) * 128 + (s & 1) * 64;
+      for (int j = 0; j < NJ; ++j) {
+        const int slot = j & 1;
+        if (j >= 2 && !mbar_wait(&bSlotFree[slot], ((j >> 1) - 1) & 1, abort_flag)) break;
+        const int q0 = (kt + j) * 128;
         uint8_t* base = smem + Lay::oRing + slot * Lay::kSlot;
-        mbar_expect_tx(&bLoad[slot], 2 * 64 * D * 2);
+        mbar_expect_tx(&bLoad[slot], 2 * 128 * D * 2);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + c * kHalfRegion, &tmQh, &bLoad[slot], c * 64, q0, bh);
-          tma_load_3d(base + Lay::kHalf + c * kHalfRegion, &tmOh, &bLoad[slot], c * 64, q0, bh);
+          tma_load_3d(base + c * kRegion, &tmQ, &bLoad[slot], c * 64, q0, bh);
+          tma_load_3d(base + Lay::kTile + c * kRegion, &tmO, &bLoad[slot], c * 64, q0, bh);
         }
       }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per step j: dV(j) once P^T(j) is back, S^T(j+1) (over the P^T
+    // columns dV(j) has read: the tensor core runs in issue order), dK(j) once
+    // dS^T(j) is back, dP^T(j+1) (over the dS^T columns dK(j) has read).
     {  // the whole warp; one elected lane issues each instruction
-      constexpr uint32_t idF = idesc_bf16(128, 64, false, false);  // S^T, dP^T: N = 64 queries
-      constexpr uint32_t idG = idesc_bf16(128, D, false, true);    // dV, dK: A from TMEM, B MN-major
+      constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S^T, dP^T: N = 128 queries
+      constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dV, dK: A from TMEM, B MN-major
       const uint32_t sRing = smem_u32(smem + Lay::oRing);
       const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
       const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
       const uint64_t kRing = sdesc_sw128(sRing, 16, 1024);
-      const uint64_t mRing = sdesc_sw128(sRing, kHalfRegion, 1024);
-      bool ok = mbar_wait_warp(bKV, 0, abort_flag);
-      // the loads of half step s landed (waited for before the products that
-      // precede its F in the issue order, so no wait sits between them)
-      auto wait_f = [&](int s) -> bool { return mbar_wait_warp(&bLoad[s & 3], (s >> 2) & 1, abort_flag); };
-      // S^T = K Q_h^T, then dP^T = V dO_h^T, of half step s into TMEM buffer s & 1,
-      // each with its own completion so the P^T pass can start on S^T alone
-      auto issue_f = [&](int s) {
-        const int slot = s & 3, b = s & 1;
-        tc_fence_after();
-        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
+      const uint64_t mRing = sdesc_sw128(sRing, kRegion, 1024);
+      auto wait_load = [&](int j) -> bool { return mbar_wait_warp(&bLoad[j & 1], (j >> 1) & 1, abort_flag); };
+      auto issue_s = [&](int j) {
+        const uint32_t qo = ((j & 1) * Lay::kSlot) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // K tile (128 rows)
-          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // Q_h (64 rows)
-          umma_bf16_w(tmem + tSP + b * 64, kK + at, kRing + qo + bt, idF, kk > 0 ? 1u : 0u);
+          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + tS, kK + at, kRing + qo + at, idF, kk > 0 ? 1u : 0u);
         }
-        umma_commit_w(&bS[b]);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;    // V tile
-          const uint32_t bt = ((kk >> 2) * kHalfRegion + (kk & 3) * 32) >> 4;  // dO_h
-          umma_bf16_w(tmem + tDP + b * 64, kV + at, kRing + oo + bt, idF, kk > 0 ? 1u : 0u);
-        }
-        umma_commit_w(&bDP[b]);
+        umma_commit_w(bS);
       };
-      if (ok && (ok = wait_f(0))) issue_f(0);
-      if (ok && NS > 1 && (ok = wait_f(1))) issue_f(1);
-      for (int s = 0; ok && s < NS; ++s) {
-        const int slot = s & 3, b = s & 1;
-        if (s + 2 < NS && !wait_f(s + 2)) { ok = false; break; }
-        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kHalf) >> 4;
-        // dV += P^T dO_h as soon as P^T is back (16 queries per step; hi of
-        // chunk kk/2 at +(kk&1)*8, lo at +16), then dK += dS^T Q_h
-        if (!mbar_wait_warp(&bP[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
+      auto issue_dp = [&](int j) {
+        const uint32_t oo = ((j & 1) * Lay::kSlot + Lay::kTile) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
+          umma_bf16_w(tmem + tDP, kV + at, kRing + oo + at, idF, kk > 0 ? 1u : 0u);
+        }
+        umma_commit_w(bDP);
+      };
+      bool ok = mbar_wait_warp(bKV, 0, abort_flag) && wait_load(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
+      for (int j = 0; ok && j < NJ; ++j) {
+        const int slot = j & 1;
+        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kTile) >> 4;
+        // dV += P^T dO_j (16 queries per MMA; hi of chunk kk/2 at +(kk&1)*8, lo at +16)
+        if (!mbar_wait_warp(bP, j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a = tmem + tSP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           const uint64_t bo = mRing + oo + ((kk * 2048) >> 4);
           umma_bf16_tmem_a_w(tmem + tDV, a, bo, idG, acc);
           umma_bf16_tmem_a_w(tmem + tDV, a + 16, bo, idG, 1u);
         }
-        if (!mbar_wait_warp(&bDS[b], (s >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (j + 1 < NJ) {
+          if (!wait_load(j + 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        // dK += dS^T Q_j
+        if (!mbar_wait_warp(bDS, j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a = tmem + tDP + b * 64 + (kk >> 1) * 32 + (kk & 1) * 8;
-          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a = tmem + tDP + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           const uint64_t bq = mRing + qo + ((kk * 2048) >> 4);
           umma_bf16_tmem_a_w(tmem + tDK, a, bq, idG, acc);
           umma_bf16_tmem_a_w(tmem + tDK, a + 16, bq, idG, 1u);
         }
         umma_commit_w(&bSlotFree[slot]);
-        // the next half step that uses this TMEM buffer; its S^T, dP^T land
-        // after the products above have read P^T and dS^T (in-order issue)
-        if (s + 2 < NS) issue_f(s + 2);
+        if (j + 1 < NJ) issue_dp(j + 1);
       }
       if (ok) umma_commit_w(bDone);
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
     const int ct = threadIdx.x;            // 0..255
-    const int g = warp >> 2;               // query columns [32g, 32g+32) of each half
+    const int g = warp >> 2;               // query columns [64g, 64g+64) of each step
     const int t = (warp & 3) * 32 + lane;  // key row of the tile (TMEM lane)
     const int kv_g = kt * 128 + t;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     bool ok = true;
-    // LSE (ct < 64) or Delta (64 <= ct < 128) of query row ct & 63 of half
-    // step s, loaded one half step ahead and converted when it is stored
-    auto vec_row = [&](int s) { return (kt + (s >> 1)) * 128 + (s & 1) * 64 + (ct & 63); };
-    auto vec_raw = [&](int s) -> float {
-      const int qg = vec_row(s);
-      return qg < S ? ldg_nc_f32((ct < 64 ? LSE : Delta) + (int64_t)bh * S + qg) : 0.f;
+    // LSE (ct < 128) or Delta (ct >= 128) of query row ct & 127 of step j,
+    // loaded one step ahead and converted when it is stored
+    auto vec_row = [&](int j) { return (kt + j) * 128 + (ct & 127); };
+    auto vec_raw = [&](int j) -> float {
+      const int qg = vec_row(j);
+      return qg < S ? ldg_nc_f32((ct < 128 ? LSE : Delta) + (int64_t)bh * S + qg) : 0.f;
     };
-    float vec_next = ct < 128 ? vec_raw(0) : 0.f;
+    float vec_next = vec_raw(0);
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
-    for (int s = 0; s < NS; ++s) {
-      const int b = s & 1;
+    const uint64_t sc2 = f2_pack(scale, scale);
+    for (int j = 0; j < NJ; ++j) {
+      const int b = j & 1;
       const float vec_cur = vec_next;
-      if (ct < 128 && s + 1 < NS) vec_next = vec_raw(s + 1);
-      if (ct < 64) sVec[b * 128 + ct] = vec_row(s) < S ? vec_cur * 1.4426950408889634f : INFINITY;
-      else if (ct < 128) sVec[b * 128 + ct] = vec_cur;
+      if (j + 1 < NJ) vec_next = vec_raw(j + 1);
+      if (ct < 128) sVec[b * 256 + ct] = vec_row(j) < S ? vec_cur * 1.4426950408889634f : INFINITY;
+      else sVec[b * 256 + ct] = vec_cur;
       compute_sync();
-      const float* lse = sVec + b * 128;
-      const float* del = lse + 64;
-      const int q0 = (kt + (s >> 1)) * 128 + (s & 1) * 64;
-      const bool diag = (s >> 1) == 0;  // the diagonal query tile
+      const float* lse = sVec + b * 256;
+      const float* del = lse + 128;
+      const int q0 = (kt + j) * 128;
+      const bool diag = j == 0;  // the diagonal query tile
       // warp-uniform outcome for the collective TMEM accesses; after a failed
       // wait the loop keeps its compute_sync count and skips the work
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&bS[b], (s >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bS, j & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      // P^T as a bf16 pair over the S^T columns just read (hi in the first 16
-      // columns of the 32-query chunk, lo in the last 16); the dV product
-      // starts on it while dP^T is still being computed
-      float p[32];
-      {
+      // P^T as bf16 pairs over the S^T columns just read (per 32-query chunk:
+      // hi in the first 16 columns, lo in the last 16); dV starts on it while
+      // dP^T is still being computed
+      float p[2][32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t sr[32];
-        tmem_ld32(tl + tSP + b * 64 + g * 32, sr);
+        tmem_ld32(tl + tS + g * 64 + c * 32, sr);
         tmem_ld_wait();
         uint32_t phi[16], plo[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int qi = g * 32 + e;
+          const int qi = g * 64 + c * 32 + e;
           const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
           float pa, pb;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)),
@@ -270,39 +275,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q0 + qi < kv_g) pa = 0.f;
             if (q0 + qi + 1 < kv_g) pb = 0.f;
           }
-          p[e] = pa;
-          p[e + 1] = pb;
+          p[c][e] = pa;
+          p[c][e + 1] = pb;
           split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
         }
-        store_pair_chunk(tl + tSP + b * 64 + g * 32, phi, plo);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bP[b]);
+        store_pair_chunk(tl + tS + g * 64 + c * 32, phi, plo);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&bDP[b], (s >> 1) & 1, abort_flag));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bP);
+      ok = __all_sync(0xffffffffu, mbar_wait(bDP, j & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      // dS^T = P^T (dP^T - Delta) / sqrt(d) as a bf16 pair over the dP^T columns
-      {
+      // dS^T = P^T (dP^T - Delta) / sqrt(d) as bf16 pairs over the dP^T columns
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(tl + tDP + b * 64 + g * 32, dr);
+        tmem_ld32(tl + tDP + g * 64 + c * 32, dr);
         tmem_ld_wait();
         uint32_t dhi[16], dlo[16];
-        const uint64_t sc2 = f2_pack(scale, scale);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float2 d2 = *reinterpret_cast<const float2*>(del + g * 32 + e);
+          const float2 d2 = *reinterpret_cast<const float2*>(del + g * 64 + c * 32 + e);
           const uint64_t diff2 =
               f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(d2.x, d2.y));
           float da, db;
-          f2_unpack(f2_mul(f2_mul(f2_pack(p[e], p[e + 1]), sc2), diff2), da, db);
+          f2_unpack(f2_mul(f2_mul(f2_pack(p[c][e], p[c][e + 1]), sc2), diff2), da, db);
           split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
         }
-        store_pair_chunk(tl + tDP + b * 64 + g * 32, dhi, dlo);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bDS[b]);
+        store_pair_chunk(tl + tDP + g * 64 + c * 32, dhi, dlo);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bDS);
     }
     if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
       tc_fence_after();
@@ -590,9 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) report_error(errw, ERRW_TIMEOUT);
 }
 
-// TMA maps of the sequences: full 128-row boxes and 64-row half boxes
+// TMA maps of the sequences, 128-row boxes
 struct SeqMaps {
-  CUtensorMap q, qh, k, v, o, oh;
+  CUtensorMap q, k, v, o;
 };
 
 template <int D>
@@ -602,7 +607,7 @@ cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* l
   int smem = KvSmem<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.qh, m.k, m.v, m.oh, lse, delta, dks, dvs,
+  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
                                                                          errw, (int)S, scale_log2, scale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -620,9 +625,8 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const 
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
                             float* dvs, int* errw, cudaStream_t st) {
   SeqMaps m;
-  if (!make_seq_map(&m.q, qs, BH, S, d, 128) || !make_seq_map(&m.qh, qs, BH, S, d, 64) ||
-      !make_seq_map(&m.k, ks, BH, S, d, 128) || !make_seq_map(&m.v, vs, BH, S, d, 128) ||
-      !make_seq_map(&m.o, dos, BH, S, d, 128) || !make_seq_map(&m.oh, dos, BH, S, d, 64))
+  if (!make_seq_map(&m.q, qs, BH, S, d, 128) || !make_seq_map(&m.k, ks, BH, S, d, 128) ||
+      !make_seq_map(&m.v, vs, BH, S, d, 128) || !make_seq_map(&m.o, dos, BH, S, d, 128))
     return cudaErrorInvalidValue;
   const double scale = 1.0 / sqrt((double)d);
   const float scale_log2 = (float)(1.4426950408889634 * scale);
