@@ -45,11 +45,14 @@ bool make_seq_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, in
 namespace {
 using namespace sm100;
 
-constexpr int kCompute = 256;
+constexpr int kCompute = 256;    // dQ kernel: two compute warpgroups
 constexpr int kThreads = kCompute + 64;
+constexpr int kComputeKV = 512;  // dK/dV kernel: four compute warpgroups
+constexpr int kThreadsKV = kComputeKV + 64;
 constexpr int kRegion = 128 * 128;  // one [128 rows][64 bf16] SW128 region
 
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void compute_sync_kv() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
 // P^T / dS (hi, lo) of 32 columns c0..c0+31 of one row as bf16 pairs over the
 // 32 TMEM columns they were read from: hi in the first 16, lo in the last 16.
@@ -75,7 +78,7 @@ struct KvSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsKV, 1)
     attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dK,
@@ -89,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bSlotFree = bars + 3;  // [2] dV, dK products done with a slot
   uint64_t* bS = bars + 5;         // S^T of the step in TMEM
   uint64_t* bDP = bars + 6;        // dP^T of the step in TMEM
-  uint64_t* bP = bars + 7;         // P^T written back (256 arrivals)
-  uint64_t* bDS = bars + 8;        // dS^T written back (256 arrivals)
+  uint64_t* bP = bars + 7;         // P^T written back (one arrival per compute thread)
+  uint64_t* bDS = bars + 8;        // dS^T written back (one arrival per compute thread)
   uint64_t* bDone = bars + 9;      // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
@@ -110,20 +113,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bS, 1);
     mbar_init(bDP, 1);
-    mbar_init(bP, kCompute);
-    mbar_init(bDS, kCompute);
+    mbar_init(bP, kComputeKV);
+    mbar_init(bDS, kComputeKV);
     mbar_init(bDone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  if (warp == 17) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   constexpr uint32_t tS = 0, tDP = 128, tDV = 256, tDK = 256 + D;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer
     // Order per step j: dV(j) once P^T(j) is back, S^T(j+1) (over the P^T
     // columns dV(j) has read: the tensor core runs in issue order), dK(j) once
@@ -220,29 +223,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
-    const int ct = threadIdx.x;            // 0..255
-    const int g = warp >> 2;               // query columns [64g, 64g+64) of each step
+    const int ct = threadIdx.x;            // 0..511
+    const int g = warp >> 2;               // query columns [32g, 32g+32) of each step
     const int t = (warp & 3) * 32 + lane;  // key row of the tile (TMEM lane)
     const int kv_g = kt * 128 + t;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     bool ok = true;
-    // LSE (ct < 128) or Delta (ct >= 128) of query row ct & 127 of step j,
-    // loaded one step ahead and converted when it is stored
+    // LSE (ct < 128) or Delta (128 <= ct < 256) of query row ct & 127 of
+    // step j, loaded one step ahead and converted when it is stored
     auto vec_row = [&](int j) { return (kt + j) * 128 + (ct & 127); };
     auto vec_raw = [&](int j) -> float {
       const int qg = vec_row(j);
       return qg < S ? ldg_nc_f32((ct < 128 ? LSE : Delta) + (int64_t)bh * S + qg) : 0.f;
     };
-    float vec_next = vec_raw(0);
+    float vec_next = ct < 256 ? vec_raw(0) : 0.f;
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const uint64_t sc2 = f2_pack(scale, scale);
     for (int j = 0; j < NJ; ++j) {
       const int b = j & 1;
       const float vec_cur = vec_next;
-      if (j + 1 < NJ) vec_next = vec_raw(j + 1);
+      if (ct < 256 && j + 1 < NJ) vec_next = vec_raw(j + 1);
       if (ct < 128) sVec[b * 256 + ct] = vec_row(j) < S ? vec_cur * 1.4426950408889634f : INFINITY;
-      else sVec[b * 256 + ct] = vec_cur;
-      compute_sync();
+      else if (ct < 256) sVec[b * 256 + ct] = vec_cur;
+      compute_sync_kv();
       const float* lse = sVec + b * 256;
       const float* del = lse + 128;
       const int q0 = (kt + j) * 128;
@@ -252,19 +255,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok && mbar_wait(bS, j & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      // P^T as bf16 pairs over the S^T columns just read (per 32-query chunk:
-      // hi in the first 16 columns, lo in the last 16); dV starts on it while
-      // dP^T is still being computed
-      float p[2][32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      // P^T as bf16 pairs over the 32 S^T columns just read (hi in the first
+      // 16, lo in the last 16); dV starts on it while dP^T is still being
+      // computed
+      float p[32];
+      {
         uint32_t sr[32];
-        tmem_ld32(tl + tS + g * 64 + c * 32, sr);
+        tmem_ld32(tl + tS + g * 32, sr);
         tmem_ld_wait();
         uint32_t phi[16], plo[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int qi = g * 64 + c * 32 + e;
+          const int qi = g * 32 + e;
           const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
           float pa, pb;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)),
@@ -275,11 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q0 + qi < kv_g) pa = 0.f;
             if (q0 + qi + 1 < kv_g) pb = 0.f;
           }
-          p[c][e] = pa;
-          p[c][e + 1] = pb;
+          p[e] = pa;
+          p[e + 1] = pb;
           split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
         }
-        store_pair_chunk(tl + tS + g * 64 + c * 32, phi, plo);
+        store_pair_chunk(tl + tS + g * 32, phi, plo);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -288,53 +290,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) continue;
       tc_fence_after();
       // dS^T = P^T (dP^T - Delta) / sqrt(d) as bf16 pairs over the dP^T columns
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      {
         uint32_t dr[32];
-        tmem_ld32(tl + tDP + g * 64 + c * 32, dr);
+        tmem_ld32(tl + tDP + g * 32, dr);
         tmem_ld_wait();
         uint32_t dhi[16], dlo[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float2 d2 = *reinterpret_cast<const float2*>(del + g * 64 + c * 32 + e);
+          const float2 d2 = *reinterpret_cast<const float2*>(del + g * 32 + e);
           const uint64_t diff2 =
               f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2_pack(d2.x, d2.y));
           float da, db;
-          f2_unpack(f2_mul(f2_mul(f2_pack(p[c][e], p[c][e + 1]), sc2), diff2), da, db);
+          f2_unpack(f2_mul(f2_mul(f2_pack(p[e], p[e + 1]), sc2), diff2), da, db);
           split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
         }
-        store_pair_chunk(tl + tDP + g * 64 + c * 32, dhi, dlo);
+        store_pair_chunk(tl + tDP + g * 32, dhi, dlo);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bDS);
     }
+    // dV and dK of this thread's key row, columns [g D/4, (g+1) D/4)
     if (__all_sync(0xffffffffu, ok && mbar_wait(bDone, 0, abort_flag))) {
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        const int col = g * (D / 2) + c * 32;
-        uint32_t rv[32], rk[32];
-        tmem_ld32(tl + tDV + col, rv);
-        tmem_ld32(tl + tDK + col, rk);
-        tmem_ld_wait();
-        if (kv_g < S) {
-          float4* dv4 = reinterpret_cast<float4*>(dV + ((int64_t)bh * S + kv_g) * D + col);
-          float4* dk4 = reinterpret_cast<float4*>(dK + ((int64_t)bh * S + kv_g) * D + col);
+      constexpr int CW = D / 4;
+      uint32_t rv[CW], rk[CW];
+      if constexpr (CW == 32) {
+        tmem_ld32(tl + tDV + g * CW, rv);
+        tmem_ld32(tl + tDK + g * CW, rk);
+      } else {
+        tmem_ld16(tl + tDV + g * CW, rv);
+        tmem_ld16(tl + tDK + g * CW, rk);
+      }
+      tmem_ld_wait();
+      if (kv_g < S) {
+        float4* dv4 = reinterpret_cast<float4*>(dV + ((int64_t)bh * S + kv_g) * D + g * CW);
+        float4* dk4 = reinterpret_cast<float4*>(dK + ((int64_t)bh * S + kv_g) * D + g * CW);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            dv4[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
-                                 __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
-            dk4[q] = make_float4(__uint_as_float(rk[4 * q]), __uint_as_float(rk[4 * q + 1]),
-                                 __uint_as_float(rk[4 * q + 2]), __uint_as_float(rk[4 * q + 3]));
-          }
+        for (int q = 0; q < CW / 4; ++q) {
+          dv4[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
+                               __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+          dk4[q] = make_float4(__uint_as_float(rk[4 * q]), __uint_as_float(rk[4 * q + 1]),
+                               __uint_as_float(rk[4 * q + 2]), __uint_as_float(rk[4 * q + 3]));
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -607,7 +611,7 @@ cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* l
   int smem = KvSmem<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
+  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreadsKV, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
                                                                          errw, (int)S, scale_log2, scale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
