@@ -23,10 +23,11 @@
 // attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over the
 //   128-key tiles up to the diagonal.  S = Q K_j^T runs two tiles ahead into a
 //   double-buffered TMEM region and dP = dO V_j^T one tile ahead; the compute
-//   warpgroups turn the scores into P as soon as they land, then write dS
-//   (hi/lo) over the dP columns, and dQ += dS K_j reads it from TMEM.  K
-//   streams through 3 stages (read by S(j) and, two tiles later, by dQ(j)),
-//   V through 2.
+//   warpgroups turn the scores into P as soon as they land, take dP into
+//   registers (which frees it for the next tile's dP), then write dS (hi/lo)
+//   over the tile's S columns, and dQ += dS K_j reads it from TMEM.  K streams
+//   through 3 stages (read by S(j) and, two tiles later, by dQ(j)), V
+//   through 2.
 //
 // Warp roles in both: warps 0-7 two compute warpgroups (thread (g, t) owns
 // TMEM lane t and 64 columns of each step: [64g, 64g+64) in the dK/dV kernel,
@@ -376,9 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bKfree = bars + 6;  // [3] the dQ product is done with a K stage
   uint64_t* bVfree = bars + 9;  // [2] the dP product is done with a V stage
   uint64_t* bS = bars + 11;     // [2] S of a key tile in TMEM buffer
-  uint64_t* bSfree = bars + 13; // [2] the scores of a buffer are in registers (256 arrivals)
+  uint64_t* bDPread = bars + 13;  // dP of the key tile is in registers (256 arrivals)
   uint64_t* bDP = bars + 15;    // dP of the current key tile in TMEM
-  uint64_t* bPS = bars + 16;    // dS written over dP (256 arrivals)
+  uint64_t* bPS = bars + 16;    // dS written over the tile's S columns (256 arrivals)
   uint64_t* bDone = bars + 17;  // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
@@ -399,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bV[i], 1);
       mbar_init(&bVfree[i], 1);
       mbar_init(&bS[i], 1);
-      mbar_init(&bSfree[i], kCompute);
     }
+    mbar_init(bDPread, kCompute);
     mbar_init(bDP, 1);
     mbar_init(bPS, kCompute);
     mbar_init(bDone, 1);
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  constexpr uint32_t tS = 0, tDP = 256, tDQ = 384;  // S: [2] x 128 columns; dP, then dS (hi/lo): 128
+  constexpr uint32_t tS = 0, tDP = 256, tDQ = 384;  // S, then dS (hi/lo): [2] x 128 columns; dP: 128
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -440,10 +441,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Per key tile j: dQ += dS(j) K_j, then dP(j+1) = dO V_{j+1}^T (over the dS
-    // columns just read), then S(j+2) = Q K_{j+2}^T into the S buffer that
-    // tile j's scores have left, so the scores are two tiles ahead of the
-    // softmax-gradient pass and dP one tile ahead.
+    // Per key tile j: dP(j+1) = dO V_{j+1}^T as soon as the compute warps hold
+    // dP(j) in registers, then dQ += dS(j) K_j once dS(j) is written over
+    // tile j's S columns, then S(j+2) = Q K_{j+2}^T into that S buffer (after
+    // dQ(j) has read it: the tensor core runs in issue order).  The scores
+    // are two tiles ahead of the softmax-gradient pass and dP one tile ahead.
     {  // the whole warp; one elected lane issues each instruction
       constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S, dP: N = 128 keys
       constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dQ: A from TMEM, B MN-major
@@ -486,26 +488,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int j = 0; ok && j < NJ; ++j) {
-        // operands of the products after dQ(j), waited for first so that no
-        // wait sits between them
-        if (j + 1 < NJ && !mbar_wait_warp(&bV[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (j + 2 < NJ) {
-          if (!mbar_wait_warp(&bK[(j + 2) % 3], ((j + 2) / 3) & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait_warp(&bSfree[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (j + 1 < NJ) {
+          if (!mbar_wait_warp(&bV[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(bDPread, j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(j + 1);
         }
         if (!mbar_wait_warp(bPS, j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint64_t mk = mK + (((j % 3) * Lay::kTile) >> 4);
+        const uint32_t sb = tmem + tS + (j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // 16 keys per step; hi of chunk kk/2 at +(kk&1)*8, lo at +16
-          const uint32_t a = tmem + tDP + (kk >> 1) * 32 + (kk & 1) * 8;
+          const uint32_t a = sb + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint64_t bk = mk + ((kk * 2048) >> 4);
           umma_bf16_tmem_a_w(tmem + tDQ, a, bk, idG, (j > 0 || kk > 0) ? 1u : 0u);
           umma_bf16_tmem_a_w(tmem + tDQ, a + 16, bk, idG, 1u);
         }
         umma_commit_w(&bKfree[j % 3]);
-        if (j + 1 < NJ) issue_dp(j + 1);  // after dQ(j) has read dS(j) (in-order issue)
-        if (j + 2 < NJ) issue_s(j + 2);
+        if (j + 2 < NJ) {
+          if (!mbar_wait_warp(&bK[(j + 2) % 3], ((j + 2) / 3) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(j + 2);
+        }
       }
       if (ok) umma_commit_w(bDone);
     }
@@ -525,14 +530,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bS[b], (j >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // P = 2^(s*scale*log2e - lse*log2e) of this thread's 64 keys; the S
-      // buffer is free once the scores are in registers
+      // P = 2^(s*scale*log2e - lse*log2e) of this thread's 64 keys
       uint32_t r[2][32];
       tmem_ld32(tl + tS + b * 128 + g * 64, r[0]);
       tmem_ld32(tl + tS + b * 128 + g * 64 + 32, r[1]);
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bSfree[b]);
       // keys after the row are masked on the diagonal tile: limit = row there,
       // past every key elsewhere
       const int limit = j == qt ? t - g * 64 : 1 << 20;
@@ -551,22 +553,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bDP, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // dS = P (dP - Delta) / sqrt(d) as a bf16 pair over the dP columns just
-      // read: per 32 keys, hi in the first 16 columns and lo in the last 16
+      // dS = P (dP - Delta) / sqrt(d) as a bf16 pair over this tile's S
+      // columns (read into registers above): per 32 keys, hi in the first 16
+      // columns and lo in the last 16.  dP is released as soon as it is in
+      // registers, so the next tile's dP can be computed meanwhile.
+      uint32_t dr[2][32];
+      tmem_ld32(tl + tDP + g * 64, dr[0]);
+      tmem_ld32(tl + tDP + g * 64 + 32, dr[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bDPread);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dr[32];
-        tmem_ld32(tl + tDP + g * 64 + ch * 32, dr);
-        tmem_ld_wait();
         uint32_t dhi[16], dlo[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), d2);
+          const uint64_t diff2 = f2_sub(f2_pack(__uint_as_float(dr[ch][e]), __uint_as_float(dr[ch][e + 1])), d2);
           float da, db;
           f2_unpack(f2_mul(f2_mul(f2_pack(p[ch][e], p[ch][e + 1]), sc2), diff2), da, db);
           split_bf16x2(da, db, dhi[e >> 1], dlo[e >> 1]);
         }
-        store_pair_chunk(tl + tDP + g * 64 + ch * 32, dhi, dlo);
+        store_pair_chunk(tl + tS + b * 128 + g * 64 + ch * 32, dhi, dlo);
       }
       tmem_st_wait();
       tc_fence_before();
