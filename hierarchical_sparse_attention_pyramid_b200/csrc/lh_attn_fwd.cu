@@ -5,16 +5,16 @@
 // One CTA owns two 128-row query tiles (A = 2c, B = 2c+1) of one (batch,
 // head) and streams the key/value tiles 0..2c+1 once for both (causal; each
 // tile's diagonal block is masked).  Warp roles:
-//   warps 0-7  softmax, both warpgroups on every tile (A, then B, of each
-//              key tile): thread (g, t) owns query row t (TMEM lane t) and
-//              keys [64g, 64g+64); it loads its 64 scores from TMEM once,
-//              exchanges the row max with the other group, keeps the running
-//              max and its partial row sum, rescales its half of O in TMEM
-//              when the max moves, and writes P back over the S columns it
-//              came from as a bf16 pair (per 32 keys: 16 columns of hi, 16 of
-//              lo), where the P V product reads it
-//   warp 8     TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
-//   warp 9     MMA issuer (the converged warp; one elected lane issues):
+//   warps 0-15 softmax, a warpgroup pair per query tile (warps 0-7 tile A,
+//              8-15 tile B, side by side): thread (g, t) of a pair owns query
+//              row t (TMEM lane t) and keys [64g, 64g+64); it loads its 64
+//              scores from TMEM once, exchanges the row max with the other
+//              group, keeps the running max and its partial row sum, rescales
+//              its half of O in TMEM when the max moves, and writes P back
+//              over the S columns it came from as a bf16 pair (per 32 keys: 16
+//              columns of hi, 16 of lo), where the P V product reads it
+//   warp 16    TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
+//   warp 17    MMA issuer (the converged warp; one elected lane issues):
 //              for each key tile, P_A V, then the next S_A = Q_A K^T, then
 //              P_B V and the next S_B, so the tensor core works on one tile
 //              while the other tile's softmax runs
@@ -33,7 +33,8 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kSoftmax = 256;
+constexpr int kSoftmax = 512;          // two warpgroup pairs, one per query tile
+constexpr int kPair = kSoftmax / 2;    // softmax threads of one query tile
 constexpr int kThreads = kSoftmax + 64;
 
 
@@ -44,8 +45,8 @@ struct FwdSmem {
   static constexpr int oQ = 0;              // Q_A, Q_B
   static constexpr int oK = oQ + 2 * kTile; // 2 stages
   static constexpr int oV = oK + 2 * kTile; // 2 stages
-  static constexpr int oXch = oV + 2 * kTile;  // softmax exchange: 4 x 128 maxima, 4 x 128 sums
-  static constexpr int oBar = oXch + 4096;
+  static constexpr int oXch = oV + 2 * kTile;  // softmax exchange, per tile: [2][2][128] maxima, [2][128] sums
+  static constexpr int oBar = oXch + 2 * 768 * 4;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -64,11 +65,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bV = bars + 3;       // [2]
   uint64_t* bKVfree = bars + 5;  // [2]
   uint64_t* bS = bars + 7;       // [2] tiles: S of the tile in TMEM (and its previous P V done)
-  uint64_t* bP = bars + 9;       // [2] tiles: P in TMEM, O rescaled (128 arrivals)
+  uint64_t* bP = bars + 9;       // [2] tiles: P in TMEM, O rescaled (one arrival per thread of the tile's pair)
   uint64_t* bO = bars + 11;      // [2] tiles: a P V product of the tile done
-  uint64_t* bX = bars + 13;      // [2] softmax exchange (256 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 132);
+  uint64_t* bX = bars + 13;      // [2 tiles][2] softmax exchange within a tile's warpgroup pair
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
@@ -87,20 +88,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bV[s], 1);
       mbar_init(&bKVfree[s], 1);
       mbar_init(&bS[s], 1);
-      mbar_init(&bP[s], kSoftmax);
+      mbar_init(&bP[s], kPair);
       mbar_init(&bO[s], 1);
-      mbar_init(&bX[s], kSoftmax);
+      mbar_init(&bX[s], kPair);
+      mbar_init(&bX[2 + s], kPair);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  if (warp == 17) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(smem + Lay::oV + st * Lay::kTile + ch * Lay::kChunk, &tmV, &bV[st], ch * 64, j * BN, bh);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ------------------------------------------------------------ MMA issuer
     {  // the whole warp; one elected lane issues each instruction
       constexpr uint32_t idQK = idesc_bf16(BM, BN, false, false);
@@ -180,134 +182,129 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // Both warpgroups work on every tile, tile A then tile B of each key
-    // tile: thread (g, t) owns query row t (TMEM lane t) and keys
-    // [64g, 64g+64) of the key tile, so two warps per sub-partition share the
-    // exponentials.  The row max is exchanged through shared memory (one
-    // shared-memory barrier per tile, a bounded wait); each group keeps its
-    // partial row sum, and both use the same running reference m, so the
-    // partial sums add at the end.
-    const int g = warp >> 2;
+    // Warpgroup pair x (warps 8x .. 8x+7) works on query tile x, so the two
+    // tiles' softmax passes run side by side.  Within a pair, thread (g, t)
+    // owns query row t (TMEM lane t) and keys [64g, 64g+64) of the key tile:
+    // it loads its 64 scores from TMEM once, exchanges the row max with the
+    // other group through shared memory (one barrier per key tile, a bounded
+    // wait), keeps the running max and its partial row sum, rescales its half
+    // of O when the max moves, and writes P back over the S columns it came
+    // from as a bf16 pair (per 32 keys: 16 columns of hi, 16 of lo), where
+    // the P V product reads it.  Both groups use the same running reference
+    // m, so the partial sums add at the end.
+    const int x = warp >> 3;
+    const int g = (warp >> 2) & 1;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    float* sXch = reinterpret_cast<float*>(smem + Lay::oXch);  // [2 parity][2 groups][128] row maxima, then [2 groups][2 tiles][128] sums
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float* sXch = reinterpret_cast<float*>(smem + Lay::oXch) + x * 768;  // [2 parity][2 groups][128] maxima, then [2 groups][128] sums
+    uint64_t* bXx = bX + 2 * x;
+    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int n_x = 0;  // exchanges so far: buffer n_x & 1 of sXch, barrier bX[n_x & 1]
-    // all 256 softmax threads have written their part of the exchange buffer
+    int n_x = 0;  // exchanges so far: buffer n_x & 1 of sXch, barrier bXx[n_x & 1]
+    // all 256 threads of the pair have written their part of the exchange buffer
     auto exchange = [&]() -> bool {
-      mbar_arrive(&bX[n_x & 1]);
-      const bool done = mbar_wait(&bX[n_x & 1], (n_x >> 1) & 1, abort_flag);
+      mbar_arrive(&bXx[n_x & 1]);
+      const bool done = mbar_wait(&bXx[n_x & 1], (n_x >> 1) & 1, abort_flag);
       ++n_x;
       return done;
     };
-    const int j_end = hasB ? last[1] : last[0];
-    for (int j = 0; ok && j <= j_end; ++j) {
-      for (int x = 0; x < 2; ++x) {
-        if (j > last[x]) continue;
-        const uint32_t ts = tl + x * 128 + g * 64, to = tl + 256 + x * D + g * (D / 2);
-        ok = __all_sync(0xffffffffu, mbar_wait(&bS[x], j & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        const bool diag = (j == last[x]);
-        uint32_t r[2][32];
-        tmem_ld32(ts, r[0]);
-        tmem_ld32(ts + 32, r[1]);
-        tmem_ld_wait();
-        // row max of the raw scores over this group's keys (the scale is
-        // positive); on the diagonal tile the keys after the row are masked
-        float mx = -INFINITY;
-        if (diag) {
-          const int lim = row - g * 64;
+    const uint32_t ts = tl + x * 128 + g * 64, to = tl + 256 + x * D + g * (D / 2);
+    for (int j = 0; ok && j <= last[x]; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bS[x], j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const bool diag = (j == last[x]);
+      uint32_t r[2][32];
+      tmem_ld32(ts, r[0]);
+      tmem_ld32(ts + 32, r[1]);
+      tmem_ld_wait();
+      // row max of the raw scores over this group's keys (the scale is
+      // positive); on the diagonal tile the keys after the row are masked
+      float mx = -INFINITY;
+      if (diag) {
+        const int lim = row - g * 64;
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (ch * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(r[ch][i]));
-        } else {
+          for (int i = 0; i < 32; ++i)
+            if (ch * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(r[ch][i]));
+      } else {
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[ch][i]), __uint_as_float(r[ch][i + 1]));
-        }
-        float* xch = sXch + (n_x & 1) * 256;
-        xch[g * 128 + row] = mx;
-        ok = __all_sync(0xffffffffu, exchange());
-        if (!ok) break;
-        mx = fmaxf(mx, xch[(1 - g) * 128 + row]);
-        // Lazy rescaling: the reference m_run moves only when the row max
-        // exceeds it by more than 8 (so every P stays <= 2^8); O and l share
-        // the reference, so the result is exact either way.
-        const float m_tile = mx * scale_log2;
-        const bool move = m_tile > m_run[x] + 8.f;
-        const float m_new = move ? m_tile : m_run[x];
-        const float alpha = move ? fast_exp2(m_run[x] - m_new) : 1.f;
-        // P = 2^(s*scale - m) as a bf16 pair written back over the chunk it
-        // came from: chunk ch (keys 32ch..32ch+31 of the group) holds hi in
-        // its first 16 columns and lo in its last 16, where P V reads them.
-        // Keys after the row (diagonal tile only) are masked: limit = row
-        // there and past every key elsewhere, so one code path serves both.
-        const int limit = diag ? row - g * 64 : 1 << 20;
-        const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
-        uint64_t rs2 = f2_pack(0.f, 0.f);
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t hi[16], lo[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float a, b;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][2 * q]), __uint_as_float(r[ch][2 * q + 1])), c2, nm2), a,
-                      b);
-            a = fast_exp2(a);
-            b = fast_exp2(b);
-            const int col = ch * 32 + 2 * q;
-            a = col > limit ? 0.f : a;
-            b = col + 1 > limit ? 0.f : b;
-            rs2 = f2_add(rs2, f2_pack(a, b));
-            split_bf16x2(a, b, hi[q], lo[q]);
-          }
-          tmem_st16(ts + ch * 32, hi);
-          tmem_st16(ts + ch * 32 + 16, lo);
-        }
-        float rsa, rsb;
-        f2_unpack(rs2, rsa, rsb);
-        const float rs = rsa + rsb;
-        // rescale this group's half of the O row; the previous P V of this
-        // tile is done (its completion preceded this S)
-        if (j >= 1 && __any_sync(0xffffffffu, move)) {
-#pragma unroll 1
-          for (int ch = 0; ch < D / 64; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(to + ch * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(to + ch * 32, o);
-          }
-        }
-        l_run[x] = l_run[x] * alpha + rs;
-        m_run[x] = m_new;
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bP[x]);
+          for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[ch][i]), __uint_as_float(r[ch][i + 1]));
       }
-    }
-    // row sums: the two groups' partial sums of each tile
-    if (ok) {
-      float* sL = sXch + 512;
-      sL[(g * 2 + 0) * 128 + row] = l_run[0];
-      sL[(g * 2 + 1) * 128 + row] = l_run[1];
+      float* xch = sXch + (n_x & 1) * 256;
+      xch[g * 128 + row] = mx;
       ok = __all_sync(0xffffffffu, exchange());
+      if (!ok) break;
+      mx = fmaxf(mx, xch[(1 - g) * 128 + row]);
+      // Lazy rescaling: the reference m_run moves only when the row max
+      // exceeds it by more than 8 (so every P stays <= 2^8); O and l share
+      // the reference, so the result is exact either way.
+      const float m_tile = mx * scale_log2;
+      const bool move = m_tile > m_run + 8.f;
+      const float m_new = move ? m_tile : m_run;
+      const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;
+      // P = 2^(s*scale - m) as a bf16 pair written back over the chunk it
+      // came from: chunk ch (keys 32ch..32ch+31 of the group) holds hi in
+      // its first 16 columns and lo in its last 16, where P V reads them.
+      // Keys after the row (diagonal tile only) are masked: limit = row there
+      // and past every key elsewhere, so one code path serves both.
+      const int limit = diag ? row - g * 64 : 1 << 20;
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
+      uint64_t rs2 = f2_pack(0.f, 0.f);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float a, b;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][2 * q]), __uint_as_float(r[ch][2 * q + 1])), c2, nm2), a, b);
+          a = fast_exp2(a);
+          b = fast_exp2(b);
+          const int col = ch * 32 + 2 * q;
+          a = col > limit ? 0.f : a;
+          b = col + 1 > limit ? 0.f : b;
+          rs2 = f2_add(rs2, f2_pack(a, b));
+          split_bf16x2(a, b, hi[q], lo[q]);
+        }
+        tmem_st16(ts + ch * 32, hi);
+        tmem_st16(ts + ch * 32 + 16, lo);
+      }
+      float rsa, rsb;
+      f2_unpack(rs2, rsa, rsb);
+      const float rs = rsa + rsb;
+      // rescale this group's half of the O row; the previous P V of this
+      // tile is done (its completion preceded this S)
+      if (j >= 1 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+        for (int ch = 0; ch < D / 64; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(to + ch * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(to + ch * 32, o);
+        }
+      }
+      l_run = l_run * alpha + rs;
+      m_run = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bP[x]);
     }
-    if (ok) {
-      const float* sL = sXch + 512;
-      for (int x = 0; x < (hasB ? 2 : 1); ++x) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bO[x], last[x] & 1, abort_flag))) break;
+    // row sums: the two groups' partial sums of the tile
+    if (ok && last[x] >= 0) {
+      float* sL = sXch + 512;
+      sL[g * 128 + row] = l_run;
+      ok = __all_sync(0xffffffffu, exchange());
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bO[x], last[x] & 1, abort_flag));
+      if (ok) {
         tc_fence_after();
-        const float l = l_run[x] + sL[((1 - g) * 2 + x) * 128 + row];
+        const float l = l_run + sL[(1 - g) * 128 + row];
         const float inv_l = 1.f / l;
         const int row_g = qtile[x] * BM + row;
-        const uint32_t to = tl + 256 + x * D + g * (D / 2);
 #pragma unroll 1
         for (int ch = 0; ch < D / 64; ++ch) {
           uint32_t o[32];
@@ -321,13 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
           }
         }
-        if (g == 0 && row_g < S) LSE[(int64_t)bh * S + row_g] = (m_run[x] + log2f(l)) * 0.69314718055994530942f;
+        if (g == 0 && row_g < S) LSE[(int64_t)bh * S + row_g] = (m_run + log2f(l)) * 0.69314718055994530942f;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
