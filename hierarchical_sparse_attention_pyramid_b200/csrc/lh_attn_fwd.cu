@@ -25,6 +25,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "lh_common.cuh"
 #include "sm100.cuh"
 
@@ -249,29 +251,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(s*scale - m) as a bf16 pair written back over the chunk it
       // came from: chunk ch (keys 32ch..32ch+31 of the group) holds hi in
       // its first 16 columns and lo in its last 16, where P V reads them.
-      // Keys after the row (diagonal tile only) are masked: limit = row there
-      // and past every key elsewhere, so one code path serves both.
-      const int limit = diag ? row - g * 64 : 1 << 20;
+      // Keys after the row are masked on the diagonal tile only.
       const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
       uint64_t rs2 = f2_pack(0.f, 0.f);
+      auto p_pass = [&](auto masked) {
+        const int limit = row - g * 64;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t hi[16], lo[16];
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float a, b;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][2 * q]), __uint_as_float(r[ch][2 * q + 1])), c2, nm2), a, b);
-          a = fast_exp2(a);
-          b = fast_exp2(b);
-          const int col = ch * 32 + 2 * q;
-          a = col > limit ? 0.f : a;
-          b = col + 1 > limit ? 0.f : b;
-          rs2 = f2_add(rs2, f2_pack(a, b));
-          split_bf16x2(a, b, hi[q], lo[q]);
+          for (int q = 0; q < 16; ++q) {
+            float a, b;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][2 * q]), __uint_as_float(r[ch][2 * q + 1])), c2, nm2), a,
+                      b);
+            a = fast_exp2(a);
+            b = fast_exp2(b);
+            if constexpr (decltype(masked)::value) {
+              const int col = ch * 32 + 2 * q;
+              a = col > limit ? 0.f : a;
+              b = col + 1 > limit ? 0.f : b;
+            }
+            rs2 = f2_add(rs2, f2_pack(a, b));
+            split_bf16x2(a, b, hi[q], lo[q]);
+          }
+          tmem_st16(ts + ch * 32, hi);
+          tmem_st16(ts + ch * 32 + 16, lo);
         }
-        tmem_st16(ts + ch * 32, hi);
-        tmem_st16(ts + ch * 32 + 16, lo);
-      }
+      };
+      if (diag) p_pass(std::true_type{});
+      else p_pass(std::false_type{});
       float rsa, rsb;
       f2_unpack(rs2, rsa, rsb);
       const float rs = rsa + rsb;
