@@ -36,6 +36,8 @@
 // and TMEM owner.
 #include <math.h>
 
+#include <type_traits>
+
 #include "lh_common.cuh"
 #include "sm100.cuh"
 
@@ -535,21 +537,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tl + tS + b * 128 + g * 64, r[0]);
       tmem_ld32(tl + tS + b * 128 + g * 64 + 32, r[1]);
       tmem_ld_wait();
-      // keys after the row are masked on the diagonal tile: limit = row there,
-      // past every key elsewhere
-      const int limit = j == qt ? t - g * 64 : 1 << 20;
+      // keys after the row are masked on the diagonal tile only
       float p[2][32];
+      auto p_pass = [&](auto masked) {
+        const int limit = t - g * 64;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pa, pb;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][e]), __uint_as_float(r[ch][e + 1])), c2, nl2), pa, pb);
-          pa = fast_exp2(pa);
-          pb = fast_exp2(pb);
-          p[ch][e] = ch * 32 + e > limit ? 0.f : pa;
-          p[ch][e + 1] = ch * 32 + e + 1 > limit ? 0.f : pb;
-        }
+          for (int e = 0; e < 32; e += 2) {
+            float pa, pb;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][e]), __uint_as_float(r[ch][e + 1])), c2, nl2), pa, pb);
+            pa = fast_exp2(pa);
+            pb = fast_exp2(pb);
+            if constexpr (decltype(masked)::value) {
+              pa = ch * 32 + e > limit ? 0.f : pa;
+              pb = ch * 32 + e + 1 > limit ? 0.f : pb;
+            }
+            p[ch][e] = pa;
+            p[ch][e + 1] = pb;
+          }
+      };
+      if (j == qt) p_pass(std::true_type{});
+      else p_pass(std::false_type{});
       ok = __all_sync(0xffffffffu, mbar_wait(bDP, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
