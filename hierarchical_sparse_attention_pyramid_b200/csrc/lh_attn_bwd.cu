@@ -267,23 +267,28 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
         tmem_ld32(tl + tS + g * 32, sr);
         tmem_ld_wait();
         uint32_t phi[16], plo[16];
+        // queries before the key are masked on the diagonal tile only
+        auto p_pass = [&](auto masked) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int qi = g * 32 + e;
-          const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
-          float pa, pb;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)),
-                    pa, pb);
-          pa = fast_exp2(pa);
-          pb = fast_exp2(pb);
-          if (diag) {
-            if (q0 + qi < kv_g) pa = 0.f;
-            if (q0 + qi + 1 < kv_g) pb = 0.f;
+          for (int e = 0; e < 32; e += 2) {
+            const int qi = g * 32 + e;
+            const float2 l2 = *reinterpret_cast<const float2*>(lse + qi);
+            float pa, pb;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, f2_pack(-l2.x, -l2.y)),
+                      pa, pb);
+            pa = fast_exp2(pa);
+            pb = fast_exp2(pb);
+            if constexpr (decltype(masked)::value) {
+              if (q0 + qi < kv_g) pa = 0.f;
+              if (q0 + qi + 1 < kv_g) pb = 0.f;
+            }
+            p[e] = pa;
+            p[e + 1] = pb;
+            split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
           }
-          p[e] = pa;
-          p[e + 1] = pb;
-          split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
-        }
+        };
+        if (diag) p_pass(std::true_type{});
+        else p_pass(std::false_type{});
         store_pair_chunk(tl + tS + g * 32, phi, plo);
       }
       tmem_st_wait();
