@@ -226,7 +226,7 @@ lh_status lh_pyramid_pool(const lh_config* cfg, const void* q, const void* k, co
   if (s != LH_OK) return s;
   LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v); LH_CHECK_PTR(norms);
   if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); }
-  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, (cudaStream_t)stream), "lh_pyramid_pool");
+  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, nullptr, (cudaStream_t)stream), "lh_pyramid_pool");
   return LH_OK;
 }
 
@@ -241,7 +241,7 @@ lh_status lh_pyramid_pool_from(const lh_config* cfg, int32_t first_level, const 
     return fail(LH_ERR_INVALID_ARG, "lh_pyramid_pool_from: first_level outside [1, max(1, L-1)]");
   LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v); LH_CHECK_PTR(norms);
   if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); }
-  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, (cudaStream_t)stream, first_level),
+  LH_CUDA(launch_pool(D, q, k, v, pyr_q, pyr_k, pyr_v, norms, nullptr, (cudaStream_t)stream, first_level),
           "lh_pyramid_pool_from");
   return LH_OK;
 }
@@ -384,7 +384,7 @@ lh_status lh_forward(const lh_config* cfg, const void* q, const void* k, const v
   float* os = reinterpret_cast<float*>(c + I.ctx_off_os);
   float* lse = reinterpret_cast<float*>(c + I.ctx_off_lse);
   const int first = I.first_level;
-  LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, st, first), "lh_forward: pool");
+  LH_CUDA(launch_pool(D, q, k, v, pq, pk, pv, norms, errw, st, first), "lh_forward: pool");
   LH_CUDA(launch_score_topk(D, norms, spyr, sel, errw, st), "lh_forward: score_topk");
   LH_CUDA(launch_gather(D, q, k, v, pq, pk, pv, sel, qs, ks, vs, seq_map, slot_of, errw, st, first),
           "lh_forward: gather");

@@ -104,8 +104,9 @@ __device__ __forceinline__ void load_f32(const float* src, float (&x)[VE]) {
 // launchers (host side, one per stage); all return cudaGetLastError()
 // ---------------------------------------------------------------------------
 // levels below first_level are not written (their sums still carry upward)
+// errw may be null (no error word): a bounded wait that runs out is then not reported
 cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void* v, void* pq, void* pk, void* pv,
-                        float* norms, cudaStream_t st, int first_level = 1);
+                        float* norms, int* errw, cudaStream_t st, int first_level = 1);
 cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, int32_t* sel, int* errw,
                               cudaStream_t st);
 // kept entries of levels 1 .. first_level-1 are averaged from level 0 here

@@ -9,6 +9,7 @@
 // Both kernels are HBM streams: one warp walks a contiguous run of rows of
 // one head and one of Q, K, V, so every load or store instruction of the warp
 // touches whole rows.
+#include <algorithm>
 #include <type_traits>
 
 #include "lh_common.cuh"
@@ -18,16 +19,25 @@ namespace lh {
 namespace {
 using namespace sm100;
 
-constexpr int kWarps = 8;  // warps per block
+constexpr int kWarps = 8;  // warps per block (pool adjoint)
 constexpr unsigned kFull = 0xffffffffu;
+// pooling: one CTA per SM of kPoolWarps warps, each with a ring of kStages
+// shared-memory stages of kStageBytes (192 KB per CTA).  Measured on the
+// 512K-token layer (16 heads, d = 128, bf16): the pass is bound by the warps'
+// own summing work below 16 warps per SM (4 warps: 3.29 ms, 8: 1.83, 12: 1.46,
+// 16: 1.133) and by DRAM above (24 warps with 2 stages: 1.122 ms)
+constexpr int kPoolWarps = 24;
+constexpr int kStages = 2;
+constexpr int kStageBytes = 4096;
 
 struct PoolArgs {
   const void* x[3];
   void* pyr[3];
   float* norms;  // [2][BH][N]
+  int* errw;     // error word, or null
   int64_t BH, N, upper_entries;
   int64_t upper_off[LH_MAX_LEVELS];
-  int64_t tasks_per_head;
+  int64_t tasks_per_head, tasks;  // tasks = 3 * BH * tasks_per_head
   int task_rows, log2p, first_level;
 };
 
@@ -62,28 +72,81 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[U], int lane) {
   return t;
 }
 
-// One warp walks task_rows consecutive rows of one head of one of Q, K, V.
+// One warp walks whole tasks: task_rows consecutive rows of one head of one
+// of Q, K, V (a whole number of top-level blocks, so every level's sums start
+// and end inside a task).  The grid is one CTA per SM; warp w takes tasks w,
+// w + W, w + 2W, ... (W = warps in the grid).  The rows reach shared memory
+// through a per-warp ring of kStages bulk copies of kStageBytes, issued by
+// lane 0 kStages stages ahead of the rows being summed, so about
+// kPoolWarps * kStages * kStageBytes bytes per SM are in flight at all times.
 // Lane l holds channels [l*VE, l*VE+VE) of every row, so the pooled sums need
 // no cross-lane work; only the norms of Q and K rows are reduced across lanes.
 template <typename T, int D, int NL>
-__global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
+__global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
   constexpr int VE = D / 32;
-  constexpr int U = 8;  // rows loaded per batch (two batches in flight)
+  constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int SR = kStageBytes / ROWB;  // rows per stage
+  constexpr int U = 8;                    // rows summed per batch
+  static_assert(SR % U == 0, "stage rows");
   using Raw = typename RawVec<sizeof(T) * VE>::type;
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int tensor = (int)(wid % 3);
-  const int64_t rest = wid / 3;
-  const int64_t bh = rest / a.tasks_per_head;
-  if (bh >= a.BH) return;
-  const int64_t row0 = (rest % a.tasks_per_head) * a.task_rows;
-  const int rows = (int)min((int64_t)a.task_rows, a.N - row0);
+  extern __shared__ __align__(128) uint8_t pool_ring[];
+  __shared__ __align__(8) uint64_t pool_bars[kPoolWarps][kStages];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint8_t* ring = pool_ring + warp * (kStages * kStageBytes);
+  uint64_t* bar = pool_bars[warp];
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const int64_t nw = (int64_t)gridDim.x * kPoolWarps;
+  const int64_t gw = (int64_t)blockIdx.x * kPoolWarps + warp;
   const int log2p = a.log2p;
-  const Raw* src = reinterpret_cast<const Raw*>(static_cast<const T*>(a.x[tensor]) + (bh * a.N + row0) * D) + lane;
-  T* dst = static_cast<T*>(a.pyr[tensor]) + bh * a.upper_entries * D + lane * VE;
-  const bool want_norm = tensor < 2;
-  float* norm_out = a.norms + ((int64_t)tensor * a.BH + bh) * a.N + row0;
   const int rid = scatter_row<U>(lane);
+
+  // task t: tensor t % 3, head (t / 3) / tasks_per_head, rows from row0
+  // (task counts fit 32 bits: the host checks)
+  const uint32_t tph = (uint32_t)a.tasks_per_head, ntasks = (uint32_t)a.tasks;
+  auto task_at = [&](uint32_t t, int& tensor, int64_t& bh, int64_t& row0) {
+    tensor = (int)(t % 3u);
+    const uint32_t rest = t / 3u;
+    bh = rest / tph;
+    row0 = (int64_t)(rest % tph) * a.task_rows;
+    return (int)min((int64_t)a.task_rows, a.N - row0);
+  };
+
+  // producer cursor, kept by every lane (lane 0 alone issues the copies):
+  // task pt, its first source byte and row count, row pr within it
+  uint32_t pt = (uint32_t)gw;
+  int pr = 0, prows = 0;
+  const uint8_t* psrc = nullptr;
+  auto producer_task = [&]() {
+    if (pt >= ntasks) return;
+    int tensor;
+    int64_t bh, row0;
+    prows = task_at(pt, tensor, bh, row0);
+    psrc = static_cast<const uint8_t*>(a.x[tensor]) + (bh * a.N + row0) * ROWB;
+  };
+  producer_task();
+  uint32_t pending = 0;  // slots with a copy issued and not yet consumed
+  auto issue = [&](int slot) {
+    if (pt >= ntasks) return;
+    const int n = min(SR, prows - pr);
+    if (lane == 0) {
+      mbar_expect_tx(&bar[slot], (uint32_t)(n * ROWB));
+      bulk_load(ring + slot * kStageBytes, psrc + (int64_t)pr * ROWB, (uint32_t)(n * ROWB), &bar[slot]);
+    }
+    pending |= 1u << slot;
+    pr += SR;
+    if (pr >= prows) {
+      pr = 0;
+      pt += (uint32_t)nw;
+      producer_task();
+    }
+  };
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) issue(s);
 
   // bf16 rows are widened and summed as fp32 pairs (f32x2 arithmetic): one
   // packed fma for the squares and one packed add per two channels
@@ -91,109 +154,127 @@ __global__ void __launch_bounds__(kWarps * 32, 2) pool_kernel(PoolArgs a) {
   constexpr int NP = kPacked ? VE / 2 : 1;
   float acc[NL + 1][kPacked ? 1 : VE];
   uint64_t acc2[NL + 1][NP];
-#pragma unroll
-  for (int l = 0; l <= NL; ++l) {
-#pragma unroll
-    for (int i = 0; i < (kPacked ? 1 : VE); ++i) acc[l][i] = 0.f;
-#pragma unroll
-    for (int i = 0; i < NP; ++i) acc2[l][i] = 0ull;
-  }
 
-  auto load = [&](Raw (&x)[U], int r0) {
+  uint32_t phase = 0;
+  int slot = 0;
+  for (uint32_t t = (uint32_t)gw; t < ntasks; t += (uint32_t)nw) {
+    int tensor;
+    int64_t bh, row0;
+    const int rows = task_at(t, tensor, bh, row0);
+    T* dst = static_cast<T*>(a.pyr[tensor]) + bh * a.upper_entries * D + lane * VE;
+    const bool want_norm = tensor < 2;
+    float* norm_out = a.norms + ((int64_t)tensor * a.BH + bh) * a.N + row0;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (r0 + u < rows) x[u] = __ldg(src + (int64_t)(r0 + u) * (D / VE));
-      else x[u] = Raw{};
+    for (int l = 0; l <= NL; ++l) {
+#pragma unroll
+      for (int i = 0; i < (kPacked ? 1 : VE); ++i) acc[l][i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < NP; ++i) acc2[l][i] = 0ull;
     }
-  };
-  auto process = [&](const Raw (&x)[U], int r0) {
-    float sq[U];
+
+    auto process = [&](const Raw (&x)[U], int r0) {
+      float sq[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if constexpr (kPacked) {
-        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&x[u]);  // channels 2i, 2i+1 in word i
-        uint64_t q2 = 0ull;
+      for (int u = 0; u < U; ++u) {
+        if constexpr (kPacked) {
+          const uint32_t* wd = reinterpret_cast<const uint32_t*>(&x[u]);  // channels 2i, 2i+1 in word i
+          uint64_t q2 = 0ull;
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          const uint64_t v2 = f2_pack(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xffff0000u));
-          q2 = f2_fma(v2, v2, q2);
-          if constexpr (NL > 1) acc2[1][i] = f2_add(acc2[1][i], v2);
+          for (int i = 0; i < NP; ++i) {
+            const uint64_t v2 = f2_pack(__uint_as_float(wd[i] << 16), __uint_as_float(wd[i] & 0xffff0000u));
+            q2 = f2_fma(v2, v2, q2);
+            if constexpr (NL > 1) acc2[1][i] = f2_add(acc2[1][i], v2);
+          }
+          float qa, qb;
+          f2_unpack(q2, qa, qb);
+          sq[u] = qa + qb;
+        } else {
+          const T* e = reinterpret_cast<const T*>(&x[u]);
+          float v[VE];
+#pragma unroll
+          for (int i = 0; i < VE; ++i) v[i] = Elem<T>::to_f(e[i]);
+          float q = 0.f;
+#pragma unroll
+          for (int i = 0; i < VE; ++i) q = fmaf(v[i], v[i], q);
+          sq[u] = q;
+          if constexpr (NL > 1) {
+#pragma unroll
+            for (int i = 0; i < VE; ++i) acc[1][i] += v[i];
+          }
         }
-        float qa, qb;
-        f2_unpack(q2, qa, qb);
-        sq[u] = qa + qb;
-      } else {
-        const T* e = reinterpret_cast<const T*>(&x[u]);
-        float v[VE];
-#pragma unroll
-        for (int i = 0; i < VE; ++i) v[i] = Elem<T>::to_f(e[i]);
-        float q = 0.f;
-#pragma unroll
-        for (int i = 0; i < VE; ++i) q = fmaf(v[i], v[i], q);
-        sq[u] = q;
         if constexpr (NL > 1) {
+          const int done = r0 + u + 1;  // rows of this task consumed
+          if (done <= rows && (done & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
-          for (int i = 0; i < VE; ++i) acc[1][i] += v[i];
-        }
-      }
-      if constexpr (NL > 1) {
-        const int done = r0 + u + 1;  // rows of this task consumed
-        if (done <= rows && (done & ((1 << log2p) - 1)) == 0) {
+            for (int l = 1; l < NL; ++l) {
+              if ((done & ((1 << (l * log2p)) - 1)) != 0) break;
+              const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
+              const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
+              if constexpr (kPacked) {
+                const uint64_t inv2 = f2_pack(inv, inv);
+                if (l >= a.first_level) {
+                  Raw o;
+                  uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-          for (int l = 1; l < NL; ++l) {
-            if ((done & ((1 << (l * log2p)) - 1)) != 0) break;
-            const float inv = __int_as_float((127 - l * log2p) << 23);  // 2^(-l log2p), exact
-            const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
-            if constexpr (kPacked) {
-              const uint64_t inv2 = f2_pack(inv, inv);
-              if (l >= a.first_level) {
-                Raw o;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+                  for (int i = 0; i < NP; ++i) {
+                    float ma, mb;
+                    f2_unpack(f2_mul(acc2[l][i], inv2), ma, mb);
+                    ow[i] = pack_bf16x2(ma, mb);
+                  }
+                  *reinterpret_cast<Raw*>(dst + (a.upper_off[l] + e_idx) * D) = o;
+                }
 #pragma unroll
                 for (int i = 0; i < NP; ++i) {
-                  float ma, mb;
-                  f2_unpack(f2_mul(acc2[l][i], inv2), ma, mb);
-                  ow[i] = pack_bf16x2(ma, mb);
+                  acc2[l + 1][i] = f2_add(acc2[l + 1][i], acc2[l][i]);
+                  acc2[l][i] = 0ull;
                 }
-                *reinterpret_cast<Raw*>(dst + (a.upper_off[l] + e_idx) * D) = o;
-              }
+              } else {
+                float m[VE];
 #pragma unroll
-              for (int i = 0; i < NP; ++i) {
-                acc2[l + 1][i] = f2_add(acc2[l + 1][i], acc2[l][i]);
-                acc2[l][i] = 0ull;
-              }
-            } else {
-              float m[VE];
+                for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
+                if (l >= a.first_level) store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
 #pragma unroll
-              for (int i = 0; i < VE; ++i) m[i] = acc[l][i] * inv;
-              if (l >= a.first_level) store_vec<T, VE>(dst + (a.upper_off[l] + e_idx) * D, m);
-#pragma unroll
-              for (int i = 0; i < VE; ++i) {
-                acc[l + 1][i] += acc[l][i];
-                acc[l][i] = 0.f;
+                for (int i = 0; i < VE; ++i) {
+                  acc[l + 1][i] += acc[l][i];
+                  acc[l][i] = 0.f;
+                }
               }
             }
           }
         }
       }
-    }
-    if (want_norm) {
-      const float tot = reduce_scatter<U>(sq, lane);
-      const int r = r0 + rid;
-      if ((lane & (32 / U - 1)) == 0 && r < rows) norm_out[r] = sqrtf(tot);
-    }
-  };
+      if (want_norm) {
+        const float tot = reduce_scatter<U>(sq, lane);
+        const int r = r0 + rid;
+        if ((lane & (32 / U - 1)) == 0 && r < rows) norm_out[r] = sqrtf(tot);
+      }
+    };
 
-  // two batches in flight: the loads of the next batch are issued before the
-  // current one is processed (one copy of the processing code, so the loop
-  // body stays small in the instruction cache)
-  Raw cur[U], nxt[U];
-  load(cur, 0);
-  for (int r0 = 0; r0 < rows; r0 += U) {
-    if (r0 + U < rows) load(nxt, r0 + U);
-    process(cur, r0);
+    for (int r0 = 0; r0 < rows; r0 += SR) {
+      if (!mbar_wait_bounded_warp(&bar[slot], (phase >> slot) & 1u)) {
+        // a copy never landed: report it, give the other copies in flight a
+        // bounded time to land (the CTA must not exit with copies pending
+        // into its shared memory) and leave
+        report_error(a.errw, ERRW_TIMEOUT);
+#pragma unroll 1
+        for (int s = 0; s < kStages; ++s)
+          if (s != slot && (pending >> s & 1u)) mbar_wait_bounded_warp(&bar[s], (phase >> s) & 1u);
+        return;
+      }
+      const Raw* stage = reinterpret_cast<const Raw*>(ring + slot * kStageBytes) + lane;
+#pragma unroll 1
+      for (int b = 0; b < SR; b += U) {
+        Raw x[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+        for (int u = 0; u < U; ++u) x[u] = (r0 + b + u < rows) ? stage[(b + u) * (ROWB / (int)sizeof(Raw))] : Raw{};
+        process(x, r0 + b);
+      }
+      __syncwarp();  // every lane has read the stage before it is refilled
+      pending &= ~(1u << slot);
+      phase ^= 1u << slot;
+      issue(slot);
+      slot = slot + 1 == kStages ? 0 : slot + 1;
+    }
   }
 }
 
@@ -287,16 +368,31 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
   }
 }
 
+// persistent grid: as many CTAs as fit on the GPU at once, fewer for small inputs
+template <typename T, int D, int NL>
+cudaError_t pool_launch(const PoolArgs& a, cudaStream_t st) {
+  constexpr int smem = kPoolWarps * kStages * kStageBytes;
+  cudaError_t e = cudaFuncSetAttribute(pool_kernel<T, D, NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int dev = 0, sms = 0, per_sm = 0;
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_kernel<T, D, NL>, kPoolWarps * 32, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = std::min<int64_t>((int64_t)sms * std::max(per_sm, 1), (a.tasks + kPoolWarps - 1) / kPoolWarps);
+  pool_kernel<T, D, NL><<<(unsigned)blocks, kPoolWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
-cudaError_t pool_dispatch_L(int L, const PoolArgs& a, int64_t blocks, cudaStream_t st) {
+cudaError_t pool_dispatch_L(int L, const PoolArgs& a, cudaStream_t st) {
   switch (L) {
 #define LH_CASE(n) \
-  case n: pool_kernel<T, D, n><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a); break;
+  case n: return pool_launch<T, D, n>(a, st);
     LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
 #undef LH_CASE
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 template <typename T, int D>
@@ -321,24 +417,25 @@ int task_rows_for(const Dims& D, int min_rows) {
 }  // namespace
 
 cudaError_t launch_pool(const Dims& D, const void* q, const void* k, const void* v, void* pq, void* pk, void* pv,
-                        float* norms, cudaStream_t st, int first_level) {
+                        float* norms, int* errw, cudaStream_t st, int first_level) {
   PoolArgs a{};
   a.x[0] = q; a.x[1] = k; a.x[2] = v;
   a.pyr[0] = pq; a.pyr[1] = pk; a.pyr[2] = pv;
   a.norms = norms;
+  a.errw = errw;
   a.BH = D.BH; a.N = D.N; a.upper_entries = D.upper_entries;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) a.upper_off[l] = D.upper_off[l];
-  a.task_rows = task_rows_for(D, 512);
+  a.task_rows = task_rows_for(D, 64);
   a.tasks_per_head = (D.N + a.task_rows - 1) / a.task_rows;
+  a.tasks = 3 * D.BH * a.tasks_per_head;
+  if (a.tasks >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;  // task ids are 32-bit in the kernel
   a.log2p = D.log2p;
   a.first_level = first_level;
-  const int64_t warps = 3 * D.BH * a.tasks_per_head;
-  const int64_t blocks = (warps + kWarps - 1) / kWarps;
   if (D.dtype == LH_BF16) {
-    return D.d == 128 ? pool_dispatch_L<__nv_bfloat16, 128>(D.L, a, blocks, st)
-                      : pool_dispatch_L<__nv_bfloat16, 64>(D.L, a, blocks, st);
+    return D.d == 128 ? pool_dispatch_L<__nv_bfloat16, 128>(D.L, a, st)
+                      : pool_dispatch_L<__nv_bfloat16, 64>(D.L, a, st);
   }
-  return D.d == 128 ? pool_dispatch_L<float, 128>(D.L, a, blocks, st) : pool_dispatch_L<float, 64>(D.L, a, blocks, st);
+  return D.d == 128 ? pool_dispatch_L<float, 128>(D.L, a, st) : pool_dispatch_L<float, 64>(D.L, a, st);
 }
 
 cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dks, const float* dvs,

@@ -138,7 +138,11 @@ lh_status lh_plan(const lh_config *cfg, lh_plan_info *info);
  *      at row upper_off[l]; entry i is the mean of tokens [i p^l, (i+1) p^l),
  *      summed in fp32 and rounded once.
  *      norms [2][BH][N] fp32: plane 0 = ||Q_t||_2, plane 1 = ||K_t||_2.
- * With L = 1 the pyramid buffers are not touched (may be NULL). */
+ * With L = 1 the pyramid buffers are not touched (may be NULL).
+ * The rows reach shared memory by bulk copies whose waits are bounded; this
+ * call has no workspace, so a wait that runs out (a copy that never lands)
+ * leaves the outputs incomplete without a status (lh_forward reports it
+ * through its error word). */
 lh_status lh_pyramid_pool(const lh_config *cfg, const void *q, const void *k, const void *v, void *pyr_q,
                           void *pyr_k, void *pyr_v, float *norms, lh_stream_t stream);
 
