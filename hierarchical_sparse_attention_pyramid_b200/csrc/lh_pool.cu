@@ -104,6 +104,13 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
   const int64_t gw = (int64_t)blockIdx.x * kPoolWarps + warp;
   const int log2p = a.log2p;
   const int rid = scatter_row<U>(lane);
+  // rows u of an aligned batch of U after which a level-1 block ends: every
+  // p-th row when p <= U, else the last row (when the batch ends a block)
+  constexpr int kLog2U = 3;
+  static_assert(U == 1 << kLog2U, "batch");
+  uint32_t bmask = 1u << (U - 1);
+  if (log2p < kLog2U)
+    for (int u = (1 << log2p) - 1; u < U; u += 1 << log2p) bmask |= 1u << u;
 
   // task t: tensor t % 3, head (t / 3) / tasks_per_head, rows from row0
   // (task counts fit 32 bits: the host checks)
@@ -173,6 +180,13 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
     }
 
     auto process = [&](const Raw (&x)[U], int r0) {
+      // bit u: a level-1 block of this task ends after row r0 + u (blocks are
+      // aligned to the task; rows past the task's end never end one)
+      uint32_t bnd = 0;
+      if constexpr (NL > 1) {
+        bnd = (log2p <= kLog2U || ((r0 + U) & ((1 << log2p) - 1)) == 0) ? bmask : 0u;
+        if (rows - r0 < U) bnd &= (1u << (rows - r0)) - 1u;
+      }
       float sq[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
         }
         if constexpr (NL > 1) {
           const int done = r0 + u + 1;  // rows of this task consumed
-          if (done <= rows && (done & ((1 << log2p) - 1)) == 0) {
+          if (bnd >> u & 1u) {
 #pragma unroll
             for (int l = 1; l < NL; ++l) {
               if ((done & ((1 << (l * log2p)) - 1)) != 0) break;
@@ -261,12 +275,16 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
           if (s != slot && (pending >> s & 1u)) mbar_wait_bounded_warp(&bar[s], (phase >> s) & 1u);
         return;
       }
+      // rows of a stage past the task's end hold stale bytes: their sums are
+      // never written (no block ends there, their norms are not stored) and
+      // the task's sums are reset before the next task
       const Raw* stage = reinterpret_cast<const Raw*>(ring + slot * kStageBytes) + lane;
+      const int stage_rows = min(SR, rows - r0);
 #pragma unroll 1
-      for (int b = 0; b < SR; b += U) {
+      for (int b = 0; b < stage_rows; b += U) {
         Raw x[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) x[u] = (r0 + b + u < rows) ? stage[(b + u) * (ROWB / (int)sizeof(Raw))] : Raw{};
+        for (int u = 0; u < U; ++u) x[u] = stage[(b + u) * (ROWB / (int)sizeof(Raw))];
         process(x, r0 + b);
       }
       __syncwarp();  // every lane has read the stage before it is refilled
