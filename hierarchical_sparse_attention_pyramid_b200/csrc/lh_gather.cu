@@ -184,10 +184,14 @@ struct RowLayout {
   static_assert(R == 1 || R == 2, "layout");
 };
 
-// Rows are visited in instruction steps u = 0, R, 2R, ...; step u covers rows
-// u - (R-1) .. u.  With R = 2 the pair (u-1, u) has (j+1) in {u, u+1}, u even,
-// so both rows take the same entry at every level >= 1 and the refresh of the
-// cached contribution is uniform over the warp.
+// A warp runs R tasks side by side, one per group of LPR lanes (R = 2 for a
+// bf16 row of 128: two half-warps).  Task t of a head covers the rows
+// j = t*task_rows - 1 ... (t+1)*task_rows - 2 (keys j+1 from t*task_rows), one
+// row per step, so a step of the warp stores one row of each task.  Tasks
+// start on top-level boundaries, so every task meets its level boundaries at
+// the same steps: the refreshes of the cached contributions are uniform over
+// the warp while their lookups (slot index, then the Os row) go out for all
+// of the warp's tasks at once.
 template <typename T, int D, int NL>
 __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a) {
   using Lay = RowLayout<T, D>;
@@ -195,22 +199,27 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
   const int lane = threadIdx.x & 31;
   const int lr = lane / LPR, cv = lane % LPR;
   const int64_t wid = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int64_t bh = wid / a.tasks_per_head;
-  if (bh >= a.BH) return;
-  const int64_t u0 = (wid % a.tasks_per_head) * a.task_rows;
-  const int steps = (int)min((int64_t)a.task_rows, a.N + R - 1 - u0);
+  const int64_t ntasks = a.BH * a.tasks_per_head;
+  if (wid * R >= ntasks) return;
+  const int64_t task = wid * R + lr;  // this lane group's task
+  const bool active = task < ntasks;
+  const int64_t bh = active ? task / a.tasks_per_head : 0;
+  const int u0 = active ? (int)(task % a.tasks_per_head) * a.task_rows : 0;  // rows within a head fit 32 bits
+  const int N = (int)a.N;
   const int log2p = a.log2p;
   const int32_t* so = a.slot_of + bh * a.pyr_entries;
   const float* os = a.os + bh * a.S * D + cv * VE;
   T* out = static_cast<T*>(a.y) + bh * a.N * D + cv * VE;
 
-  // contribution of level 1, refreshed when the level-1 entry changes, and the
-  // summed contribution of levels >= 2, refreshed when the level-2 entry does
+  // contribution of level 1, refreshed at level-1 boundaries, and the summed
+  // contribution of levels >= 2, refreshed at level-2 boundaries
   float up1[VE], high[VE];
 #pragma unroll
   for (int c = 0; c < VE; ++c) up1[c] = high[c] = 0.f;
-  auto contribution = [&](int l, int64_t i, float (&acc)[VE]) {
-    const int s = i >= 0 ? so[a.level_off[l] + i] : -1;
+  // live: a row of this task inside the head (keys past N would index past
+  // the level tables); i < 0 is the part of a level before its first entry
+  auto contribution = [&](bool live, int l, int i, float (&acc)[VE]) {
+    const int s = (live && i >= 0) ? so[a.level_off[l] + i] : -1;
     if (s >= 0) {
       float v[VE];
       load_f32<VE>(os + (int64_t)s * D, v);
@@ -218,36 +227,32 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
       for (int c = 0; c < VE; ++c) acc[c] += v[c];
     }
   };
-  int64_t cur1 = -2, cur2 = -2;  // level-1 and level-2 entries of the previous step
+  constexpr int SW = 32 / R;  // level-0 slots fetched per lane group at a time
   int s0w = -1;
-  for (int r = 0; r < steps; r += R) {
-    const int64_t u = u0 + r;
-    const int64_t j = u - (R - 1) + lr;  // this lane's row
-    if ((r & 31) == 0) {
-      const int64_t jw = u - (R - 1) + lane;
-      s0w = (jw >= 0 && jw < a.N && r + lane < steps) ? so[a.level_off[0] + jw] : -1;
+  for (int r = 0; r < a.task_rows; ++r) {
+    const int key = u0 + r;  // j + 1
+    const int j = key - 1;
+    const bool live = active && j < N;
+    if (r % SW == 0) {
+      const int jw = j + cv % SW;
+      s0w = (active && jw >= 0 && jw < N) ? so[a.level_off[0] + jw] : -1;
     }
     if constexpr (NL > 1) {
-      const int64_t key = (R == 2) ? u : u + 1;  // (j+1) rounded down to the step, same for both rows
-      const int64_t i1 = (key >> log2p) - 1;
-      if (i1 != cur1) {
-        cur1 = i1;
+      if ((r & ((1 << log2p) - 1)) == 0) {
 #pragma unroll
         for (int c = 0; c < VE; ++c) up1[c] = 0.f;
-        contribution(1, i1, up1);
+        contribution(live, 1, (key >> log2p) - 1, up1);
         if constexpr (NL > 2) {
-          const int64_t i2 = (key >> (2 * log2p)) - 1;
-          if (i2 != cur2) {
-            cur2 = i2;
+          if ((r & ((1 << (2 * log2p)) - 1)) == 0) {
 #pragma unroll
             for (int c = 0; c < VE; ++c) high[c] = 0.f;
 #pragma unroll
-            for (int l = NL - 1; l >= 2; --l) contribution(l, (key >> (l * log2p)) - 1, high);
+            for (int l = NL - 1; l >= 2; --l) contribution(live, l, (key >> (l * log2p)) - 1, high);
           }
         }
       }
     }
-    const int s0 = __shfl_sync(kFull, s0w, (r & 31) + lr);
+    const int s0 = __shfl_sync(kFull, s0w, lr * LPR + r % SW);
     float y[VE];
 #pragma unroll
     for (int c = 0; c < VE; ++c) y[c] = up1[c] + high[c];
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 #pragma unroll
       for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
     }
-    if (j >= 0 && j < a.N) store_vec<T, VE>(out + j * D, y);
+    if (live && j >= 0) store_vec<T, VE>(out + (int64_t)j * D, y);
   }
 }
 
@@ -341,7 +346,9 @@ __global__ void __launch_bounds__(kSadjWarps * 32) scatter_adjoint_kernel(Scatte
 }
 
 template <typename T, int D>
-cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t blocks, cudaStream_t st) {
+cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaStream_t st) {
+  constexpr int R = RowLayout<T, D>::R;  // tasks per warp
+  const int64_t blocks = ((tasks + R - 1) / R + kWarps - 1) / kWarps;
   switch (L) {
 #define LH_CASE(n) \
   case n: scatter_back_kernel<T, D, n><<<(unsigned)blocks, kWarps * 32, 0, st>>>(a); break;
@@ -406,13 +413,13 @@ cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* s
   a.task_rows = (int)(ptop > 64 ? ptop : 64);
   a.tasks_per_head = (D.N + 1 + a.task_rows - 1) / a.task_rows;  // steps cover rows -1 .. N-1
   a.log2p = D.log2p;
-  const int64_t blocks = (D.BH * a.tasks_per_head + kWarps - 1) / kWarps;
+  const int64_t tasks = D.BH * a.tasks_per_head;
   if (D.dtype == LH_BF16) {
-    return D.d == 128 ? scatter_dispatch_L<__nv_bfloat16, 128>(D.L, a, blocks, st)
-                      : scatter_dispatch_L<__nv_bfloat16, 64>(D.L, a, blocks, st);
+    return D.d == 128 ? scatter_dispatch_L<__nv_bfloat16, 128>(D.L, a, tasks, st)
+                      : scatter_dispatch_L<__nv_bfloat16, 64>(D.L, a, tasks, st);
   }
-  return D.d == 128 ? scatter_dispatch_L<float, 128>(D.L, a, blocks, st)
-                    : scatter_dispatch_L<float, 64>(D.L, a, blocks, st);
+  return D.d == 128 ? scatter_dispatch_L<float, 128>(D.L, a, tasks, st)
+                    : scatter_dispatch_L<float, 64>(D.L, a, tasks, st);
 }
 
 cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
