@@ -21,6 +21,8 @@ SMALL = {
         synth.WORKLOADS["tiny_4k_fp32"],
         Workload("chunked_lognorm", 1, 2, 8192, 128, 3, 4, 96, "bf16", "qk_sum", "lognormal_token", 11, chunk=512),
         Workload("ragged", 1, 2, 1000, 128, 3, 2, 37, "bf16", "qk_sum", "iid", 12, chunk=64),
+        # N not a multiple of the pool's 8-row batches or 16-row stages, with level-1 block ends in the last stage
+        Workload("odd_rows_p2", 1, 1, 1002, 64, 2, 2, 37, "bf16", "qk_sum", "iid", 21, chunk=64),
         Workload("deep_p4", 1, 1, 8192, 128, 6, 4, 5, "bf16", "qk_sum", "outlier_tokens", 13),
         Workload("keep_all_kscore", 2, 1, 512, 64, 3, 2, 1000, "bf16", "k", "iid", 14),
         Workload("dense_L1", 1, 2, 700, 64, 1, 2, 1, "bf16", "qk_sum", "iid", 15),
