@@ -178,13 +178,14 @@ def pool_adjoint(layer: Layer, dqs, dks, dvs, slot_of):
 def kernels_per_step(layer: Layer) -> int:
     """liblh kernel launches of one lh_forward + lh_backward (memsets excluded):
     pool, score pyramid (one launch per 11/log2(p) levels), top-k, gather,
-    attention forward, scatter-back; scatter adjoint, attention backward,
-    pool adjoint."""
+    attention forward, scatter-back; scatter adjoint, attention backward (two
+    kernels: dK/dV and dQ), pool adjoint.  With L = 1 there is no selection
+    (no score pyramid or top-k)."""
     if layer.L == 1:
-        return 7
+        return 8
     log2p = layer.p.bit_length() - 1
     per_launch = 11 // log2p
-    return 8 + -(-(layer.L - 1) // per_launch)
+    return 9 + -(-(layer.L - 1) // per_launch)
 
 
 class Buffers:

@@ -10,6 +10,7 @@ import subprocess
 import pytest
 
 from hierarchical_sparse_attention_pyramid_b200 import _lib, plan, Layer
+from hierarchical_sparse_attention_pyramid_b200.api import kernels_per_step
 from hierarchical_sparse_attention_pyramid_b200.synth import WORKLOADS, Workload
 from oracle import lighthouse_oracle as lo
 
@@ -175,3 +176,13 @@ def test_pisa_calls_reject_bad_pointers_before_any_launch(lib):
     assert lib.lh_pisa_pool_keys(ctypes.byref(cfg), odd, odd, None) == 1
     assert lib.lh_pisa_select(ctypes.byref(cfg), None, None, None, None, None, None, None) == 1
     assert lib.lh_pisa_plan(None, None) == 1
+
+
+@pytest.mark.parametrize("L,p,want", [(5, 4, 10), (1, 2, 8), (3, 2, 10), (8, 2, 10), (7, 4, 11), (3, 8, 10)])
+def test_kernels_per_step(L, p, want):
+    """bench.py's gpu_launches claim: one pool, ceil((L-1) / (11 // log2 p))
+    score-pyramid launches, one top-k, gather, attention forward and
+    scatter-back; scatter adjoint, the two attention-backward kernels and the
+    pool adjoint (no selection kernels at L = 1).  The 512K-token launch list
+    under profiles/ shows the 10 of (L, p) = (5, 4) per step."""
+    assert kernels_per_step(Layer(1, 1, 4096, 64, L, p, 1)) == want
