@@ -49,6 +49,17 @@ Readings of points the pages leave open (each one is listed in the design doc):
       the backward passes gradients through those casts unchanged.
       attn_dtype=None keeps them exact.
 
+What pins each step (tests/test_oracle_pins.py; planted mistakes in
+tests/test_oracle_mutants.py): pooling, norms, max-pooling and the scatter sum
+against their definitions computed another way; the top-k against brute force
+over all subsets; S and the entry count against hand-worked values; L = 1
+against torch's causal attention; the backward against finite differences,
+adjoint identities and torch autograd of an independent forward.  Two
+readings are pinned only to their own statement, because the pages give no
+value to check them against: the chunk length T = 2048 of R3 (parity unpinned
+against the pages' own top-K kernel) and the shift of R7 beyond the causality
+it must keep (parity unpinned against the pages' own scatter).
+
 All arrays are float64 numpy arrays; one head at a time is ``[N, d]``.
 """
 
