@@ -27,7 +27,7 @@ algorithm's own steps in the pages' order, written plainly in float64:
   7. backward by hand-derived adjoints; top-k passes no gradient
                                          (LH-summary Method step 5; LH-post How it works (2))
 
-Readings of points the pages leave open (each one is listed in the design doc):
+Readings of points the pages leave open:
   R1  N must be divisible by p^(L-1).
   R2  scorer: "qk_sum" = ||Q_t|| + ||K_t|| (default), "k" = ||K_t|| (the
       projection-norm run), "q" = ||Q_t||.

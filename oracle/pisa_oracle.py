@@ -17,7 +17,7 @@ level, down to the finest level; the cost is O(N log N) (section 3, second
 paragraph); block sparse attention splits the keys into contiguous blocks
 and selects some of them per query (section 1, "Block Sparse Attention").
 
-Readings of what it leaves open (each is listed in the design doc):
+Readings of what it leaves open:
   P1  the hierarchy is the mean-pooled key pyramid with factor p: level-l entry
       j is the mean of keys [j p^l, (j+1) p^l); level 0 holds the keys as given.
       Pooled keys are stored in bf16, rounded to nearest even from the exact

@@ -59,13 +59,21 @@ def test_full_size(name):
 
     # sampled heads against the oracle
     flat = lambda t: t.reshape(w.B * w.H, w.N, w.d)  # noqa: E731
+    checks = []
     for bh, h in cases.items():
         o = pu.oracle_head(w, h["q"], h["k"], h["v"], h["dy"])
         sv = o["saved"]
         np.testing.assert_array_equal(v["sel"][bh].cpu().numpy().astype(np.int64), pu.oracle_sel_flat(w, sv))
         np.testing.assert_array_equal(v["seq_map"][bh].cpu().numpy().astype(np.int64), pu.oracle_seq_map(sv))
         np.testing.assert_array_equal(v["slot_of"][bh].cpu().numpy().astype(np.int64), pu.oracle_slot_of(sv))
-        pu.assert_close(pu.to_np(flat(y)[bh]), o["Y"], f"{name} head {bh} Y")
-        pu.assert_close(pu.to_np(flat(dq)[bh]), o["dQ"], f"{name} head {bh} dQ")
-        pu.assert_close(pu.to_np(flat(dk)[bh]), o["dK"], f"{name} head {bh} dK")
-        pu.assert_close(pu.to_np(flat(dv)[bh]), o["dV"], f"{name} head {bh} dV")
+        checks += [(v["os"][bh], sv["Os"], f"{name} head {bh} Os"), (flat(y)[bh], o["Y"], f"{name} head {bh} Y"),
+                   (flat(dq)[bh], o["dQ"], f"{name} head {bh} dQ"), (flat(dk)[bh], o["dK"], f"{name} head {bh} dK"),
+                   (flat(dv)[bh], o["dV"], f"{name} head {bh} dV")]
+        if bh == SAMPLED[name][0]:
+            # for information: against the oracle without the bf16 rounding of
+            # the attention's inputs
+            ox = pu.oracle_head(w, h["q"], h["k"], h["v"], h["dy"], attn_dtype=None)
+            pu.record_info(v["os"][bh], ox["saved"]["Os"], f"{name} head {bh} Os [exact attention inputs]")
+            for t, n in ((y, "Y"), (dq, "dQ"), (dk, "dK"), (dv, "dV")):
+                pu.record_info(flat(t)[bh], ox[n], f"{name} head {bh} {n} [exact attention inputs]")
+    pu.assert_all_close(checks)

@@ -22,17 +22,25 @@ def test_forward_backward(name):
     lh.check_error(bufs)
     v = bufs.ctx_views()
     flat = lambda t: t.reshape(w.B * w.H, w.N, w.d)  # noqa: E731
+    checks = []
     for bh, o in enumerate(heads):
         sv = o["saved"]
         if w.L > 1:
             np.testing.assert_array_equal(v["sel"][bh].cpu().numpy().astype(np.int64), pu.oracle_sel_flat(w, sv))
         np.testing.assert_array_equal(v["seq_map"][bh].cpu().numpy().astype(np.int64), pu.oracle_seq_map(sv))
         np.testing.assert_array_equal(v["slot_of"][bh].cpu().numpy().astype(np.int64), pu.oracle_slot_of(sv))
-        pu.assert_close(pu.to_np(v["os"][bh]), sv["Os"], f"{name} Os")
-        pu.assert_close(pu.to_np(flat(y)[bh]), o["Y"], f"{name} Y")
-        pu.assert_close(pu.to_np(flat(dq)[bh]), o["dQ"], f"{name} dQ")
-        pu.assert_close(pu.to_np(flat(dk)[bh]), o["dK"], f"{name} dK")
-        pu.assert_close(pu.to_np(flat(dv)[bh]), o["dV"], f"{name} dV")
+        checks += [(v["os"][bh], sv["Os"], f"{name} head {bh} Os"), (flat(y)[bh], o["Y"], f"{name} head {bh} Y"),
+                   (flat(dq)[bh], o["dQ"], f"{name} head {bh} dQ"), (flat(dk)[bh], o["dK"], f"{name} head {bh} dK"),
+                   (flat(dv)[bh], o["dV"], f"{name} head {bh} dV")]
+        # for information: the same outputs against the oracle run without the
+        # bf16 rounding of the attention's inputs (how far that reading moves
+        # the reference point)
+        ox = pu.oracle_head(w, x["q"][bh // w.H, bh % w.H], x["k"][bh // w.H, bh % w.H], x["v"][bh // w.H, bh % w.H],
+                            x["dy"][bh // w.H, bh % w.H], attn_dtype=None)
+        pu.record_info(v["os"][bh], ox["saved"]["Os"], f"{name} head {bh} Os [exact attention inputs]")
+        for t, n in ((y, "Y"), (dq, "dQ"), (dk, "dK"), (dv, "dV")):
+            pu.record_info(flat(t)[bh], ox[n], f"{name} head {bh} {n} [exact attention inputs]")
+    pu.assert_all_close(checks)
 
 
 def test_forward_is_deterministic():
@@ -45,9 +53,10 @@ def test_forward_is_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
     assert torch.equal(b1.ctx, b2.ctx)
-    # dK and dV have one writer per row; dQ sums tiles with atomics (order may vary)
-    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
-    pu.assert_close(pu.to_np(g1[0]), pu.to_np(g2[0]), "dQ repeat", max_err=1e-5, mean_err=1e-6)
+    # every output row has one writer and a fixed summation order (no atomics
+    # anywhere): repeated runs agree bit for bit
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
 
 
 def test_autograd_function_matches_direct_calls():
@@ -60,5 +69,4 @@ def test_autograd_function_matches_direct_calls():
     dq2, dk2, dv2 = lh.backward(L, x["dy"], bufs)
     torch.cuda.synchronize()
     assert torch.equal(y.detach(), y2)
-    assert torch.equal(k.grad, dk2) and torch.equal(v.grad, dv2)
-    pu.assert_close(pu.to_np(q.grad), pu.to_np(dq2), "dQ autograd", max_err=1e-5, mean_err=1e-6)
+    assert torch.equal(q.grad, dq2) and torch.equal(k.grad, dk2) and torch.equal(v.grad, dv2)
