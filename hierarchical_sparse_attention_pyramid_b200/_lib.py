@@ -13,6 +13,7 @@ from ctypes import POINTER, c_char_p, c_int, c_int32, c_int64, c_size_t, c_void_
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblh.so")
 MAX_LEVELS = 16
 ERR_WORD_BYTES = 256
+SELFTEST_WS_BYTES = 131072
 
 LH_OK = 0
 STATUS_NAMES = {0: "LH_OK", 1: "LH_ERR_INVALID_ARG", 2: "LH_ERR_UNSUPPORTED", 3: "LH_ERR_WORKSPACE",
@@ -77,6 +78,7 @@ SIGNATURES = {
     "lh_pisa_plan": [_PCFG, POINTER(LhPisaInfo)],
     "lh_pisa_pool_keys": [_PCFG, _P, _P, _P],
     "lh_pisa_select": [_PCFG, _P, _P, _P, _P, _P, _P, _P],
+    "lh_selftest_wait_timeout": [_P, c_size_t, c_int64, _P],
     "lh_check_error": [_P, _P],
     "lh_clear_error": [_P, _P],
     "lh_status_string": [c_int],

@@ -425,6 +425,28 @@ lh_status lh_backward(const lh_config* cfg, const void* dy, const void* ctx, siz
   return LH_OK;
 }
 
+lh_status lh_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t wait_cycles, lh_stream_t stream) {
+  LH_CHECK_PTR(ws);
+  if (ws_bytes < LH_SELFTEST_WS_BYTES)
+    return fail(LH_ERR_WORKSPACE, "lh_selftest_wait_timeout: ws smaller than LH_SELFTEST_WS_BYTES");
+  if (wait_cycles < 1 || wait_cycles > 4000000000ll)
+    return fail(LH_ERR_INVALID_ARG, "lh_selftest_wait_timeout: wait_cycles outside [1, 4e9]");
+  // one 128 x 64 tile each of Qs, Ks, Vs (bf16, 16 KB) after the error word,
+  // then O (fp32, 32 KB) and LSE (512 B): 256 + 3 * 16384 + 32768 + 512 bytes
+  char* w = static_cast<char*>(ws);
+  const int64_t S = 128;
+  const int d = 64;
+  void* qs = w + LH_ERR_WORD_BYTES;
+  void* ks = w + LH_ERR_WORD_BYTES + 16384;
+  void* vs = w + LH_ERR_WORD_BYTES + 2 * 16384;
+  float* os = reinterpret_cast<float*>(w + LH_ERR_WORD_BYTES + 3 * 16384);
+  float* lse = reinterpret_cast<float*>(w + LH_ERR_WORD_BYTES + 3 * 16384 + 32768);
+  LH_CUDA(launch_attn_fwd(1, S, d, qs, ks, vs, os, lse, err_word(ws), (cudaStream_t)stream, (long long)wait_cycles,
+                          /*issue_loads=*/0),
+          "lh_selftest_wait_timeout");
+  return LH_OK;
+}
+
 lh_status lh_check_error(void* ws, lh_stream_t stream) {
   if (!ws) return fail(LH_ERR_INVALID_ARG, "lh_check_error: NULL ws");
   const cudaStream_t st = (cudaStream_t)stream;

@@ -5,19 +5,19 @@
 // One CTA owns two 128-row query tiles (A = 2c, B = 2c+1) of one (batch,
 // head) and streams the key/value tiles 0..2c+1 once for both (causal; each
 // tile's diagonal block is masked).  Warp roles:
-//   warps 0-15 softmax, a warpgroup pair per query tile (warps 0-7 tile A,
-//              8-15 tile B, side by side): thread (g, t) of a pair owns query
-//              row t (TMEM lane t) and keys [64g, 64g+64); it loads its 64
-//              scores from TMEM once, exchanges the row max with the other
-//              group, keeps the running max and its partial row sum, rescales
-//              its half of O in TMEM when the max moves, and writes P back
-//              over the S columns it came from as a bf16 pair (per 32 keys: 16
-//              columns of hi, 16 of lo), where the P V product reads it
-//   warp 16    TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
-//   warp 17    MMA issuer (the converged warp; one elected lane issues):
+//   warps 0-7  softmax, one warpgroup per query tile (warps 0-3 tile A, 4-7
+//              tile B): thread t of a group owns query row t (TMEM lane t) and
+//              all 128 keys of a key tile, so the row max needs no exchange
+//              between threads; it keeps the running max and row sum,
+//              rescales its O row in TMEM when the max moves, and writes P
+//              back over the S columns it came from as a bf16 pair (per 32
+//              keys: 16 columns of hi, 16 of lo), where the P V product reads it
+//   warp 8     TMA producer: both Q tiles once, K and V tiles into a 2-stage ring
+//   warp 9     MMA issuer (the converged warp; one elected lane issues):
 //              for each key tile, P_A V, then the next S_A = Q_A K^T, then
-//              P_B V and the next S_B, so the tensor core works on one tile
-//              while the other tile's softmax runs
+//              P_B V and the next S_B.  One tile's softmax runs while the
+//              tensor core works on the other tile's products, so the two
+//              groups take turns rather than sharing the issue slots.
 // TMEM columns: S_A/P_A [0,128), S_B/P_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 // The P pair keeps P V at fp32 accuracy (the backward's Delta = rowsum(dO O)
 // cancels against P (dP - Delta), so O errors would reach dQ); O is written
@@ -35,9 +35,10 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BN = 128;
-constexpr int kSoftmax = 512;          // two warpgroup pairs, one per query tile
-constexpr int kPair = kSoftmax / 2;    // softmax threads of one query tile
+constexpr int kSoftmax = 256;          // two warpgroups, one per query tile
+constexpr int kPair = kSoftmax / 2;    // softmax threads of one query tile (one per row)
 constexpr int kThreads = kSoftmax + 64;
+constexpr int kWarpTma = kSoftmax / 32, kWarpMma = kWarpTma + 1;
 
 
 template <int D>
@@ -47,17 +48,19 @@ struct FwdSmem {
   static constexpr int oQ = 0;              // Q_A, Q_B
   static constexpr int oK = oQ + 2 * kTile; // 2 stages
   static constexpr int oV = oK + 2 * kTile; // 2 stages
-  static constexpr int oXch = oV + 2 * kTile;  // softmax exchange, per tile: [2][2][128] maxima, [2][128] sums
-  static constexpr int oBar = oXch + 2 * 768 * 4;
+  static constexpr int oBar = oV + 2 * kTile;
   static constexpr int kBytes = oBar + 256;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
+// 10 warps, three on some SM sub-partitions: at most 168 registers a thread
+// (a sub-partition holds 16384).  A softmax thread holds its row's 128 scores
+// in registers and writes P back 16 keys at a time.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, float* __restrict__ LSE,
-                    int* errw, int S, float scale_log2) {
+                    int* errw, int S, float scale_log2, long long wait_cycles, int issue_loads) {
   using Lay = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -69,7 +72,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bS = bars + 7;       // [2] tiles: S of the tile in TMEM (and its previous P V done)
   uint64_t* bP = bars + 9;       // [2] tiles: P in TMEM, O rescaled (one arrival per thread of the tile's pair)
   uint64_t* bO = bars + 11;      // [2] tiles: a P V product of the tile done
-  uint64_t* bX = bars + 13;      // [2 tiles][2] softmax exchange within a tile's warpgroup pair
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
@@ -92,21 +94,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bS[s], 1);
       mbar_init(&bP[s], kPair);
       mbar_init(&bO[s], 1);
-      mbar_init(&bX[s], kPair);
-      mbar_init(&bX[2 + s], kPair);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 17) tmem_alloc(tmem_slot, 512);
+  if (warp == kWarpMma) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 16) {
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // issue_loads == 0 only in the timeout self-test: nothing is loaded, so
+    // the other roles' bounded waits run out with no copy or MMA in flight
+    if (lane == 0 && issue_loads) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(smem + Lay::oQ + x * Lay::kTile + ch * Lay::kChunk, &tmQ, bQ, ch * 64, qtile[x] * BM, bh);
       for (int j = 0; j < n_kv; ++j) {
         const int st = j & 1, use = j >> 1;
-        if (j >= 2 && !mbar_wait(&bKVfree[st], (use - 1) & 1, abort_flag)) break;
+        if (j >= 2 && !mbar_wait(&bKVfree[st], (use - 1) & 1, abort_flag, wait_cycles)) break;
         mbar_expect_tx(&bK[st], BN * D * 2);
         for (int ch = 0; ch < D / 64; ++ch)
           tma_load_3d(smem + Lay::oK + st * Lay::kTile + ch * Lay::kChunk, &tmK, &bK[st], ch * 64, j * BN, bh);
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(smem + Lay::oV + st * Lay::kTile + ch * Lay::kChunk, &tmV, &bV[st], ch * 64, j * BN, bh);
       }
     }
-  } else if (warp == 17) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     {  // the whole warp; one elected lane issues each instruction
       constexpr uint32_t idQK = idesc_bf16(BM, BN, false, false);
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit_w(&bS[x]);
       };
-      bool ok = mbar_wait_warp(bQ, 0, abort_flag) && mbar_wait_warp(&bK[0], 0, abort_flag);
+      bool ok = mbar_wait_warp(bQ, 0, abort_flag, wait_cycles) && mbar_wait_warp(&bK[0], 0, abort_flag, wait_cycles);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -154,9 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool v_ready = false, k_next_ready = false;
         for (int x = 0; x < 2 && ok; ++x) {
           if (j > last[x]) continue;
-          if (!mbar_wait_warp(&bP[x], j & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bP[x], j & 1, abort_flag, wait_cycles)) { ok = false; break; }
           if (!v_ready) {
-            if (!mbar_wait_warp(&bV[st], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(&bV[st], (j >> 1) & 1, abort_flag, wait_cycles)) { ok = false; break; }
             v_ready = true;
           }
           tc_fence_after();
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit_w(&bO[x]);
           if (j + 1 <= last[x]) {
             if (!k_next_ready) {
-              if (!mbar_wait_warp(&bK[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+              if (!mbar_wait_warp(&bK[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, wait_cycles)) { ok = false; break; }
               k_next_ready = true;
               tc_fence_after();
             }
@@ -184,63 +186,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // Warpgroup pair x (warps 8x .. 8x+7) works on query tile x, so the two
-    // tiles' softmax passes run side by side.  Within a pair, thread (g, t)
-    // owns query row t (TMEM lane t) and keys [64g, 64g+64) of the key tile:
-    // it loads its 64 scores from TMEM once, exchanges the row max with the
-    // other group through shared memory (one barrier per key tile, a bounded
-    // wait), keeps the running max and its partial row sum, rescales its half
-    // of O when the max moves, and writes P back over the S columns it came
-    // from as a bf16 pair (per 32 keys: 16 columns of hi, 16 of lo), where
-    // the P V product reads it.  Both groups use the same running reference
-    // m, so the partial sums add at the end.
-    const int x = warp >> 3;
-    const int g = (warp >> 2) & 1;
+    // Warpgroup x (warps 4x .. 4x+3) works on query tile x; thread t owns
+    // query row t (TMEM lane t) and all 128 keys of each key tile.  It loads
+    // the row's scores from TMEM once, takes their max, keeps the running max
+    // and row sum, rescales its O row when the max moves, and writes P back
+    // over the S columns it came from as a bf16 pair (per 32 keys: 16
+    // columns of hi, 16 of lo), where the P V product reads it.
+    const int x = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    float* sXch = reinterpret_cast<float*>(smem + Lay::oXch) + x * 768;  // [2 parity][2 groups][128] maxima, then [2 groups][128] sums
-    uint64_t* bXx = bX + 2 * x;
+    const uint32_t ts = tl + x * 128, to = tl + 256 + x * D;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int n_x = 0;  // exchanges so far: buffer n_x & 1 of sXch, barrier bXx[n_x & 1]
-    // all 256 threads of the pair have written their part of the exchange buffer
-    auto exchange = [&]() -> bool {
-      mbar_arrive(&bXx[n_x & 1]);
-      const bool done = mbar_wait(&bXx[n_x & 1], (n_x >> 1) & 1, abort_flag);
-      ++n_x;
-      return done;
-    };
-    const uint32_t ts = tl + x * 128 + g * 64, to = tl + 256 + x * D + g * (D / 2);
     for (int j = 0; ok && j <= last[x]; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bS[x], j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bS[x], j & 1, abort_flag, wait_cycles));
       if (!ok) break;
       tc_fence_after();
       const bool diag = (j == last[x]);
+      // row max of the raw scores (the scale is positive), as eight
+      // independent chains over two 64-key halves loaded in turn (the scores
+      // are read again for the P pass, so no more than 64 are held at once);
+      // on the diagonal tile the keys after the row are masked
       uint32_t r[2][32];
-      tmem_ld32(ts, r[0]);
-      tmem_ld32(ts + 32, r[1]);
-      tmem_ld_wait();
-      // row max of the raw scores over this group's keys (the scale is
-      // positive); on the diagonal tile the keys after the row are masked
-      float mx = -INFINITY;
-      if (diag) {
-        const int lim = row - g * 64;
+      float mc[8];
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+      for (int c8 = 0; c8 < 8; ++c8) mc[c8] = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (ch * 32 + i <= lim) mx = fmaxf(mx, __uint_as_float(r[ch][i]));
-      } else {
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(ts + hh * 64, r[0]);
+        tmem_ld32(ts + hh * 64 + 32, r[1]);
+        tmem_ld_wait();
+        if (diag) {
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+          for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) mx = max3f(mx, __uint_as_float(r[ch][i]), __uint_as_float(r[ch][i + 1]));
+            for (int i = 0; i < 32; ++i)
+              if (hh * 64 + ch * 32 + i <= row)
+                mc[ch * 4 + (i >> 3)] = fmaxf(mc[ch * 4 + (i >> 3)], __uint_as_float(r[ch][i]));
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              mc[ch * 4 + (i >> 3)] =
+                  max3f(mc[ch * 4 + (i >> 3)], __uint_as_float(r[ch][i]), __uint_as_float(r[ch][i + 1]));
+        }
       }
-      float* xch = sXch + (n_x & 1) * 256;
-      xch[g * 128 + row] = mx;
-      ok = __all_sync(0xffffffffu, exchange());
-      if (!ok) break;
-      mx = fmaxf(mx, xch[(1 - g) * 128 + row]);
+      const float mx = fmaxf(fmaxf(max3f(mc[0], mc[1], mc[2]), max3f(mc[3], mc[4], mc[5])), fmaxf(mc[6], mc[7]));
       // Lazy rescaling: the reference m_run moves only when the row max
       // exceeds it by more than 8 (so every P stays <= 2^8); O and l share
       // the reference, so the result is exact either way.
@@ -249,45 +241,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = move ? m_tile : m_run;
       const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;
       // P = 2^(s*scale - m) as a bf16 pair written back over the chunk it
-      // came from: chunk ch (keys 32ch..32ch+31 of the group) holds hi in
-      // its first 16 columns and lo in its last 16, where P V reads them.
-      // Keys after the row are masked on the diagonal tile only.
+      // came from: chunk ch (keys 32ch..32ch+31) holds hi in its first 16
+      // columns and lo in its last 16, where P V reads them.  Keys after the
+      // row are masked on the diagonal tile only.
       const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_new, -m_new);
-      uint64_t rs2 = f2_pack(0.f, 0.f);
+      uint64_t rs2[4];
       auto p_pass = [&](auto masked) {
-        const int limit = row - g * 64;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t hi[16], lo[16];
+        for (int hh = 0; hh < 2; ++hh) {
+          tmem_ld32(ts + hh * 64, r[0]);
+          tmem_ld32(ts + hh * 64 + 32, r[1]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float a, b;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[ch][2 * q]), __uint_as_float(r[ch][2 * q + 1])), c2, nm2), a,
-                      b);
-            a = fast_exp2(a);
-            b = fast_exp2(b);
-            if constexpr (decltype(masked)::value) {
-              const int col = ch * 32 + 2 * q;
-              a = col > limit ? 0.f : a;
-              b = col + 1 > limit ? 0.f : b;
+          for (int c = 0; c < 2; ++c) {
+            const int ch = hh * 2 + c;
+            rs2[ch] = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // keys 32ch+16h .. +15: hi to columns 32ch+8h, lo to 32ch+16+8h
+              uint32_t hi[8], lo[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const int e = 16 * h + 2 * q;
+                float a, b;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(r[c][e]), __uint_as_float(r[c][e + 1])), c2, nm2), a, b);
+                a = fast_exp2(a);
+                b = fast_exp2(b);
+                if constexpr (decltype(masked)::value) {
+                  const int col = ch * 32 + e;
+                  a = col > row ? 0.f : a;
+                  b = col + 1 > row ? 0.f : b;
+                }
+                rs2[ch] = f2_add(rs2[ch], f2_pack(a, b));
+                split_bf16x2(a, b, hi[q], lo[q]);
+              }
+              tmem_st8(ts + ch * 32 + 8 * h, hi);
+              tmem_st8(ts + ch * 32 + 16 + 8 * h, lo);
             }
-            rs2 = f2_add(rs2, f2_pack(a, b));
-            split_bf16x2(a, b, hi[q], lo[q]);
           }
-          tmem_st16(ts + ch * 32, hi);
-          tmem_st16(ts + ch * 32 + 16, lo);
         }
       };
       if (diag) p_pass(std::true_type{});
       else p_pass(std::false_type{});
       float rsa, rsb;
-      f2_unpack(rs2, rsa, rsb);
+      f2_unpack(f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3])), rsa, rsb);
       const float rs = rsa + rsb;
-      // rescale this group's half of the O row; the previous P V of this
-      // tile is done (its completion preceded this S)
+      // rescale the O row; the previous P V of this tile is done (its
+      // completion preceded this S)
       if (j >= 1 && __any_sync(0xffffffffu, move)) {
 #pragma unroll 1
-        for (int ch = 0; ch < D / 64; ++ch) {
+        for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t o[32];
           tmem_ld32(to + ch * 32, o);
           tmem_ld_wait();
@@ -302,37 +304,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bP[x]);
     }
-    // row sums: the two groups' partial sums of the tile
     if (ok && last[x] >= 0) {
-      float* sL = sXch + 512;
-      sL[g * 128 + row] = l_run;
-      ok = __all_sync(0xffffffffu, exchange());
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bO[x], last[x] & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bO[x], last[x] & 1, abort_flag, wait_cycles));
       if (ok) {
         tc_fence_after();
-        const float l = l_run + sL[(1 - g) * 128 + row];
-        const float inv_l = 1.f / l;
+        const float inv_l = 1.f / l_run;
         const int row_g = qtile[x] * BM + row;
 #pragma unroll 1
-        for (int ch = 0; ch < D / 64; ++ch) {
+        for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t o[32];
           tmem_ld32(to + ch * 32, o);
           tmem_ld_wait();
           if (row_g < S) {
-            float4* dst = reinterpret_cast<float4*>(O + ((int64_t)bh * S + row_g) * D + g * (D / 2) + ch * 32);
+            float4* dst = reinterpret_cast<float4*>(O + ((int64_t)bh * S + row_g) * D + ch * 32);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               dst[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
                                    __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
           }
         }
-        if (g == 0 && row_g < S) LSE[(int64_t)bh * S + row_g] = (m_run + log2f(l)) * 0.69314718055994530942f;
+        if (row_g < S) LSE[(int64_t)bh * S + row_g] = (m_run + log2f(l_run)) * 0.69314718055994530942f;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 17) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -380,7 +377,7 @@ bool make_f32_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, in
 }
 
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
-                            float* lse, int* errw, cudaStream_t st) {
+                            float* lse, int* errw, cudaStream_t st, long long wait_cycles, int issue_loads) {
   CUtensorMap mq, mk, mv;
   if (!make_seq_map(&mq, qs, BH, S, d, BM) || !make_seq_map(&mk, ks, BH, S, d, BN) ||
       !make_seq_map(&mv, vs, BH, S, d, BN))
@@ -392,12 +389,14 @@ cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const 
     const int smem = FwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2);
+    attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2, wait_cycles,
+                                                               issue_loads);
   } else {
     const int smem = FwdSmem<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2);
+    attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2, wait_cycles,
+                                                               issue_loads);
   }
   return cudaGetLastError();
 }

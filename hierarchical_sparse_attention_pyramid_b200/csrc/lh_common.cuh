@@ -123,8 +123,11 @@ cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t*
                                    void* dos, float* delta, int* errw, cudaStream_t st);
 cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dks, const float* dvs,
                                 const int32_t* slot_of, void* dq, void* dk, void* dv, cudaStream_t st);
+// wait_cycles bounds every barrier wait of the kernel (SM clocks);
+// issue_loads = 0 only for the timeout self-test (the producer loads nothing)
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
-                            float* lse, int* errw, cudaStream_t st);
+                            float* lse, int* errw, cudaStream_t st, long long wait_cycles = 4000000000ll,
+                            int issue_loads = 1);
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
                             float* dvs, int* errw, cudaStream_t st);

@@ -45,14 +45,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Returns false when
-// the CTA is aborting (another role gave up) or this wait ran out of time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// the CTA is aborting (another role gave up) or this wait ran out of time
+// (`limit` SM clocks).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       return false;
     }
@@ -60,8 +62,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // mbar_wait by every lane of a converged warp, with one outcome for all lanes
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               long long limit = kWaitCycles) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, limit));
 }
 
 // ---------------------------------------------------------------- TMA
@@ -259,12 +262,6 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   f2_unpack(f2_sub(f2_pack(a, b), hf), ra, rb);
   const __nv_bfloat162 l = __floats2bfloat162_rn(ra, rb);
   lo = *reinterpret_cast<const uint32_t*>(&l);
-}
-// fp32 vector add into global memory without a returned value (a reduction,
-// performed at the L2)
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 // Whole-warp forms of the MMA issue: every lane of a converged warp makes
 // the call and one lane, chosen by elect.sync, issues the instruction.  An

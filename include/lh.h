@@ -176,16 +176,21 @@ lh_status lh_score_topk(const lh_config *cfg, const float *norms, void *ws, int3
 /* Stage 2 without workspace, for callers that cannot allocate device memory
  * (a host whose allocator owns every device buffer, a runtime whose memory
  * plan is fixed, a plugin that only receives its inputs and outputs).  The
- * pages have no counterpart: this is lh_score_topk with its score pyramid
- * kept in a file-scope device array of 16 MiB (B*H * upper_entries * 4 bytes
- * at most; larger configurations return LH_ERR_UNSUPPORTED) that every GPU
- * loading the library holds until exit.  It calls no allocator.
+ * pages have no counterpart: this is lh_score_topk with its scratch kept in a
+ * file-scope device array of 16 MiB that every GPU loading the library holds
+ * until exit.  It calls no allocator.  The scratch a call needs is lh_plan's
+ * topk_ws_bytes - LH_ERR_WORD_BYTES: the score pyramid, B*H * upper_entries * 4
+ * bytes, plus B*H * N * 4 bytes of level-0 scores with LH_SELECT_DIRECT;
+ * configurations above 16 MiB return LH_ERR_UNSUPPORTED.
  * In:  norms as for lh_score_topk.  Out: sel as for lh_score_topk.
- * The first call on a device looks up the array's device address (with
- * cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture.  All calls share the array: calls that overlap on the GPU (other
- * streams, other threads) race and must be serialised by the caller.  The
- * array keeps the last call's contents; every call rewrites all it reads. */
+ * The first call on a device (and the first after a cudaDeviceReset, which
+ * makes a new context) looks up the array's device address with
+ * cudaGetSymbolAddress and caches it per device and context; make that first
+ * call before any stream capture.  All calls share the array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  The array keeps the last call's contents; every
+ * call rewrites all it reads.  There is no error word: the selection's one
+ * device-side check is kept unreachable by lh_plan's limits. */
 lh_status lh_score_topk_static(const lh_config *cfg, const float *norms, int32_t *sel, lh_stream_t stream);
 
 /* Stage 3 - gather the kept entries into one causally ordered sequence.
@@ -334,6 +339,22 @@ lh_status lh_pisa_pool_keys(const lh_pisa_config *cfg, const void *k, void *kpyr
  * level has fewer than topk candidates.  Level 0 is the selection. */
 lh_status lh_pisa_select(const lh_pisa_config *cfg, const void *q, const void *k, const void *kpyr,
                          int32_t *kept_idx, float *kept_score, void *ws, lh_stream_t stream);
+
+/* Self-test of the device-side timeout path (the pages have no counterpart).
+ * Launches the stage-4 forward kernel on one 128-row tile (d = 64) with its
+ * TMA producer told to load nothing and every barrier wait bounded by
+ * `wait_cycles` SM clocks.  Its MMA and softmax warps then wait on barriers
+ * that never complete; the first wait to run out stops every role, the kernel
+ * returns (no copy or MMA was ever issued, so nothing is in flight) and sets
+ * the timeout bit of the error word at the start of ws.  The GPU context
+ * stays usable.
+ * In:  wait_cycles in [1, 4e9] (about 2 s at the boost clock for 4e9).
+ * ws:  device buffer of at least LH_SELFTEST_WS_BYTES bytes: the error word,
+ *      then room the kernel's tensor maps and outputs point into.
+ * Returns LH_OK once the kernel is queued; lh_check_error(ws, stream) then
+ * returns LH_ERR_TIMEOUT, which is the expected outcome. */
+#define LH_SELFTEST_WS_BYTES 131072
+lh_status lh_selftest_wait_timeout(void *ws, size_t ws_bytes, int64_t wait_cycles, lh_stream_t stream);
 
 /* Synchronise `stream`, read the error word at the start of ws, clear it and
  * return LH_OK, LH_ERR_TIMEOUT or LH_ERR_DEVICE (or LH_ERR_CUDA). */

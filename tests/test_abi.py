@@ -186,3 +186,15 @@ def test_kernels_per_step(L, p, want):
     pool adjoint (no selection kernels at L = 1).  The 512K-token launch list
     under profiles/ shows the 10 of (L, p) = (5, 4) per step."""
     assert kernels_per_step(Layer(1, 1, 4096, 64, L, p, 1)) == want
+
+
+def test_selftest_timeout_argument_checks(lib):
+    # refused on the host before anything is queued
+    fake = ctypes.c_void_p(1 << 40)
+    assert lib.lh_selftest_wait_timeout(fake, ctypes.c_size_t(_lib.SELFTEST_WS_BYTES - 1), ctypes.c_int64(1000),
+                                        None) == 3
+    assert lib.lh_selftest_wait_timeout(fake, ctypes.c_size_t(_lib.SELFTEST_WS_BYTES), ctypes.c_int64(0), None) == 1
+    assert lib.lh_selftest_wait_timeout(fake, ctypes.c_size_t(_lib.SELFTEST_WS_BYTES), ctypes.c_int64(5_000_000_000),
+                                        None) == 1
+    assert lib.lh_selftest_wait_timeout(None, ctypes.c_size_t(_lib.SELFTEST_WS_BYTES), ctypes.c_int64(1000),
+                                        None) == 1
