@@ -9,6 +9,7 @@
 // a plugin that is only given its inputs and outputs.  For them this entry
 // point keeps the score pyramid in one file-scope device array of fixed size
 // that the library carries from load to exit, and calls no allocator.
+#include <cuda.h>
 #include <mutex>
 
 #include "lh_common.cuh"
@@ -16,9 +17,12 @@
 namespace lh {
 namespace {
 
-// Largest score pyramid the static array holds: 16 MiB, i.e. B*H times the
-// entries of levels >= 1 times 4 bytes.  The 512K-token, 16-head layer needs
-// 11.1 MB; the 1M-token, 8-head layer 11.2 MB.
+// Largest scratch the static array holds: 16 MiB.  A call needs the score
+// pyramid, B*H times the entries of levels >= 1 times 4 bytes, plus (direct
+// selection only) the level-0 scores, B*H*N*4 bytes, after it: lh_plan's
+// topk_ws_bytes minus the error word.  The 512K-token, 16-head layer needs
+// 11.1 MB (45 MB with direct selection, which is refused); the 1M-token,
+// 8-head layer 11.2 MB.
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;
 
 // Held by every GPU that loads the library until the process exits.
@@ -27,21 +31,44 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 constexpr int kMaxDevices = 128;
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+// The current context, read through the runtime's driver entry point (no
+// link against libcuda).  A cudaDeviceReset replaces the device's primary
+// context, which reloads the module and can move the array.
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  }
+  CUcontext c = nullptr;
+  if (fn) fn(&c);
+  return c;
+}
 
 // Device address of the array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with cudaGetSymbolAddress (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress (with that device current) and cached per device,
+// keyed by the context it was looked up in: a call in a new context (after a
+// cudaDeviceReset) looks it up again.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const CUcontext ctx = current_context();  // NULL before the runtime made one current
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // makes the primary context current if none is
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -77,7 +104,9 @@ extern "C" lh_status lh_score_topk_static(const lh_config* cfg, const float* nor
     return LH_ERR_CUDA;
   }
   // every entry of the pyramid is written before it is read, so nothing in
-  // the array has to start at zero
+  // the array has to start at zero.  There is no error word: the one
+  // device-side check of the selection (a nested chunk larger than its
+  // staging buffer) is kept unreachable by lh_plan's limits.
   e = launch_score_topk(D, norms, static_cast<float*>(scratch), sel, nullptr, (cudaStream_t)stream);
   if (e != cudaSuccess) {
     set_error_message("lh_score_topk_static: %s", cudaGetErrorString(e));
