@@ -94,19 +94,64 @@ def max_over_ranks(x: float, world: int, device) -> float:
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    """SM clock and clock-event (throttle) reasons sampled while running: NVML
+    every 5 ms when pynvml can open the device, else nvidia-smi every 200 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.005):
         self.gpu = gpu_index
+        self.period = period_s
         self.proc = None
         self.lines = []
+        self.samples = []  # (sm_mhz, reasons bitmask) from NVML
         self.thread = None
+        self.stop_evt = threading.Event()
+        self.nvml = None
+        self.max_mhz = None
+        self.recording = False
+
+    def window(self, on: bool):
+        """NVML samples are kept only inside the window (the timed region)."""
+        self.recording = on
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:  # noqa: BLE001
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self.stop_evt.is_set():
+                    if self.recording:
+                        try:
+                            self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                                 int(get_reasons(h))))
+                        except Exception:  # noqa: BLE001
+                            pass
+                    time.sleep(self.period)
+
+            self.nvml = nv
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:  # noqa: BLE001
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
@@ -121,6 +166,13 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=2)
+            sm = [c for c, _ in self.samples]
+            reasons = sorted(n for n, bit in self.REASON_BITS.items() if any(r & bit for _, r in self.samples))
+            return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(sm), "source": f"NVML every {self.period * 1e3:.0f} ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
@@ -144,7 +196,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi every 200 ms"}
 
 
 # ------------------------------------------------------------------ stage-by-stage timing
@@ -206,7 +258,7 @@ def stage_work(layer: lh.Layer, info) -> dict:
     kept = [p * info.kprime[lvl] for lvl in range(L - 1)] + [info.level_len[L - 1]] if L > 1 else [N]
     read_rows = sum(n * (p ** lvl if 1 <= lvl < first else 1) for lvl, n in enumerate(kept))
     return {
-        "pool": ("hbm", 3 * BH * N * d * e + 3 * BH * U_first * d * e + 2 * BH * N * 4),
+        "pool": ("hbm", 3 * BH * N * d * e),
         "score_topk": ("hbm", 2 * BH * N * 4 + 2 * BH * U * 4 + BH * info.sel_per_head * 4),
         "gather": ("hbm", 3 * BH * read_rows * d * e + 3 * BH * S * d * 2 + BH * S * 4 + BH * E * 4),
         "attn_fwd": ("tensor", 2 * S * S * d * BH),
@@ -215,6 +267,43 @@ def stage_work(layer: lh.Layer, info) -> dict:
         "attn_bwd": ("tensor", 5 * S * S * d * BH),
         "pool_adjoint": ("hbm", 3 * BH * N * d * e + 3 * BH * S * d * 4 + BH * E * 4),
     }
+
+
+def stage_extra_bytes(layer: lh.Layer, info) -> dict:
+    """Bytes a stage moves beyond its algorithmic figure: the pool's writes of
+    the pyramid levels >= first_level and of the level-0 norms."""
+    e = 2 if layer.dtype == "bf16" else 4
+    L, first = layer.L, info.first_level
+    U_first = sum(info.level_len[lvl] for lvl in range(first, L)) if L > 1 else 0
+    return {"pool": 3 * layer.BH * U_first * layer.d * e + 2 * layer.BH * layer.N * 4}
+
+
+def stage_clocks(calls, gpu: int, seconds: float = 0.25) -> dict:
+    """Median SM clock while each stage call runs back to back for about
+    `seconds` (NVML samples every 5 ms): the clock a kernel settles at under
+    its own power draw, which a whole-step sample averages away."""
+    out = {}
+    st = torch.cuda.current_stream()
+    for n, f in calls:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        f()
+        b.record(st)
+        torch.cuda.synchronize()
+        reps = max(1, int(seconds * 1e3 / max(a.elapsed_time(b), 1e-3)))
+        smp = ClockSampler(gpu)
+        smp.start()
+        if smp.nvml is None:
+            smp.stop()
+            return {}
+        smp.window(True)
+        for _ in range(reps):
+            f()
+        torch.cuda.synchronize()
+        smp.window(False)
+        c = smp.stop()
+        out[n] = {"sm_mhz": c["sm_mhz"], "reasons": c["reasons"], "samples": c["samples"]}
+    return out
 
 
 def time_stages(calls, iters: int) -> dict:
@@ -283,39 +372,48 @@ def oracle_sample(w: synth.Workload, heads: int = 1, max_seconds: float = 60.0) 
 
 
 def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores: each step is one head's forward +
+    backward of the timed workload (a bounded sample of the layer), timed by
+    wall clock.  ms_per_step is that measured step; value extrapolates it to
+    the layer (all heads).  Nothing here loads the CUDA library: S comes from
+    the oracle's own size formula."""
     if rank != 0:
         return
+    from oracle import lighthouse_oracle as lo
     w = synth.WORKLOADS[args.workload]
     if args.selection != "parents":
         w = w.with_(selection=args.selection)
-    # one head per step; the oracle keeps no state between steps, so warm-up
-    # steps only load the code paths
-    for _ in range(min(args.warmup, 1)):
-        oracle_sample(w.with_(N=min(w.N, 4096)), 1)
+    # warm-up steps run the same one-head sample (at most 2: the oracle keeps
+    # no state between steps, so they only load code paths and caches)
+    for _ in range(min(args.warmup, 2)):
+        oracle_sample(w, 1)
     r_times = []
     cores = None
     for s in range(args.steps):
         r = oracle_sample(w, 1)
         r_times.append(r["sec_per_head"])
         cores = r["cores"]
-    sec_layer = float(np.mean(r_times)) * w.B * w.H
+    sec_step = float(np.mean(r_times))
+    sec_layer = sec_step * w.B * w.H
     value = w.B * w.N / sec_layer
-    sample = f"one of {w.B * w.H} heads per step (fp64 forward + backward), scaled to the layer"
+    sample = f"one of {w.B * w.H} heads per step (fp64 forward + backward), extrapolated to the layer"
+    S = lo.gathered_length(w.N, w.p, w.L, w.k, w.selection)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": sec_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": sec_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, S),
+        "layer_extrapolation": {"heads_per_step": 1, "heads_per_layer": w.B * w.H, "ms_per_layer": sec_layer * 1e3,
+                                "warmup_steps_run": min(args.warmup, 2)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w: synth.Workload) -> dict:
-    info = lh.plan(lh.Layer.of(w))
+def workload_config(w: synth.Workload, S: int) -> dict:
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "L": w.L, "p": w.p, "k": w.k,
-            "chunk": w.chunk, "scorer": w.scorer, "selection": w.selection, "S": int(info.S),
+            "chunk": w.chunk, "scorer": w.scorer, "selection": w.selection, "S": int(S),
             "parallelism": "replicas (one layer per GPU)",
             "l2": "inputs larger than L2 (Q,K,V,dY %.1f GB per GPU)" % (4 * w.B * w.H * w.N * w.d * 2 / 1e9)}
 
@@ -446,11 +544,13 @@ def run_pisa(args, world, rank, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
+    sampler.window(True)
     e0.record(st)
     for _ in range(args.steps):
         step()
     e1.record(st)
     torch.cuda.synchronize()
+    sampler.window(False)
     barrier(world)
     clocks = sampler.stop()
     _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
@@ -509,7 +609,8 @@ def run_pisa(args, world, rank, local):
         b.record(st)
         torch.cuda.synchronize()
         barrier(world)
-        lh.check_error(bufs)
+        _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()),
+                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         ms_e = max_over_ranks(a.elapsed_time(b) / k_e, world, dev)
         e2e = {"value": world * w.B * w.N / (ms_e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e, "steps": k_e}
@@ -532,24 +633,89 @@ def run_pisa(args, world, rank, local):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ one attention stage alone
+
+def run_stage(args, world, rank, local):
+    """The S-token attention of the workload alone (its B*H and S), on seeded
+    N(0,1) bf16 sequences: a small-memory run of the tensor-core kernels at
+    their full launch shape, for timing and for ncu captures.  Prints one
+    JSON line with the stage's time and its fraction of the bf16 peak."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
+    layer = lh.Layer.of(w)
+    S = lh.plan(layer).S
+    BH, d = layer.BH, w.d
+    g = torch.Generator(device=dev).manual_seed(1234 + rank)
+    qs, ks, vs, dos = (torch.randn(BH, S, d, generator=g, device=dev).to(torch.bfloat16) for _ in range(4))
+    ws = torch.zeros(_lib.ERR_WORD_BYTES, dtype=torch.uint8, device=dev)
+    os_, lse = lh.attn_fwd(layer, qs, ks, vs, ws)
+    delta = (dos.float() * os_).sum(-1)
+    calls = {"attn_fwd": lambda: lh.attn_fwd(layer, qs, ks, vs, ws),
+             "attn_bwd": lambda: lh.attn_bwd(layer, qs, ks, vs, lse, dos, delta, ws)}
+    f = calls[args.stage]
+    for _ in range(max(args.warmup, 1)):
+        f()
+    _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    sampler = ClockSampler(local)
+    sampler.start()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler.window(True)
+    e0.record(st)
+    for _ in range(args.steps):
+        f()
+    e1.record(st)
+    torch.cuda.synchronize()
+    sampler.window(False)
+    barrier(world)
+    clocks = sampler.stop()
+    _lib.call("lh_check_error", ctypes.c_void_p(ws.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    flops = (2 if args.stage == "attn_fwd" else 5) * S * S * d * BH
+    pk, pk_src = peaks()
+    tf = flops / (ms / 1e3) / 1e12
+    if rank == 0:
+        print(json.dumps({"stage": args.stage, "workload": w.name, "BH": BH, "S": S, "d": d, "ms": ms,
+                          "tflops": tf, "frac_burst": tf / pk["bf16_tflops"],
+                          "frac_sustained": tf / pk["bf16_tflops_sustained"], "peak_source": pk_src,
+                          "clocks": clocks, "steps": args.steps, "n_gpus": world}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ main
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 200 for the GPU arms, about 1 s at 512K; 20 for --impl reference, "
+                         "one oracle head per step)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="sparse64_512k", choices=sorted(synth.WORKLOADS) + sorted(synth.PISA_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-stage-clocks", action="store_true")
+    ap.add_argument("--stage", choices=["attn_fwd", "attn_bwd"], default=None,
+                    help="time only this attention stage of the workload (its B*H and S, random sequences)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead (a smaller cut for profiling)")
     ap.add_argument("--selection", default="parents", choices=["parents", "direct", "nested"],
                     help="what a level keeps (the default reading, or one of the two others)")
     args = ap.parse_args()
 
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 200
     world, rank, local = dist_setup()
     if args.workload in synth.PISA_WORKLOADS:
         if args.impl == "reference":
@@ -559,6 +725,9 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args, world, rank)
+        return
+    if args.stage:
+        run_stage(args, world, rank, local)
         return
 
     if not torch.cuda.is_available():
@@ -594,11 +763,13 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(world)
+    sampler.window(True)
     e0.record(st)
     for _ in range(args.steps):
         step()
     e1.record(st)
     torch.cuda.synchronize()
+    sampler.window(False)
     barrier(world)
     clocks = sampler.stop()
     lh.check_error(bufs)
@@ -608,6 +779,8 @@ def main():
     # per-stage durations (same buffers, stage entry points one at a time)
     calls = stage_calls(layer, bufs, x, y, grads)
     stage_ms = time_stages(calls, max(3, min(args.steps, 10)))
+    lh.check_error(bufs)
+    st_clk = stage_clocks(calls, local) if not args.no_stage_clocks else {}
     lh.check_error(bufs)
     pk, pk_src = peaks()
     work = stage_work(layer, bufs.info)
@@ -621,12 +794,16 @@ def main():
             ach = amount / (t / 1e3) / 1e12
             stages[n] = {"ms": t, "bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
                          "frac": ach / pk["bf16_tflops"]}
+        if n in st_clk:
+            stages[n]["clock"] = st_clk[n]
     top = max(stage_ms, key=stage_ms.get)
     ts = stages[top]
     roofline = {"bound": ts["bound"], "kernel": top, "kernels": STAGE_KERNELS[top], "achieved": ts["achieved"],
                 "peak": pk["hbm_gbs"] if ts["bound"] == "hbm" else pk["bf16_tflops"], "unit": ts["unit"],
                 "frac": ts["frac"], "traffic": measured_traffic(top, w.name), "peak_source": pk_src,
-                "share_of_step": stage_ms[top] / sum(stage_ms.values())}
+                "share_of_step": stage_ms[top] / sum(stage_ms.values()),
+                "alg_bytes": work[top][1] if ts["bound"] == "hbm" else None,
+                "extra_bytes": stage_extra_bytes(layer, bufs.info).get(top, 0) if ts["bound"] == "hbm" else None}
     # whole-layer roofline: algorithmic bytes (Q,K,V,dY in; Y,dQ,dK,dV out) at the HBM
     # peak plus the attention flops at the tensor peak
     e = 2 if layer.dtype == "bf16" else 4
@@ -716,7 +893,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic",
-            "config": workload_config(w), "clocks": clocks, "e2e": e2e, "gpu_launches": launches * args.steps,
+            "config": workload_config(w, bufs.info.S), "clocks": clocks, "e2e": e2e, "gpu_launches": launches * args.steps,
             "roofline": roofline, "layer_roofline": layer_roof, "stages": stages, "cpu_baseline": cpu,
             "dense_sdpa": dense,
         }
