@@ -22,11 +22,12 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
         return
     tr = terminalreporter
     tr.section("parity errors (bound: |err| <= 2e-2 + half an ulp of the stored dtype; mean <= 2e-3 + mean half ulp)")
-    tr.write_line(f"{'check':70s} {'dtype':5s} {'max-abs':>10s} {'of bound':>8s} {'mean-abs':>10s} {'of bound':>8s}")
+    tr.write_line(f"{'check':70s} {'dtype':5s} {'max-abs':>10s} {'of bound':>8s} {'mean-abs':>10s} {'of bound':>8s} "
+                  f"{'max-abs |x|<=1':>14s}")
     for r in rows:
         tag = "" if r["kind"] == "check" else "  (info)"
         tr.write_line(f"{r['name'][:70]:70s} {r['dtype']:5s} {r['max_abs']:10.3e} {r['max_ratio']:8.3f} "
-                      f"{r['mean_abs']:10.3e} {r['mean_ratio']:8.3f}{tag}")
+                      f"{r['mean_abs']:10.3e} {r['mean_ratio']:8.3f} {r.get('max_abs_unit', 0.0):14.3e}{tag}")
     path = os.environ.get("LH_PARITY_LOG")
     if path:
         with open(path, "a") as f:

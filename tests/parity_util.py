@@ -63,13 +63,17 @@ def err_stats(got, want, dtype: str | None = None, max_abs: float = MAX_ABS, mea
     dtype = dtype or gd or "fp32"
     assert g.shape == w.shape, (g.shape, w.shape)
     if g.size == 0:
-        return dict(dtype=dtype, n=0, max_abs=0.0, mean_abs=0.0, max_ratio=0.0, mean_ratio=0.0, rms_ref=0.0,
-                    finite=True)
+        return dict(dtype=dtype, n=0, max_abs=0.0, mean_abs=0.0, max_ratio=0.0, mean_ratio=0.0, max_abs_unit=0.0,
+                    rms_ref=0.0, finite=True)
     err = np.abs(g - w)
     hu = half_ulp(w, dtype)
     bound = max_abs + hu
+    # the elements at unit scale, where the store's rounding is small next to
+    # the absolute bar: their largest error shows the arithmetic's own margin
+    unit = np.abs(w) <= 1.0
     return dict(dtype=dtype, n=int(g.size), max_abs=float(err.max()), mean_abs=float(err.mean()),
                 max_ratio=float((err / bound).max()), mean_ratio=float(err.mean() / (mean_abs + hu.mean())),
+                max_abs_unit=float(err[unit].max()) if unit.any() else 0.0,
                 rms_ref=float(np.sqrt(np.mean(w * w))), finite=bool(np.all(np.isfinite(g))))
 
 
