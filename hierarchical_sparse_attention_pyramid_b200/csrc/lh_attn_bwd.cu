@@ -104,8 +104,11 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + 127) / 128;
-  const int kt = (int)blockIdx.x;  // key tile; small kt = most query tiles, launched first
-  const int bh = (int)blockIdx.y;
+  // one CTA per (key tile, head), tile-major: small kt (most query tiles) of
+  // every head is started first, the short tiles fill the tail
+  const int BHn = (int)(gridDim.x / (unsigned)n_qt);
+  const int kt = (int)(blockIdx.x / (unsigned)BHn);
+  const int bh = (int)(blockIdx.x % (unsigned)BHn);
   const int NJ = n_qt - kt;        // 128-query steps, from the diagonal tile on
 
   if (threadIdx.x == 0) {
@@ -393,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + 127) / 128;
-  const int qt = n_qt - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = (int)blockIdx.y;
+  // one CTA per (query tile, head), tile-major with the longest rows first
+  const int BHn = (int)(gridDim.x / (unsigned)n_qt);
+  const int qt = n_qt - 1 - (int)(blockIdx.x / (unsigned)BHn);
+  const int bh = (int)(blockIdx.x % (unsigned)BHn);
   const int NJ = qt + 1;  // key tiles up to the diagonal
 
   if (threadIdx.x == 0) {
@@ -629,17 +634,18 @@ template <int D>
 cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* lse, const float* delta, float* dqs,
                          float* dks, float* dvs, int* errw, float scale_log2, float scale, cudaStream_t st) {
   const unsigned n_qt = (unsigned)((S + 127) / 128);
+  if ((int64_t)n_qt * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
   int smem = KvSmem<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_kv_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreadsKV, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
+  attn_bwd_kv_kernel<D><<<dim3((unsigned)(n_qt * BH)), kThreadsKV, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
                                                                          errw, (int)S, scale_log2, scale);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   smem = QSmem<D>::kAlloc;
   e = cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_bwd_q_kernel<D><<<dim3(n_qt, (unsigned)BH), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dqs, errw,
+  attn_bwd_q_kernel<D><<<dim3((unsigned)(n_qt * BH)), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dqs, errw,
                                                                         (int)S, scale_log2, scale);
   return cudaGetLastError();
 }

@@ -78,8 +78,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + BM - 1) / BM;
   const int n_pairs = (n_qt + 1) / 2;
-  const int c = n_pairs - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = (int)blockIdx.y;
+  // one CTA per (tile pair, head), pair-major: the block scheduler starts
+  // blocks in index order, so every head's longest pairs run first and the
+  // short ones fill the tail
+  const int BHn = (int)(gridDim.x / (unsigned)n_pairs);
+  const int c = n_pairs - 1 - (int)(blockIdx.x / (unsigned)BHn);
+  const int bh = (int)(blockIdx.x % (unsigned)BHn);
   const int qtile[2] = {2 * c, 2 * c + 1};
   const bool hasB = qtile[1] < n_qt;
   const int last[2] = {qtile[0], hasB ? qtile[1] : -1};  // last key tile of each query tile
@@ -384,7 +388,8 @@ cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const 
     return cudaErrorInvalidValue;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   const int64_t n_qt = (S + BM - 1) / BM;
-  const dim3 grid((unsigned)((n_qt + 1) / 2), (unsigned)BH);
+  if (((n_qt + 1) / 2) * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
+  const dim3 grid((unsigned)(((n_qt + 1) / 2) * BH));
   if (d == 128) {
     const int smem = FwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
