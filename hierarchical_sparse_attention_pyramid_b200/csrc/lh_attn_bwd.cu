@@ -17,8 +17,9 @@
 //   read, and the MMA warp adds dV += P^T dO_j and dK += dS^T Q_j with both A
 //   operands read from TMEM.  The next step's S^T is issued right after dV(j)
 //   and its dP^T right after dK(j), so the tensor core works on one step's
-//   products while the compute warps turn the other's scores around.  Q_j,
-//   dO_j stream through a 2-slot ring.
+//   products while the compute warps turn the other's scores around.  Q_j
+//   streams through a 3-slot ring (it is needed first, by S^T(j), and held
+//   longest, until dK(j)), dO_j through a 2-slot ring.
 //
 // attn_bwd_q_kernel (dQs) - one CTA per 128-row query tile; it steps over the
 //   128-key tiles up to the diagonal.  S = Q K_j^T runs two tiles ahead into a
@@ -67,17 +68,21 @@ __device__ __forceinline__ void store_pair_chunk(uint32_t taddr, const uint32_t 
 // ===========================================================================
 // dKs, dVs
 // ===========================================================================
+// 224 KB of tiles at D = 128: with the vectors and barriers the layout fills
+// the 227 KB a CTA can have only without alignment slack, so the kernel
+// relies on the dynamic shared memory starting 1024-byte aligned (it does
+// when the kernel has no static shared memory) and checks that it does.
 template <int D>
 struct KvSmem {
   static constexpr int kTile = D / 64 * kRegion;         // one 128-row tile: K, V, Q_j or dO_j
   static constexpr int oK = 0;
   static constexpr int oV = oK + kTile;
-  static constexpr int oRing = oV + kTile;               // 2 slots of (Q_j, dO_j)
-  static constexpr int kSlot = 2 * kTile;
-  static constexpr int oVec = oRing + 2 * kSlot;         // [2][256] floats: LSE*log2e [128], Delta [128]
+  static constexpr int oQ = oV + kTile;                  // 3 slots of Q_j
+  static constexpr int oO = oQ + 3 * kTile;              // 2 slots of dO_j
+  static constexpr int oVec = oO + 2 * kTile;            // [2][256] floats: LSE*log2e [128], Delta [128]
   static constexpr int oBar = oVec + 2048;
   static constexpr int kBytes = oBar + 256;
-  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kAlloc = kBytes;
 };
 
 template <int D>
@@ -87,17 +92,23 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
                        const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dK,
                        float* __restrict__ dV, int* errw, int S, float scale_log2, float scale) {
   using Lay = KvSmem<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (reinterpret_cast<uintptr_t>(smem_raw) & 1023) {  // the layout has no slack to align it
+    if (threadIdx.x == 0) report_error(errw, ERRW_BOUNDS);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::oBar);
   uint64_t* bKV = bars + 0;        // K, V landed
-  uint64_t* bLoad = bars + 1;      // [2] Q_j, dO_j of a ring slot landed
-  uint64_t* bSlotFree = bars + 3;  // [2] dV, dK products done with a slot
-  uint64_t* bS = bars + 5;         // S^T of the step in TMEM
-  uint64_t* bDP = bars + 6;        // dP^T of the step in TMEM
-  uint64_t* bP = bars + 7;         // P^T written back (one arrival per compute thread)
-  uint64_t* bDS = bars + 8;        // dS^T written back (one arrival per compute thread)
-  uint64_t* bDone = bars + 9;      // every product done
+  uint64_t* bQload = bars + 1;     // [3] Q_j of a slot landed
+  uint64_t* bQfree = bars + 4;     // [3] dK product done with a Q slot
+  uint64_t* bOload = bars + 7;     // [2] dO_j of a slot landed
+  uint64_t* bOfree = bars + 9;     // [2] dV product done with a dO slot
+  uint64_t* bS = bars + 11;        // S^T of the step in TMEM
+  uint64_t* bDP = bars + 12;       // dP^T of the step in TMEM
+  uint64_t* bP = bars + 13;        // P^T written back (one arrival per compute thread)
+  uint64_t* bDS = bars + 14;       // dS^T written back (one arrival per compute thread)
+  uint64_t* bDone = bars + 15;     // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
   float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);
@@ -113,9 +124,13 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bKV, 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&bQload[i], 1);
+      mbar_init(&bQfree[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bLoad[i], 1);
-      mbar_init(&bSlotFree[i], 1);
+      mbar_init(&bOload[i], 1);
+      mbar_init(&bOfree[i], 1);
     }
     mbar_init(bS, 1);
     mbar_init(bDP, 1);
@@ -143,15 +158,16 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
         tma_load_3d(smem + Lay::oV + c * kRegion, &tmV, bKV, c * 64, kt * 128, bh);
       }
       for (int j = 0; j < NJ; ++j) {
-        const int slot = j & 1;
-        if (j >= 2 && !mbar_wait(&bSlotFree[slot], ((j >> 1) - 1) & 1, abort_flag)) break;
+        const int qs = j % 3, os = j & 1;
         const int q0 = (kt + j) * 128;
-        uint8_t* base = smem + Lay::oRing + slot * Lay::kSlot;
-        mbar_expect_tx(&bLoad[slot], 2 * 128 * D * 2);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + c * kRegion, &tmQ, &bLoad[slot], c * 64, q0, bh);
-          tma_load_3d(base + Lay::kTile + c * kRegion, &tmO, &bLoad[slot], c * 64, q0, bh);
-        }
+        if (j >= 3 && !mbar_wait(&bQfree[qs], ((j / 3) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&bQload[qs], 128 * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oQ + qs * Lay::kTile + c * kRegion, &tmQ, &bQload[qs], c * 64, q0, bh);
+        if (j >= 2 && !mbar_wait(&bOfree[os], ((j >> 1) - 1) & 1, abort_flag)) break;
+        mbar_expect_tx(&bOload[os], 128 * D * 2);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + Lay::oO + os * Lay::kTile + c * kRegion, &tmO, &bOload[os], c * 64, q0, bh);
       }
     }
   } else if (warp == 17) {
@@ -162,39 +178,43 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     {  // the whole warp; one elected lane issues each instruction
       constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S^T, dP^T: N = 128 queries
       constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dV, dK: A from TMEM, B MN-major
-      const uint32_t sRing = smem_u32(smem + Lay::oRing);
+      const uint32_t sQ = smem_u32(smem + Lay::oQ), sO = smem_u32(smem + Lay::oO);
       const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
       const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
-      const uint64_t kRing = sdesc_sw128(sRing, 16, 1024);
-      const uint64_t mRing = sdesc_sw128(sRing, kRegion, 1024);
-      auto wait_load = [&](int j) -> bool { return mbar_wait_warp(&bLoad[j & 1], (j >> 1) & 1, abort_flag); };
+      const uint64_t kQ = sdesc_sw128(sQ, 16, 1024), mQ = sdesc_sw128(sQ, kRegion, 1024);
+      const uint64_t kO = sdesc_sw128(sO, 16, 1024), mO = sdesc_sw128(sO, kRegion, 1024);
+      auto wait_q = [&](int j) -> bool { return mbar_wait_warp(&bQload[j % 3], (j / 3) & 1, abort_flag); };
+      auto wait_o = [&](int j) -> bool { return mbar_wait_warp(&bOload[j & 1], (j >> 1) & 1, abort_flag); };
       auto issue_s = [&](int j) {
-        const uint32_t qo = ((j & 1) * Lay::kSlot) >> 4;
+        const uint32_t qo = ((j % 3) * Lay::kTile) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
-          umma_bf16_w(tmem + tS, kK + at, kRing + qo + at, idF, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + tS, kK + at, kQ + qo + at, idF, kk > 0 ? 1u : 0u);
         }
         umma_commit_w(bS);
       };
       auto issue_dp = [&](int j) {
-        const uint32_t oo = ((j & 1) * Lay::kSlot + Lay::kTile) >> 4;
+        const uint32_t oo = ((j & 1) * Lay::kTile) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
-          umma_bf16_w(tmem + tDP, kV + at, kRing + oo + at, idF, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + tDP, kV + at, kO + oo + at, idF, kk > 0 ? 1u : 0u);
         }
         umma_commit_w(bDP);
       };
-      bool ok = mbar_wait_warp(bKV, 0, abort_flag) && wait_load(0);
+      bool ok = mbar_wait_warp(bKV, 0, abort_flag) && wait_q(0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
+        ok = wait_o(0);
+      }
+      if (ok) {
+        tc_fence_after();
         issue_dp(0);
       }
       for (int j = 0; ok && j < NJ; ++j) {
-        const int slot = j & 1;
-        const uint32_t qo = (slot * Lay::kSlot) >> 4, oo = (slot * Lay::kSlot + Lay::kTile) >> 4;
+        const uint32_t qo = ((j % 3) * Lay::kTile) >> 4, oo = ((j & 1) * Lay::kTile) >> 4;
         // dV += P^T dO_j (16 queries per MMA; hi of chunk kk/2 at +(kk&1)*8, lo at +16)
         if (!mbar_wait_warp(bP, j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -202,12 +222,13 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t bo = mRing + oo + ((kk * 2048) >> 4);
+          const uint64_t bo = mO + oo + ((kk * 2048) >> 4);
           umma_bf16_tmem_a_w(tmem + tDV, a, bo, idG, acc);
           umma_bf16_tmem_a_w(tmem + tDV, a + 16, bo, idG, 1u);
         }
+        umma_commit_w(&bOfree[j & 1]);  // dV(j) was the last reader of dO_j
         if (j + 1 < NJ) {
-          if (!wait_load(j + 1)) { ok = false; break; }
+          if (!wait_q(j + 1)) { ok = false; break; }
           tc_fence_after();
           issue_s(j + 1);
         }
@@ -218,12 +239,16 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t a = tmem + tDP + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t bq = mRing + qo + ((kk * 2048) >> 4);
+          const uint64_t bq = mQ + qo + ((kk * 2048) >> 4);
           umma_bf16_tmem_a_w(tmem + tDK, a, bq, idG, acc);
           umma_bf16_tmem_a_w(tmem + tDK, a + 16, bq, idG, 1u);
         }
-        umma_commit_w(&bSlotFree[slot]);
-        if (j + 1 < NJ) issue_dp(j + 1);
+        umma_commit_w(&bQfree[j % 3]);  // dK(j) was the last reader of Q_j
+        if (j + 1 < NJ) {
+          if (!wait_o(j + 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(j + 1);
+        }
       }
       if (ok) umma_commit_w(bDone);
     }
