@@ -654,6 +654,7 @@ def run_stage(args, world, rank, local):
     qs, ks, vs, dos = (torch.randn(BH, S, d, generator=g, device=dev).to(torch.bfloat16) for _ in range(4))
     ws = torch.zeros(_lib.ERR_WORD_BYTES, dtype=torch.uint8, device=dev)
     os_, lse = lh.attn_fwd(layer, qs, ks, vs, ws)
+    dos = dos.to(torch.float16)  # the backward takes dOs as fp16 holding bf16 values (exact)
     delta = (dos.float() * os_).sum(-1)
     calls = {"attn_fwd": lambda: lh.attn_fwd(layer, qs, ks, vs, ws),
              "attn_bwd": lambda: lh.attn_bwd(layer, qs, ks, vs, lse, dos, delta, ws)}

@@ -158,7 +158,7 @@ def scatter_back(layer: Layer, os_, slot_of):
 
 def scatter_back_adjoint(layer: Layer, dy, seq_map, os_):
     BH, S, d = os_.shape
-    dos = _empty((BH, S, d), torch.bfloat16, dy.device)
+    dos = _empty((BH, S, d), torch.float16, dy.device)  # bf16-rounded values, stored as fp16
     delta = _empty((BH, S), torch.float32, dy.device)
     call("lh_scatter_back_adjoint", ctypes.byref(layer.cfg()), _p(dy), _p(seq_map), _p(os_), _p(dos), _p(delta),
          _stream())
@@ -239,7 +239,8 @@ def backward(layer: Layer, dy, bufs: Buffers, grads=None):
 
 
 def check_error(bufs_or_ws) -> None:
-    """Synchronise and raise if a kernel reported a timeout or a bad index."""
+    """Synchronise and raise if a kernel reported a timeout, a bad index, or a
+    value beyond the fp16 range where the backward keeps one (dOs, Vs)."""
     ws = bufs_or_ws.ws if isinstance(bufs_or_ws, Buffers) else bufs_or_ws
     call("lh_check_error", _p(ws), _stream())
 

@@ -456,6 +456,7 @@ lh_status lh_check_error(void* ws, lh_stream_t stream) {
   LH_CUDA(cudaMemset(ws, 0, sizeof(int)), "lh_check_error");
   if (word & ERRW_TIMEOUT) return fail(LH_ERR_TIMEOUT, "a bounded device wait ran out");
   if (word & ERRW_BOUNDS) return fail(LH_ERR_DEVICE, "a device-side index check failed");
+  if (word & ERRW_RANGE) return fail(LH_ERR_DEVICE, "a value kept in fp16 by the backward (dOs or Vs) exceeds 65504");
   return LH_OK;
 }
 

@@ -5,8 +5,14 @@
 // With P = softmax(Qs Ks^T / sqrt(d)) (causal) recomputed from the saved LSE,
 //   dVs = P^T dOs,  dP = dOs Vs^T,  dS = P * (dP - Delta) / sqrt(d),
 //   dQs = dS Ks,    dKs = dS^T Qs,  Delta = rowsum(dOs * Os).
-// P and dS enter their products as bf16 (hi + lo) pairs, so the bf16
-// roundings of the probabilities and of dS do not show in the gradients.
+// dS enters its products as a bf16 (hi + lo) pair, so its rounding does not
+// show in dQ and dK.  P enters dV = P^T dO as one fp16 value (11 significant
+// bits; P is in [0, 1] and its products with dO are summed with positive
+// weights, so no cancellation amplifies that rounding), and dV and dP = dO V^T
+// are fp16 products: dOs arrives in fp16 and the dK/dV kernel converts its V
+// tile to fp16 in shared memory (both hold bf16 values, exact in fp16 up to
+// 65504; larger ones set the range bit of the error word).  The dQ kernel
+// converts its dO tile back to bf16 for dP = dO V^T.
 //
 // Two kernels, each writing its gradient once (no atomics):
 //
@@ -109,6 +115,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
   uint64_t* bP = bars + 13;        // P^T written back (one arrival per compute thread)
   uint64_t* bDS = bars + 14;       // dS^T written back (one arrival per compute thread)
   uint64_t* bDone = bars + 15;     // every product done
+  uint64_t* bVconv = bars + 16;    // V converted to fp16 in shared memory (one arrival per compute thread)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
   float* sVec = reinterpret_cast<float*>(smem + Lay::oVec);
@@ -137,6 +144,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     mbar_init(bP, kComputeKV);
     mbar_init(bDS, kComputeKV);
     mbar_init(bDone, 1);
+    mbar_init(bVconv, kComputeKV);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -176,8 +184,10 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     // columns dV(j) has read: the tensor core runs in issue order), dK(j) once
     // dS^T(j) is back, dP^T(j+1) (over the dS^T columns dK(j) has read).
     {  // the whole warp; one elected lane issues each instruction
-      constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S^T, dP^T: N = 128 queries
-      constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dV, dK: A from TMEM, B MN-major
+      constexpr uint32_t idF = idesc_bf16(128, 128, false, false);  // S^T = K Q^T: N = 128 queries
+      constexpr uint32_t idF16 = idesc_f16(128, 128, false, false); // dP^T = V dO^T, fp16 both
+      constexpr uint32_t idG = idesc_bf16(128, D, false, true);     // dK: A (dS^T) from TMEM, B MN-major
+      constexpr uint32_t idG16 = idesc_f16(128, D, false, true);    // dV: A (P^T, fp16) from TMEM, dO fp16
       const uint32_t sQ = smem_u32(smem + Lay::oQ), sO = smem_u32(smem + Lay::oO);
       const uint64_t kK = sdesc_sw128(smem_u32(smem + Lay::oK), 16, 1024);
       const uint64_t kV = sdesc_sw128(smem_u32(smem + Lay::oV), 16, 1024);
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t at = ((kk >> 2) * kRegion + (kk & 3) * 32) >> 4;
-          umma_bf16_w(tmem + tDP, kV + at, kO + oo + at, idF, kk > 0 ? 1u : 0u);
+          umma_bf16_w(tmem + tDP, kV + at, kO + oo + at, idF16, kk > 0 ? 1u : 0u);
         }
         umma_commit_w(bDP);
       };
@@ -207,7 +217,8 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        ok = wait_o(0);
+        // dP^T reads V as fp16: after the compute warps have converted it
+        ok = wait_o(0) && mbar_wait_warp(bVconv, 0, abort_flag);
       }
       if (ok) {
         tc_fence_after();
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       }
       for (int j = 0; ok && j < NJ; ++j) {
         const uint32_t qo = ((j % 3) * Lay::kTile) >> 4, oo = ((j & 1) * Lay::kTile) >> 4;
-        // dV += P^T dO_j (16 queries per MMA; hi of chunk kk/2 at +(kk&1)*8, lo at +16)
+        // dV += P^T dO_j (16 queries per MMA: P^T of chunk kk/2, fp16, at +(kk&1)*8)
         if (!mbar_wait_warp(bP, j & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -223,8 +234,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
           const uint32_t a = tmem + tS + (kk >> 1) * 32 + (kk & 1) * 8;
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           const uint64_t bo = mO + oo + ((kk * 2048) >> 4);
-          umma_bf16_tmem_a_w(tmem + tDV, a, bo, idG, acc);
-          umma_bf16_tmem_a_w(tmem + tDV, a + 16, bo, idG, 1u);
+          umma_bf16_tmem_a_w(tmem + tDV, a, bo, idG16, acc);
         }
         umma_commit_w(&bOfree[j & 1]);  // dV(j) was the last reader of dO_j
         if (j + 1 < NJ) {
@@ -270,6 +280,29 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     float vec_next = ct < 256 ? vec_raw(0) : 0.f;
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const uint64_t sc2 = f2_pack(scale, scale);
+    // V to fp16 in place (the operand type of dP^T = V dO^T): every thread
+    // converts its share of the tile once the TMA has landed it
+    ok = mbar_wait(bKV, 0, abort_flag);
+    if (ok) {
+      constexpr int kPer = Lay::kTile / 16 / kComputeKV;  // 16-byte words per thread
+      uint4* vt = reinterpret_cast<uint4*>(smem + Lay::oV);
+      bool in_range = true;
+#pragma unroll
+      for (int w = 0; w < kPer; ++w) {
+        uint4 u = vt[ct + w * kComputeKV];
+        uint32_t* e = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float lo = __uint_as_float(e[c] << 16), hi = __uint_as_float(e[c] & 0xffff0000u);
+          in_range &= fabsf(lo) <= 65504.f && fabsf(hi) <= 65504.f;
+          e[c] = pack_f16x2(lo, hi);
+        }
+        vt[ct + w * kComputeKV] = u;
+      }
+      if (!in_range) report_error(errw, ERRW_RANGE);
+      fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+    }
+    mbar_arrive(bVconv);
     for (int j = 0; j < NJ; ++j) {
       const int b = j & 1;
       const float vec_cur = vec_next;
@@ -286,15 +319,14 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       ok = __all_sync(0xffffffffu, ok && mbar_wait(bS, j & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
-      // P^T as bf16 pairs over the 32 S^T columns just read (hi in the first
-      // 16, lo in the last 16); dV starts on it while dP^T is still being
-      // computed
+      // P^T in fp16 over the first 16 of the 32 S^T columns just read; dV
+      // starts on it while dP^T is still being computed
       float p[32];
       {
         uint32_t sr[32];
         tmem_ld32(tl + tS + g * 32, sr);
         tmem_ld_wait();
-        uint32_t phi[16], plo[16];
+        uint32_t ph[16];
         // queries before the key are masked on the diagonal tile only
         auto p_pass = [&](auto masked) {
 #pragma unroll
@@ -312,12 +344,12 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
             }
             p[e] = pa;
             p[e + 1] = pb;
-            split_bf16x2(pa, pb, phi[e >> 1], plo[e >> 1]);
+            ph[e >> 1] = pack_f16x2(pa, pb);
           }
         };
         if (diag) p_pass(std::true_type{});
         else p_pass(std::false_type{});
-        store_pair_chunk(tl + tS + g * 32, phi, plo);
+        tmem_st16(tl + tS + g * 32, ph);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -416,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bDP = bars + 15;    // dP of the current key tile in TMEM
   uint64_t* bPS = bars + 16;    // dS written over the tile's S columns (256 arrivals)
   uint64_t* bDone = bars + 17;  // every product done
+  uint64_t* bOconv = bars + 18; // dO converted to bf16 in shared memory (one arrival per compute thread)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::oBar + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
@@ -442,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bDP, 1);
     mbar_init(bPS, kCompute);
     mbar_init(bDone, 1);
+    mbar_init(bOconv, kCompute);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -514,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        ok = mbar_wait_warp(&bV[0], 0, abort_flag);
+        // dP reads dO as bf16: after the compute warps have converted it
+        ok = mbar_wait_warp(&bV[0], 0, abort_flag) && mbar_wait_warp(bOconv, 0, abort_flag);
       }
       if (ok) {
         tc_fence_after();
@@ -561,7 +596,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float del = qg < S ? Delta[(int64_t)bh * S + qg] : 0.f;
     const uint64_t c2 = f2_pack(scale_log2, scale_log2), sc2 = f2_pack(scale, scale);
     const uint64_t nl2 = f2_pack(-lse, -lse), d2 = f2_pack(del, del);
-    bool ok = true;
+    // dO arrives in fp16 (the operand type of the dK/dV kernel); its values
+    // are bf16 values, so converting the tile back to bf16 in place is exact
+    bool ok = mbar_wait(bQO, 0, abort_flag);
+    if (ok) {
+      constexpr int kPer = Lay::kTile / 16 / kCompute;  // 16-byte words per thread
+      uint4* ot = reinterpret_cast<uint4*>(smem + Lay::oO);
+#pragma unroll
+      for (int w = 0; w < kPer; ++w) {
+        uint4 u = ot[threadIdx.x + w * kCompute];
+        uint32_t* e = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&e[c]));
+          e[c] = pack_bf16x2(f.x, f.y);
+        }
+        ot[threadIdx.x + w * kCompute] = u;
+      }
+      fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+    }
+    mbar_arrive(bOconv);
     for (int j = 0; j < NJ; ++j) {
       const int b = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bS[b], (j >> 1) & 1, abort_flag));

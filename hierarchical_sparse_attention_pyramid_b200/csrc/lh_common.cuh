@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "lh.h"
@@ -28,7 +29,9 @@ struct Dims {
 };
 
 // error word bits (first int32 of ws)
-enum : int { ERRW_TIMEOUT = 1, ERRW_BOUNDS = 2 };
+// ERRW_RANGE: a value the backward keeps in fp16 (dOs, Vs) is outside fp16's
+// finite range (|x| > 65504)
+enum : int { ERRW_TIMEOUT = 1, ERRW_BOUNDS = 2, ERRW_RANGE = 4 };
 
 __device__ __forceinline__ void report_error(int* errw, int bits) {
   if (errw) atomicOr(errw, bits);

@@ -268,13 +268,17 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 
 // ---------------------------------------------------------------------------
 // scatter-back adjoint: dOs[s] = sum_{j in R(l,i)} dY_j (fp32), Delta[s] = dOs[s] . Os[s]
-// one warp per slot, R rows per warp instruction
+// one warp per slot, R rows per warp instruction.  dOs is rounded once to
+// bf16 (the attention's 16-bit input) and stored as fp16, which holds every
+// bf16 value of magnitude up to 65504 exactly; the attention backward reads it
+// as the fp16 operand of its dV and dP products.  A larger magnitude sets the
+// range bit of the error word.
 // ---------------------------------------------------------------------------
 struct ScatterAdjArgs {
   const void* dy;
   const int32_t* seq_map;
   const float* os;
-  __nv_bfloat16* dos;
+  __half* dos;
   float* delta;
   int* errw;
   int64_t BH, N, S;
@@ -326,16 +330,21 @@ __global__ void __launch_bounds__(kSadjWarps * 32) scatter_adjoint_kernel(Scatte
   for (int c = 0; c < VE; ++c)
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) acc[c] += __shfl_xor_sync(kFull, acc[c], o);
-  // round to bf16 once; Delta from the rounded values and the bf16 Os
-  __nv_bfloat16 h[VE];
+  // round to bf16 once (stored as fp16, exact in range); Delta from the
+  // rounded values and the fp32 Os
+  __half h[VE];
   float o_row[VE];
   load_f32<VE>(a.os + (bh * a.S + s) * D + cv * VE, o_row);
   float dot = 0.f;
+  bool in_range = true;
 #pragma unroll
   for (int c = 0; c < VE; ++c) {
-    h[c] = __float2bfloat16_rn(acc[c]);
-    dot = fmaf(__bfloat162float(h[c]), o_row[c], dot);
+    const float r = __bfloat162float(__float2bfloat16_rn(acc[c]));
+    in_range &= fabsf(r) <= 65504.f;
+    h[c] = __float2half_rn(r);
+    dot = fmaf(r, o_row[c], dot);
   }
+  if (!in_range) report_error(a.errw, ERRW_RANGE);
 #pragma unroll
   for (int o = LPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(kFull, dot, o);
   if (lr == 0) {
@@ -428,7 +437,7 @@ cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t*
   a.dy = dy;
   a.seq_map = seq_map;
   a.os = os;
-  a.dos = static_cast<__nv_bfloat16*>(dos);
+  a.dos = static_cast<__half*>(dos);
   a.delta = delta;
   a.errw = errw;
   a.BH = D.BH; a.N = D.N; a.S = D.S;

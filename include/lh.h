@@ -17,7 +17,8 @@
  *    parameter says "host", and must be 16-byte aligned.
  *  - Layouts are dense row-major.  "BH" = B*H flattened; Q, K, V, Y, dY, dQ,
  *    dK, dV are [B][H][N][d] in cfg->dtype.  The gathered sequence tensors
- *    Qs, Ks, Vs, dOs are [BH][S][d] bf16; Os, dQs, dKs, dVs are [BH][S][d]
+ *    Qs, Ks, Vs are [BH][S][d] bf16, dOs [BH][S][d] fp16 (holding bf16
+ *    values); Os, dQs, dKs, dVs are [BH][S][d]
  *    fp32; LSE and Delta are [BH][S] fp32.
  *  - Support: d in {64, 128}; p a power of two >= 2; 1 <= L <= 8;
  *    N divisible by p^(L-1); N < 2^28; k >= 1; B*H <= 65535 * 65535.
@@ -105,7 +106,7 @@ typedef struct {
   size_t norms_bytes;   /* [2][BH][N] fp32 */
   size_t topk_ws_bytes; /* ws of lh_score_topk */
   size_t sel_bytes;     /* [BH][sel_per_head] int32 */
-  size_t seq_bytes;     /* one of qs/ks/vs/dos: [BH][S][d] bf16 */
+  size_t seq_bytes;     /* one of qs/ks/vs/dos: [BH][S][d], 2 bytes an element */
   size_t os_bytes;      /* os: [BH][S][d] fp32 */
   size_t seq_map_bytes; /* [BH][S] int32 */
   size_t slot_of_bytes; /* [BH][pyr_entries] int32 */
@@ -229,10 +230,15 @@ lh_status lh_attn_fwd(const lh_config *cfg, int64_t S, const void *qs, const voi
                       float *lse, void *ws, lh_stream_t stream);
 
 /* Stage 4 backward.  Cite: LH-summary "Method" step 5 (the gradient flows
- * back through the attention kernel).  P and dS enter their products as bf16
- * hi + lo pairs, so dQs, dKs, dVs keep fp32 accuracy for bf16 inputs.
- * In:  qs, ks, vs, lse from the forward; dos [BH][S][d] bf16 and
- *      delta [BH][S] fp32 (rowsum(dOs * Os)) from lh_scatter_back_adjoint.
+ * back through the attention kernel).  dS enters dQ and dK as a bf16 hi + lo
+ * pair (fp32 accuracy); P enters dV = P^T dOs as one fp16 value (P is in
+ * [0, 1], summed with positive weights), and dV and dP^T = Vs dOs^T are fp16
+ * products (the kernel converts its Vs tile to fp16; Vs and dOs hold bf16
+ * values, exact in fp16 up to magnitude 65504 - a larger one sets the error
+ * word's range bit, reported by lh_check_error as LH_ERR_DEVICE).
+ * In:  qs, ks, vs (bf16), lse from the forward; dos [BH][S][d] fp16 holding
+ *      bf16 values and delta [BH][S] fp32 (rowsum(dOs * Os)), both as
+ *      lh_scatter_back_adjoint writes them.
  * Out: dqs, dks, dvs [BH][S][d] fp32, each row written once (no accumulation).
  * ws: at least attn_bwd_ws_bytes (error word). */
 lh_status lh_attn_bwd(const lh_config *cfg, int64_t S, const void *qs, const void *ks, const void *vs,
@@ -251,8 +257,10 @@ lh_status lh_scatter_back(const lh_config *cfg, const float *os, const int32_t *
 
 /* Stage 5 backward: dOs[slot(l,i)] = sum of dY_j over j in R(l, i) (fp32,
  * rounded once to bf16), and delta[s] = sum_c dOs[s,c] * Os[s,c] (fp32, from
- * the bf16 dOs and the fp32 Os).  Cite: LH-summary "Method" step 5.
- * Out: dos [BH][S][d] bf16, delta [BH][S] fp32. */
+ * the rounded dOs and the fp32 Os).  Cite: LH-summary "Method" step 5.
+ * Out: dos [BH][S][d] fp16 (the bf16-rounded values, exact in fp16; a
+ *      magnitude above 65504 sets the error word's range bit, reported by
+ *      lh_check_error as LH_ERR_DEVICE), delta [BH][S] fp32. */
 lh_status lh_scatter_back_adjoint(const lh_config *cfg, const void *dy, const int32_t *seq_map, const float *os,
                                   void *dos, float *delta, lh_stream_t stream);
 

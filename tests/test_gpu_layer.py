@@ -70,3 +70,25 @@ def test_autograd_function_matches_direct_calls():
     torch.cuda.synchronize()
     assert torch.equal(y.detach(), y2)
     assert torch.equal(q.grad, dq2) and torch.equal(k.grad, dk2) and torch.equal(v.grad, dv2)
+
+
+@pytest.mark.parametrize("what", ["dy", "v"])
+def test_fp16_range_of_the_backward_is_reported(what):
+    """dOs and Vs enter the backward's dV and dP products in fp16: a value
+    beyond 65504 is reported as LH_ERR_DEVICE by check_error, not passed on
+    silently."""
+    w, x, _ = case("ragged")
+    L = lh.Layer.of(w)
+    q, k, v, dy = (x[n] for n in ("q", "k", "v", "dy"))
+    if what == "dy":
+        dy = torch.full_like(dy, 30000.0)  # a top-level slot sums 4 rows: 120000
+    else:
+        v = torch.full_like(v, 70000.0)
+    y, bufs = lh.forward(L, q, k, v)
+    lh.backward(L, dy, bufs)
+    with pytest.raises(Exception, match="LH_ERR_DEVICE"):
+        lh.check_error(bufs)
+    # the word is cleared and ordinary inputs run clean again
+    y, bufs = lh.forward(L, x["q"], x["k"], x["v"])
+    lh.backward(L, x["dy"], bufs)
+    lh.check_error(bufs)
