@@ -21,7 +21,7 @@ HEADER = os.path.join(ROOT, "include", "lh.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(lh_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(lh_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -36,7 +36,7 @@ def test_header_functions_are_exported(lib):
     names = declared_functions()
     assert len(names) >= 15
     out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (lh_[a-z_]+)$", out, flags=re.M))
+    exported = set(re.findall(r"\bT (lh_[a-z0-9_]+)$", out, flags=re.M))
     missing = [n for n in names if n not in exported]
     assert not missing, missing
     for n in names:
