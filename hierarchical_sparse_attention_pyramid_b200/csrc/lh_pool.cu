@@ -296,6 +296,212 @@ __global__ void __launch_bounds__(kPoolWarps * 32, 1) pool_kernel(PoolArgs a) {
   }
 }
 
+// The same pass for bf16 rows of 128 channels, with about a third of the
+// instructions per row (the pass above issues on ~80% of its cycles there).
+// Each half-warp takes every other row of the warp's task: lane l holds
+// channels [8 (l mod 16), +8) of row 2u + (l div 16) at step u, so one
+// 16-byte shared-memory load per lane moves two rows and each half-warp
+// reduces its own row's norm over 16 lanes.  The half-warps keep partial
+// sums of the levels (each holds the rows of its parity), which are linear,
+// and add them together only when a materialised entry is written.  Rows are
+// summed straight into the lowest materialised level (first_level): the
+// levels below it are never formed.
+// Warps per SM x ring stages of 4 KB, measured on the 512K-token layer (16
+// heads): 16 x 2: 1.016 ms; 20 x 2: 1.038; 24 x 2: 1.115 (at 80 registers,
+// with spills); 16 x 3: 1.087; 12 x 2: 1.101; 12 x 4: 1.103; 8 x 4: 1.354.
+// The pass above takes 1.148 ms on the same layer.
+constexpr int kPairWarps = 16;
+constexpr int kPairStages = 2;
+template <int NL>
+__global__ void __launch_bounds__(kPairWarps * 32, 1) pool_pairs_kernel(PoolArgs a) {
+  constexpr int D = 128;
+  constexpr int ROWB = D * 2;
+  constexpr int SR = kStageBytes / ROWB;  // 16 rows per stage
+  constexpr int NPAIR = SR / 2;           // two rows per step
+  static_assert(SR % 2 == 0 && NPAIR == 8, "stage rows");
+  extern __shared__ __align__(128) uint8_t pool_ring[];
+  __shared__ __align__(8) uint64_t pool_bars[kPairWarps][kPairStages];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4;
+  uint8_t* ring = pool_ring + warp * (kPairStages * kStageBytes);
+  uint64_t* bar = pool_bars[warp];
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < kPairStages; ++st) mbar_init(&bar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const int64_t nw = (int64_t)gridDim.x * kPairWarps;
+  const int64_t gw = (int64_t)blockIdx.x * kPairWarps + warp;
+  const int log2p = a.log2p, fl = a.first_level;
+  // a block of the lowest materialised level ends after `done` rows of the
+  // task when done & fl_mask == 0 (never when no level is materialised)
+  const int fl_mask = fl < NL ? (1 << (fl * log2p)) - 1 : -1;
+  // the norms are reduced every 4 steps: after the two halving stages of the
+  // reduction, lane l's partial belongs to step rid of the 4, and lanes with
+  // l mod 4 == 0 end with that row's whole sum
+  const int rid = ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+
+  const uint32_t tph = (uint32_t)a.tasks_per_head, ntasks = (uint32_t)a.tasks;
+  auto task_at = [&](uint32_t t, int& tensor, int64_t& bh, int64_t& row0) {
+    tensor = (int)(t % 3u);
+    const uint32_t rest = t / 3u;
+    bh = rest / tph;
+    row0 = (int64_t)(rest % tph) * a.task_rows;
+    return (int)min((int64_t)a.task_rows, a.N - row0);
+  };
+  uint32_t pt = (uint32_t)gw;
+  int pr = 0, prows = 0;
+  const uint8_t* psrc = nullptr;
+  auto producer_task = [&]() {
+    if (pt >= ntasks) return;
+    int tensor;
+    int64_t bh, row0;
+    prows = task_at(pt, tensor, bh, row0);
+    psrc = static_cast<const uint8_t*>(a.x[tensor]) + (bh * a.N + row0) * ROWB;
+  };
+  producer_task();
+  uint32_t pending = 0;
+  auto issue = [&](int sl) {
+    if (pt >= ntasks) return;
+    const int n = min(SR, prows - pr);
+    if (lane == 0) {
+      mbar_expect_tx(&bar[sl], (uint32_t)(n * ROWB));
+      bulk_load(ring + sl * kStageBytes, psrc + (int64_t)pr * ROWB, (uint32_t)(n * ROWB), &bar[sl]);
+    }
+    pending |= 1u << sl;
+    pr += SR;
+    if (pr >= prows) {
+      pr = 0;
+      pt += (uint32_t)nw;
+      producer_task();
+    }
+  };
+#pragma unroll
+  for (int st = 0; st < kPairStages; ++st) issue(st);
+
+  uint32_t phase = 0;
+  int slot = 0;
+  for (uint32_t t = (uint32_t)gw; t < ntasks; t += (uint32_t)nw) {
+    int tensor;
+    int64_t bh, row0;
+    const int rows = task_at(t, tensor, bh, row0);
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.pyr[tensor]) + bh * a.upper_entries * D + (lane & 15) * 8;
+    float* norm_out = a.norms + ((int64_t)tensor * a.BH + bh) * a.N + row0;
+    uint64_t run[4], acc[NL][4];  // this half's sums: the open block of level fl, and of the levels above it
+#pragma unroll
+    for (int i = 0; i < 4; ++i) run[i] = 0ull;
+#pragma unroll
+    for (int l = 0; l < NL; ++l)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[l][i] = 0ull;
+
+    // a block of level fl ended after `done` rows: write it and every level
+    // above that ends there, carrying each sum one level up
+    auto cascade = [&](int done) {
+      uint64_t sm[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sm[i] = run[i];
+        run[i] = 0ull;
+      }
+#pragma unroll
+      for (int l = 1; l < NL; ++l) {
+        if (l < fl) continue;
+        // both halves' parts of the entry, scaled by p^-l (exact) and rounded once
+        const float inv = __int_as_float((127 - l * log2p) << 23);
+        const uint64_t inv2 = f2_pack(inv, inv);
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float x0, x1;
+          f2_unpack(sm[i], x0, x1);
+          const uint64_t other = f2_pack(__shfl_xor_sync(kFull, x0, 16), __shfl_xor_sync(kFull, x1, 16));
+          float m0, m1;
+          f2_unpack(f2_mul(f2_add(sm[i], other), inv2), m0, m1);
+          ow[i] = pack_bf16x2(m0, m1);
+        }
+        const int64_t e_idx = ((row0 + done) >> (l * log2p)) - 1;
+        if (half == 0) *reinterpret_cast<uint4*>(dst + (a.upper_off[l] + e_idx) * D) = o;
+        if (l + 1 == NL) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[l + 1][i] = f2_add(acc[l + 1][i], sm[i]);
+        if ((done & ((1 << ((l + 1) * log2p)) - 1)) != 0) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sm[i] = acc[l + 1][i];
+          acc[l + 1][i] = 0ull;
+        }
+      }
+    };
+
+    // one stage: NPAIR steps of two rows; the norms of Q and K rows
+    auto stage_pass = [&](const uint4* st4, int r0, auto norm) {
+      constexpr bool kNorm = decltype(norm)::value;
+      float sq[4];
+#pragma unroll
+      for (int u = 0; u < NPAIR; ++u) {
+        const uint4 x = st4[u * 32];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint64_t q2 = 0ull;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t v2 = f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+          if constexpr (kNorm) q2 = f2_fma(v2, v2, q2);
+          run[i] = f2_add(run[i], v2);
+        }
+        if constexpr (kNorm) {
+          float qa, qb;
+          f2_unpack(q2, qa, qb);
+          sq[u & 3] = qa + qb;
+          if ((u & 3) == 3) {
+            // reduce-scatter of each half's 4 rows over its 16 lanes
+#pragma unroll
+            for (int hw = 2, b = 8; hw >= 1; hw >>= 1, b >>= 1) {
+              const bool up = lane & b;
+#pragma unroll
+              for (int i = 0; i < hw; ++i) {
+                const float send = up ? sq[i] : sq[i + hw];
+                const float keep = up ? sq[i + hw] : sq[i];
+                sq[i] = keep + __shfl_xor_sync(kFull, send, b);
+              }
+            }
+            float tot = sq[0] + __shfl_xor_sync(kFull, sq[0], 2);
+            tot += __shfl_xor_sync(kFull, tot, 1);
+            const int r = r0 + 2 * ((u & ~3) + rid) + half;
+            if ((lane & 3) == 0 && r < rows) norm_out[r] = sqrtf(tot);
+          }
+        }
+        const int done = r0 + 2 * u + 2;
+        if ((done & fl_mask) == 0 && done <= rows) cascade(done);
+      }
+    };
+
+    const bool want_norm = tensor < 2;
+    for (int r0 = 0; r0 < rows; r0 += SR) {
+      if (!mbar_wait_bounded_warp(&bar[slot], (phase >> slot) & 1u)) {
+        report_error(a.errw, ERRW_TIMEOUT);
+#pragma unroll 1
+        for (int st = 0; st < kPairStages; ++st)
+          if (st != slot && (pending >> st & 1u)) mbar_wait_bounded_warp(&bar[st], (phase >> st) & 1u);
+        return;
+      }
+      // rows of a stage past the task's end hold stale bytes: they only reach
+      // sums that are never written (no block ends past the task) and are
+      // reset with the next task, and their norms are not stored
+      const uint4* st4 = reinterpret_cast<const uint4*>(ring + slot * kStageBytes) + lane;
+      if (want_norm) stage_pass(st4, r0, std::true_type{});
+      else stage_pass(st4, r0, std::false_type{});
+      __syncwarp();  // every lane has read the stage before it is refilled
+      pending &= ~(1u << slot);
+      phase ^= 1u << slot;
+      issue(slot);
+      slot = slot + 1 == kPairStages ? 0 : slot + 1;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // adjoint: dX_t = sum_l [kept(l, t >> l log2p)] p^-l dXs[slot]  (fp32, rounded once)
 // 16-byte output lanes, R (1 or 2) rows per warp instruction; the rows of an
@@ -402,8 +608,33 @@ cudaError_t pool_launch(const PoolArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int NL>
+cudaError_t pool_pairs_launch(const PoolArgs& a, cudaStream_t st) {
+  constexpr int smem = kPairWarps * kPairStages * kStageBytes;
+  cudaError_t e = cudaFuncSetAttribute(pool_pairs_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int dev = 0, sms = 0, per_sm = 0;
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_pairs_kernel<NL>, kPairWarps * 32, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = std::min<int64_t>((int64_t)sms * std::max(per_sm, 1), (a.tasks + kPairWarps - 1) / kPairWarps);
+  pool_pairs_kernel<NL><<<(unsigned)blocks, kPairWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t pool_dispatch_L(int L, const PoolArgs& a, cudaStream_t st) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+    // the common layout: two rows per warp step (levels 1 to 4 in registers)
+    switch (L) {
+      case 2: return pool_pairs_launch<2>(a, st);
+      case 3: return pool_pairs_launch<3>(a, st);
+      case 4: return pool_pairs_launch<4>(a, st);
+      case 5: return pool_pairs_launch<5>(a, st);
+      default: break;
+    }
+  }
   switch (L) {
 #define LH_CASE(n) \
   case n: return pool_launch<T, D, n>(a, st);
