@@ -10,7 +10,7 @@
 // Entry (l, i) covers tokens [i p^l, (i+1) p^l); its key is
 // (e = (i+1) p^l - 1, -l) and its range is R(l,i) = [e, e + p^l).  The slot of
 // an entry is the number of kept entries with a smaller key, counted level by
-// level with binary searches over the sorted parent lists (or, when levels are
+// level with searches over the sorted parent lists (or, when levels are
 // selected directly, the sorted lists of kept entries), so no sort runs.
 #include "lh_common.cuh"
 
@@ -45,37 +45,76 @@ struct GatherArgs {
   int32_t kprime[LH_MAX_LEVELS];
   int L, log2p, first_level;
   int direct;  // sel lists the kept entries themselves (not parents)
+  // warp searches of the sorted lists: `rounds` rounds of 32 probes, the
+  // first at stride stride0 = 32^(rounds-1) >= every list's length / 32
+  int rounds, stride0;
 };
 
-// kept entries of level lv with index < X
-__device__ __forceinline__ int64_t kept_below(const GatherArgs& a, const int32_t* sel_h, int lv, int64_t X) {
-  if (X <= 0) return 0;
-  if (lv == a.L - 1) return min(X, a.level_len[lv]);
-  const int32_t* s = sel_h + a.sel_off[lv];
-  if (a.direct) {  // lower_bound of X in the sorted kept list
-    int lo = 0, hi = a.kprime[lv] << a.log2p;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if ((int64_t)s[mid] < X) lo = mid + 1;
-      else hi = mid;
+// Kept entries of every level whose key is below (e, -l), excluding level l
+// itself.  A coarser level lv > l counts its entries i' with (i'+1) p^lv <=
+// e + 1, a finer one those with (i'+1) p^lv <= e; the top level keeps all of
+// its entries.  The other levels search their sorted lists (the kept
+// parents, or the kept entries when levels are selected directly) with the
+// whole warp: a round probes 32 positions of every list at once, each round
+// at 1/32 of the previous stride, so a list of n entries takes ceil(log32 n)
+// rounds of one load per lane and level instead of log2 n dependent loads.
+template <int NL>
+__device__ __forceinline__ int64_t kept_below_warp(const GatherArgs& a, const int32_t* sel_h, int l, int64_t e,
+                                                   int lane) {
+  const int log2p = a.log2p;
+  const int top = NL - 1;
+  auto target = [&](int lv) -> int64_t { return (lv > l ? e + 1 : e) >> (lv * log2p); };
+  int64_t total = 0;
+  if (top != l) total += min(target(top), a.level_len[top]);
+  if constexpr (NL > 1) {
+    constexpr int K = NL - 1;
+    int tgt[K], rem[K], base[K], n[K], elem[K];
+#pragma unroll
+    for (int lv = 0; lv < K; ++lv) {
+      const int64_t X = target(lv);  // candidates below X (entries, or parents' children)
+      tgt[lv] = (int)(a.direct ? X : X >> log2p);
+      rem[lv] = a.direct ? 0 : (int)(X & ((1 << log2p) - 1));
+      n[lv] = lv == l ? 0 : (a.direct ? a.kprime[lv] << log2p : a.kprime[lv]);
+      base[lv] = 0;
+      elem[lv] = -1;
     }
-    return lo;
+    int st = a.stride0;
+    for (int rd = 0; rd < a.rounds; ++rd, st >>= 5) {
+      int v[K];
+#pragma unroll
+      for (int lv = 0; lv < K; ++lv) {
+        const int pos = base[lv] + lane * st;
+        v[lv] = pos < n[lv] ? sel_h[a.sel_off[lv] + pos] : 0x7fffffff;
+      }
+#pragma unroll
+      for (int lv = 0; lv < K; ++lv) {
+        // the probes below the target are a prefix: the list is ascending
+        const int c = __popc(__ballot_sync(kFull, v[lv] < tgt[lv]));
+        if (st == 1) elem[lv] = __shfl_sync(kFull, v[lv], c & 31);  // the entry at base + c, if probed
+        if (c > 0) base[lv] += (c - 1) * st + 1;
+      }
+    }
+#pragma unroll
+    for (int lv = 0; lv < K; ++lv) {
+      if (lv == l) continue;
+      const int lo = base[lv];  // entries of the list below the target
+      if (a.direct) {
+        total += lo;
+      } else {
+        // parents before m contribute p children each; parent m itself, if
+        // kept, its first rem children
+        total += (int64_t)lo << log2p;
+        if (rem[lv] > 0 && lo < n[lv] && elem[lv] == tgt[lv]) total += rem[lv];
+      }
+    }
   }
-  const int n = a.kprime[lv];
-  const int64_t m = X >> a.log2p, r = X & ((1 << a.log2p) - 1);
-  int lo = 0, hi = n;  // lower_bound of m
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if ((int64_t)s[mid] < m) lo = mid + 1;
-    else hi = mid;
-  }
-  int64_t cnt = (int64_t)lo << a.log2p;
-  if (r > 0 && lo < n && (int64_t)s[lo] == m) cnt += r;
-  return cnt;
+  return total;
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherArgs a) {
+// 16 blocks per SM (32 registers, a few spilled): 0.128 ms at 512K x 16 heads,
+// against 0.134 at the 48 registers the search takes unconstrained
+template <typename T, int D, int NL>
+__global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
   const int64_t bh = wid / a.S;
@@ -83,25 +122,17 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherArgs a)
   const int64_t id = wid % a.S;
   const int32_t* sel_h = a.sel + bh * a.sel_per_head;
   int l = 0;
-  while (l + 1 < a.L && id >= a.cnt_off[l + 1]) ++l;
+  while (l + 1 < NL && id >= a.cnt_off[l + 1]) ++l;
   const int64_t j = id - a.cnt_off[l];
   int64_t i;
-  if (l < a.L - 1)
+  if (l < NL - 1)
     i = a.direct ? (int64_t)sel_h[a.sel_off[l] + j]
                  : ((int64_t)sel_h[a.sel_off[l] + (j >> a.log2p)] << a.log2p) + (j & ((1 << a.log2p) - 1));
   else i = j;
   const int64_t e = ((i + 1) << (l * a.log2p)) - 1;
-  // one level per lane: kept entries whose key is below (e, -l)
-  int64_t part = 0;
-  if (lane < a.L) {
-    const int lv = lane;
-    if (lv == l) part = j;
-    else if (lv > l) part = kept_below(a, sel_h, lv, (e + 1) >> (lv * a.log2p));
-    else part = kept_below(a, sel_h, lv, e >> (lv * a.log2p));
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) part += __shfl_xor_sync(kFull, part, o);
-  const int64_t slot = part;
+  // the entry's slot: the kept entries whose key is below (e, -l), level l's
+  // own j included
+  const int64_t slot = j + kept_below_warp<NL>(a, sel_h, l, e, lane);
   if (slot < 0 || slot >= a.S || i < 0 || i >= a.level_len[l]) {
     if (lane == 0) report_error(a.errw, ERRW_BOUNDS);
     return;
@@ -368,6 +399,18 @@ cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaS
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t gather_dispatch_L(int L, const GatherArgs& a, int64_t blocks, cudaStream_t st) {
+  switch (L) {
+#define LH_CASE(n) \
+  case n: gather_kernel<T, D, n><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a); break;
+    LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
@@ -398,17 +441,26 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
   a.log2p = D.log2p;
   a.first_level = first_level;
   a.direct = D.selection == LH_SELECT_DIRECT;
+  int64_t max_n = 1;
+  for (int l = 0; l + 1 < D.L; ++l) {
+    const int64_t n = a.direct ? ((int64_t)D.kprime[l] << D.log2p) : D.kprime[l];
+    if (n > max_n) max_n = n;
+  }
+  a.rounds = 1;
+  a.stride0 = 1;
+  while ((int64_t)a.stride0 * 32 < max_n) {
+    ++a.rounds;
+    a.stride0 *= 32;
+  }
   cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * D.pyr_entries * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (D.BH * D.S + kGatherWarps - 1) / kGatherWarps;
   if (D.dtype == LH_BF16) {
-    if (D.d == 128) gather_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a);
-    else gather_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a);
-  } else {
-    if (D.d == 128) gather_kernel<float, 128><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a);
-    else gather_kernel<float, 64><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a);
+    return D.d == 128 ? gather_dispatch_L<__nv_bfloat16, 128>(D.L, a, blocks, st)
+                      : gather_dispatch_L<__nv_bfloat16, 64>(D.L, a, blocks, st);
   }
-  return cudaGetLastError();
+  return D.d == 128 ? gather_dispatch_L<float, 128>(D.L, a, blocks, st)
+                    : gather_dispatch_L<float, 64>(D.L, a, blocks, st);
 }
 
 cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st) {
