@@ -12,6 +12,9 @@
 // an entry is the number of kept entries with a smaller key, counted level by
 // level with searches over the sorted parent lists (or, when levels are
 // selected directly, the sorted lists of kept entries), so no sort runs.
+#include <algorithm>
+#include <type_traits>
+
 #include "lh_common.cuh"
 
 namespace lh {
@@ -203,8 +206,10 @@ struct ScatterArgs {
   void* y;
   int64_t BH, N, S, pyr_entries;
   int64_t level_off[LH_MAX_LEVELS];
+  int64_t level_len[LH_MAX_LEVELS];
   int64_t tasks_per_head;
   int task_rows, log2p;
+  int tbl_ints;  // slot indices of one task's entries of levels >= 1 (the streaming kernel's table)
 };
 
 template <typename T, int D>
@@ -294,6 +299,110 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
       for (int c = 0; c < VE; ++c) y[c] = v[c] + y[c];
     }
     if (live && j >= 0) store_vec<T, VE>(out + (int64_t)j * D, y);
+  }
+}
+
+// The scatter-back for bf16 rows of 128 channels as a store stream: one task
+// of task_rows keys per warp, two rows per step (lane l: channels
+// [8 (l mod 16), +8) of row 2s + l div 16; p is even, so both rows of a step
+// share their entries of every level >= 1).  When a task starts, the slot
+// indices of its entries of levels >= 1 go to a per-warp table in shared
+// memory, and the level-0 ones are fetched 32 rows ahead, so a step waits on
+// memory only where a kept entry's Os row is read.  Levels are refreshed at
+// their own boundaries: the top level's row once per top-level block, the
+// levels between it and level 1 summed at level-2 boundaries, level 1 at
+// level-1 boundaries.
+template <int NL>
+__global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(ScatterArgs a) {
+  constexpr int D = 128;
+  extern __shared__ int32_t sb_tbl[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lr = lane >> 4, cv = lane & 15;
+  const int64_t task = (int64_t)blockIdx.x * kWarps + warp;
+  if (task >= a.BH * a.tasks_per_head) return;
+  const int64_t bh = task / a.tasks_per_head;
+  const int T = a.task_rows;
+  const int u0 = (int)(task % a.tasks_per_head) * T;  // the task's first key j' = j + 1
+  const int N = (int)a.N, log2p = a.log2p;
+  const int32_t* so = a.slot_of + bh * a.pyr_entries;
+  const float* os = a.os + bh * a.S * D + cv * 8;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.y) + bh * a.N * D + cv * 8;
+  int32_t* tbl = sb_tbl + warp * a.tbl_ints;
+  // level l (>= 1): T >> l log2p entries from (u0 >> l log2p) - 1; -1 where
+  // the level has no such entry
+  int toff[NL > 1 ? NL : 1];
+  {
+    int off = 0;
+#pragma unroll
+    for (int l = 1; l < NL; ++l) {
+      toff[l] = off;
+      const int n = T >> (l * log2p);
+      const int64_t i0 = (int64_t)(u0 >> (l * log2p)) - 1;
+      for (int k = lane; k < n; k += 32) {
+        const int64_t i = i0 + k;
+        tbl[off + k] = (i >= 0 && i < a.level_len[l]) ? so[a.level_off[l] + i] : -1;
+      }
+      off += n;
+    }
+  }
+  __syncwarp();
+  auto add_row = [&](int slot, float (&acc)[8]) {
+    const float4* src = reinterpret_cast<const float4*>(os + (int64_t)slot * D);
+    const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+    acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+  };
+  // level-0 slots of task rows r (j = u0 - 1 + r), 32 at a time, one batch ahead
+  auto s0_load = [&](int r) -> int {
+    const int j = u0 - 1 + r;
+    return (r < T && j >= 0 && j < N) ? so[a.level_off[0] + j] : -1;
+  };
+  int s0_cur = s0_load(lane), s0_next = s0_load(32 + lane);
+  float ctop[8], high[8], cs[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) ctop[c] = high[c] = cs[c] = 0.f;
+  const int pm1 = (1 << log2p) - 1, pm2 = (1 << (2 * log2p)) - 1;
+  const int pmt = NL > 1 ? (1 << ((NL - 1) * log2p)) - 1 : 0;
+  for (int r0 = 0; r0 < T; r0 += 2) {
+    if ((r0 & 31) == 0 && r0 > 0) {
+      s0_cur = s0_next;
+      s0_next = s0_load(r0 + 32 + lane);
+    }
+    if constexpr (NL > 1) {
+      if ((r0 & pm1) == 0) {
+        if ((r0 & pmt) == 0) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) ctop[c] = 0.f;
+          const int st = tbl[toff[NL - 1] + (r0 >> ((NL - 1) * log2p))];
+          if (st >= 0) add_row(st, ctop);
+        }
+        if constexpr (NL > 2) {
+          if ((r0 & pm2) == 0) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) high[c] = ctop[c];
+#pragma unroll
+            for (int l = 2; l < NL - 1; ++l) {
+              const int sl = tbl[toff[l] + (r0 >> (l * log2p))];
+              if (sl >= 0) add_row(sl, high);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cs[c] = high[c];
+          const int s1 = tbl[toff[1] + (r0 >> log2p)];
+          if (s1 >= 0) add_row(s1, cs);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cs[c] = ctop[c];
+        }
+      }
+    }
+    const int s0 = __shfl_sync(kFull, s0_cur, (r0 & 31) + lr);
+    float y[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) y[c] = cs[c];
+    if (s0 >= 0) add_row(s0, y);
+    const int j = u0 - 1 + r0 + lr;
+    if (j >= 0 && j < N) store_vec<__nv_bfloat16, 8>(out + (int64_t)j * D, y);
   }
 }
 
@@ -387,6 +496,20 @@ __global__ void __launch_bounds__(kSadjWarps * 32) scatter_adjoint_kernel(Scatte
 
 template <typename T, int D>
 cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaStream_t st) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+    const size_t smem = (size_t)kWarps * a.tbl_ints * sizeof(int32_t);
+    if (smem <= 48 * 1024 && L <= 8) {
+      const int64_t blocks = (tasks + kWarps - 1) / kWarps;
+      switch (L) {
+#define LH_CASE(n) \
+  case n: scatter_back_stream_kernel<n><<<(unsigned)blocks, kWarps * 32, smem, st>>>(a); break;
+        LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
+#undef LH_CASE
+        default: return cudaErrorInvalidValue;
+      }
+      return cudaGetLastError();
+    }
+  }
   constexpr int R = RowLayout<T, D>::R;  // tasks per warp
   const int64_t blocks = ((tasks + R - 1) / R + kWarps - 1) / kWarps;
   switch (L) {
@@ -469,11 +592,17 @@ cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* s
   a.slot_of = slot_of;
   a.y = y;
   a.BH = D.BH; a.N = D.N; a.S = D.S; a.pyr_entries = D.pyr_entries;
-  for (int l = 0; l < LH_MAX_LEVELS; ++l) a.level_off[l] = D.level_off[l];
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+    a.level_off[l] = D.level_off[l];
+    a.level_len[l] = D.level_len[l];
+  }
   const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
   a.task_rows = (int)(ptop > 64 ? ptop : 64);
   a.tasks_per_head = (D.N + 1 + a.task_rows - 1) / a.task_rows;  // steps cover rows -1 .. N-1
   a.log2p = D.log2p;
+  int64_t tbl = 0;
+  for (int l = 1; l < D.L; ++l) tbl += a.task_rows >> (l * D.log2p);
+  a.tbl_ints = (int)std::min<int64_t>(tbl, 1 << 20);
   const int64_t tasks = D.BH * a.tasks_per_head;
   if (D.dtype == LH_BF16) {
     return D.d == 128 ? scatter_dispatch_L<__nv_bfloat16, 128>(D.L, a, tasks, st)
