@@ -43,8 +43,9 @@ UNIT = "tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 # the kernels each stage entry point launches (names as the ncu launch list shows them)
-STAGE_KERNELS = {"pool": ["pool_kernel"], "score_topk": ["score_pyramid_kernel", "topk_kernel"],
-                 "gather": ["gather_kernel"], "attn_fwd": ["attn_fwd_kernel"], "scatter_back": ["scatter_back_kernel"],
+STAGE_KERNELS = {"pool": ["pool_kernel", "pool_pairs_kernel"], "score_topk": ["score_pyramid_kernel", "topk_kernel"],
+                 "gather": ["gather_kernel"], "attn_fwd": ["attn_fwd_kernel"],
+                 "scatter_back": ["scatter_back_kernel", "scatter_back_stream_kernel"],
                  "scatter_adjoint": ["scatter_adjoint_kernel"], "attn_bwd": ["attn_bwd_kv_kernel", "attn_bwd_q_kernel"],
                  "pool_adjoint": ["pool_adjoint_kernel"]}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
