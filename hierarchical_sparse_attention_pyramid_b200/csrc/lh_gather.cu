@@ -363,46 +363,59 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
   for (int c = 0; c < 8; ++c) ctop[c] = high[c] = cs[c] = 0.f;
   const int pm1 = (1 << log2p) - 1, pm2 = (1 << (2 * log2p)) - 1;
   const int pmt = NL > 1 ? (1 << ((NL - 1) * log2p)) - 1 : 0;
-  for (int r0 = 0; r0 < T; r0 += 2) {
-    if ((r0 & 31) == 0 && r0 > 0) {
+  // rows of the task that exist: j = u0 - 1 + r in [0, N)
+  const int rlo = u0 == 0 ? 1 : 0, rhi = min(T, N + 1 - u0);
+  // T is a multiple of 64: batches of 32 rows, 16 steps each, unrolled
+  for (int rb = 0; rb < T; rb += 32) {
+    if (rb > 0) {
       s0_cur = s0_next;
-      s0_next = s0_load(r0 + 32 + lane);
+      s0_next = s0_load(rb + 32 + lane);
     }
-    if constexpr (NL > 1) {
-      if ((r0 & pm1) == 0) {
-        if ((r0 & pmt) == 0) {
+    __nv_bfloat16* op = out + (int64_t)(u0 - 1 + rb + lr) * D;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) ctop[c] = 0.f;
-          const int st = tbl[toff[NL - 1] + (r0 >> ((NL - 1) * log2p))];
-          if (st >= 0) add_row(st, ctop);
-        }
-        if constexpr (NL > 2) {
-          if ((r0 & pm2) == 0) {
+    for (int u = 0; u < 16; ++u) {
+      const int r0 = rb + 2 * u;
+      if constexpr (NL > 1) {
+        if ((r0 & pm1) == 0) {
+          if ((r0 & pmt) == 0) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) high[c] = ctop[c];
-#pragma unroll
-            for (int l = 2; l < NL - 1; ++l) {
-              const int sl = tbl[toff[l] + (r0 >> (l * log2p))];
-              if (sl >= 0) add_row(sl, high);
-            }
+            for (int c = 0; c < 8; ++c) ctop[c] = 0.f;
+            const int st = tbl[toff[NL - 1] + (r0 >> ((NL - 1) * log2p))];
+            if (st >= 0) add_row(st, ctop);
           }
+          if constexpr (NL > 2) {
+            if ((r0 & pm2) == 0) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cs[c] = high[c];
-          const int s1 = tbl[toff[1] + (r0 >> log2p)];
-          if (s1 >= 0) add_row(s1, cs);
-        } else {
+              for (int c = 0; c < 8; ++c) high[c] = ctop[c];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cs[c] = ctop[c];
+              for (int l = 2; l < NL - 1; ++l) {
+                const int sl = tbl[toff[l] + (r0 >> (l * log2p))];
+                if (sl >= 0) add_row(sl, high);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cs[c] = high[c];
+            const int s1 = tbl[toff[1] + (r0 >> log2p)];
+            if (s1 >= 0) add_row(s1, cs);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cs[c] = ctop[c];
+          }
         }
       }
-    }
-    const int s0 = __shfl_sync(kFull, s0_cur, (r0 & 31) + lr);
-    float y[8];
+      const int s0 = __shfl_sync(kFull, s0_cur, 2 * u + lr);
+      const int r = r0 + lr;
+      const bool ok = r >= rlo && r < rhi;
+      if (s0 >= 0) {
+        float y[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) y[c] = cs[c];
-    if (s0 >= 0) add_row(s0, y);
-    const int j = u0 - 1 + r0 + lr;
-    if (j >= 0 && j < N) store_vec<__nv_bfloat16, 8>(out + (int64_t)j * D, y);
+        for (int c = 0; c < 8; ++c) y[c] = cs[c];
+        add_row(s0, y);
+        if (ok) store_vec<__nv_bfloat16, 8>(op + 2 * u * D, y);
+      } else if (ok) {
+        store_vec<__nv_bfloat16, 8>(op + 2 * u * D, cs);
+      }
+    }
   }
 }
 
