@@ -32,6 +32,10 @@ SMALL = {
                  selection="direct"),
         Workload("nested_sel", 1, 2, 8192, 64, 5, 2, 40, "bf16", "k", "lognormal_token", 19, chunk=32,
                  selection="nested"),
+        # bf16 rows of 128 (the pool pair and scatter-back stream kernels) at L = 2 with p = 8 and at L = 5 with
+        # p = 2 (tasks of 64 rows holding several top-level blocks), N not a multiple of the 64-row task
+        Workload("two_levels_p8", 1, 2, 4000, 128, 2, 8, 64, "bf16", "qk_sum", "iid", 22, chunk=128),
+        Workload("five_levels_p2", 2, 1, 4080, 128, 5, 2, 24, "bf16", "qk_sum", "lognormal_token", 23, chunk=256),
     )
 }
 
