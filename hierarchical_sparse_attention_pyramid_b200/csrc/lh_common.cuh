@@ -76,6 +76,17 @@ __device__ __forceinline__ void load_vec_rw(const T* src, float (&x)[VE]) {
   for (int i = 0; i < VE; ++i) x[i] = Elem<T>::to_f(e[i]);
 }
 
+// store of VE elements with the streaming cache policy (st.global.cs)
+template <typename T, int VE>
+__device__ __forceinline__ void store_vec_stream(T* dst, const float (&x)[VE]) {
+  using V = typename RawVec<sizeof(T) * VE>::type;
+  V u;
+  T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+  for (int i = 0; i < VE; ++i) e[i] = Elem<T>::from_f(x[i]);
+  __stcs(reinterpret_cast<V*>(dst), u);
+}
+
 template <typename T, int VE>
 __device__ __forceinline__ void store_vec(T* dst, const float (&x)[VE]) {
   using V = typename RawVec<sizeof(T) * VE>::type;

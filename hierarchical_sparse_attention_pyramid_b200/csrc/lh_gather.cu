@@ -406,14 +406,15 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
       const int s0 = __shfl_sync(kFull, s0_cur, 2 * u + lr);
       const int r = r0 + lr;
       const bool ok = r >= rlo && r < rhi;
+      // Y with streaming stores (evict first): it is read by no later kernel
       if (s0 >= 0) {
         float y[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) y[c] = cs[c];
         add_row(s0, y);
-        if (ok) store_vec<__nv_bfloat16, 8>(op + 2 * u * D, y);
+        if (ok) store_vec_stream<__nv_bfloat16, 8>(op + 2 * u * D, y);
       } else if (ok) {
-        store_vec<__nv_bfloat16, 8>(op + 2 * u * D, cs);
+        store_vec_stream<__nv_bfloat16, 8>(op + 2 * u * D, cs);
       }
     }
   }

@@ -588,7 +588,9 @@ __global__ void __launch_bounds__(kWarps * 32) pool_adjoint_kernel(PoolAdjArgs a
 #pragma unroll
       for (int c = 0; c < VE; ++c) y[c] += v[c];
     }
-    if (r + lr < rows) store_vec<T, VE>(out + (int64_t)(r + lr) * D, y);
+    // streaming stores: measured 1.157 -> 1.138 ms inside the 512K step (they
+    // do not displace the lines the kernels after this one read)
+    if (r + lr < rows) store_vec_stream<T, VE>(out + (int64_t)(r + lr) * D, y);
   }
 }
 
