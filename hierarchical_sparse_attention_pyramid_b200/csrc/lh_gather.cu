@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
       s0_cur = s0_next;
       s0_next = s0_load(rb + 32 + lane);
     }
-    __nv_bfloat16* op = out + (int64_t)(u0 - 1 + rb + lr) * D;
+    const int64_t jb = (int64_t)u0 - 1 + rb + lr;  // output row of step 0 of the batch (-1 before the head)
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
       const int r0 = rb + 2 * u;
@@ -412,9 +412,9 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
 #pragma unroll
         for (int c = 0; c < 8; ++c) y[c] = cs[c];
         add_row(s0, y);
-        if (ok) store_vec_stream<__nv_bfloat16, 8>(op + 2 * u * D, y);
+        if (ok) store_vec_stream<__nv_bfloat16, 8>(out + (jb + 2 * u) * D, y);
       } else if (ok) {
-        store_vec_stream<__nv_bfloat16, 8>(op + 2 * u * D, cs);
+        store_vec_stream<__nv_bfloat16, 8>(out + (jb + 2 * u) * D, cs);
       }
     }
   }
