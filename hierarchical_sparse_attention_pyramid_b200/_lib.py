@@ -70,6 +70,13 @@ SIGNATURES = {
     "lh_gather_from": [_CFG, c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_fwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P],
     "lh_attn_bwd": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lh_gather_shard": [_CFG, c_int64, c_int64, _P, c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lh_scatter_back_shard": [_CFG, c_int64, _P, _P, _P, _P, _P],
+    "lh_scatter_back_adjoint_shard": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P],
+    "lh_pool_adjoint_shard": [_CFG, c_int64, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lh_head_sums": [_CFG, _P, _P, _P],
+    "lh_attn_fwd_rows": [_CFG, c_int64, c_int64, c_int64, _P, _P, _P, _P, _P, _P, _P],
+    "lh_attn_bwd_rows": [_CFG, c_int64, c_int64, c_int64, c_int64, c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lh_scatter_back": [_CFG, _P, _P, _P, _P],
     "lh_scatter_back_adjoint": [_CFG, _P, _P, _P, _P, _P, _P],
     "lh_pool_adjoint": [_CFG, _P, _P, _P, _P, _P, _P, _P, _P],

@@ -150,6 +150,30 @@ def attn_bwd(layer: Layer, qs, ks, vs, lse, dos, delta, ws=None):
     return dqs, dks, dvs
 
 
+def attn_fwd_rows(layer: Layer, qs, ks, vs, row_lo: int, row_hi: int, os_=None, lse=None, ws=None):
+    """Rows [row_lo, row_hi) of attn_fwd's os and lse, written into os_ [BH, S, d]
+    and lse [BH, S] (allocated when None; other rows left as they are)."""
+    BH, S, d = qs.shape
+    os_ = _empty((BH, S, d), torch.float32, qs.device) if os_ is None else os_
+    lse = _empty((BH, S), torch.float32, qs.device) if lse is None else lse
+    ws = _ws(0, qs.device) if ws is None else ws
+    call("lh_attn_fwd_rows", ctypes.byref(layer.cfg()), ctypes.c_int64(S), ctypes.c_int64(row_lo),
+         ctypes.c_int64(row_hi), _p(qs), _p(ks), _p(vs), _p(os_), _p(lse), _p(ws), _stream())
+    return os_, lse
+
+
+def attn_bwd_rows(layer: Layer, qs, ks, vs, lse, dos, delta, q_rows, k_rows, dqs=None, dks=None, dvs=None, ws=None):
+    """dqs rows q_rows = (lo, hi) and dks, dvs rows k_rows of attn_bwd, written into
+    [BH, S, d] fp32 buffers (allocated when None; other rows left as they are)."""
+    BH, S, d = qs.shape
+    dqs, dks, dvs = (_empty((BH, S, d), torch.float32, qs.device) if t is None else t for t in (dqs, dks, dvs))
+    ws = _ws(0, qs.device) if ws is None else ws
+    call("lh_attn_bwd_rows", ctypes.byref(layer.cfg()), ctypes.c_int64(S), ctypes.c_int64(q_rows[0]),
+         ctypes.c_int64(q_rows[1]), ctypes.c_int64(k_rows[0]), ctypes.c_int64(k_rows[1]), _p(qs), _p(ks), _p(vs),
+         _p(lse), _p(dos), _p(delta), _p(dqs), _p(dks), _p(dvs), _p(ws), _stream())
+    return dqs, dks, dvs
+
+
 def scatter_back(layer: Layer, os_, slot_of):
     y = _empty((layer.B, layer.H, layer.N, layer.d), layer.torch_dtype, os_.device)
     call("lh_scatter_back", ctypes.byref(layer.cfg()), _p(os_), _p(slot_of), _p(y), _stream())

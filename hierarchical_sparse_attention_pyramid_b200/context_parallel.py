@@ -33,22 +33,31 @@ Partition (each rank r owns tokens [t0, t1) = [r N/W, (r+1) N/W)):
 
 Backend interface (one object per rank; tensors are [BH, ...] per shard):
   pool(q, k, v) -> (levels, norms)             levels: the shard's pyramid; norms [2, BH, n]
-  select(norms) -> sel                          global selection from [2, BH, N] norms
+  select(norms) -> sel                          global selection from [2, BH, N] norms, as per
+                                                head and level lists of kept parents (or entries)
   gather(q, k, v, levels, sel_local) -> (seq, (qs, ks, vs))
                                                 seq: per head (level, index) of the shard's
                                                 segment in causal order (local indices)
   attention(qs, ks, vs, lo, hi) -> (os, lse)    rows [lo, hi) of the causal attention
-  scatter(os_seg, seq) -> y                     the shard's Y without the halo
-  halo_add_y(y, h, rows, row)                   add one Os row to Y[h, 0:rows]
-  scatter_adjoint(dy, seq) -> dos               unrounded sums of dY over each entry's range
-                                                inside the shard
-  finish_dos(dos, os_seg) -> (dos, delta)       rounding of dOs and Delta = rowsum(dOs * Os)
+  scatter(os_seg, seq, os_all, halo) -> y       the shard's Y; halo: per head the previous
+                                                shard's kept boundary entries (level, slot in
+                                                os_all, rows), summed into the first rows
+  head_sums(dy) -> [BH, L-1, d]                 sums of dY over the shard's first p^l - 1 rows
+  scatter_adjoint(dy, seq, os_seg, nxt) -> (dos, delta)
+                                                dOs over each entry's range inside the shard,
+                                                plus nxt[h, l-1] (the next shard's head_sums,
+                                                None on the last shard) for the boundary
+                                                entries, rounded; Delta = rowsum(dOs * Os)
   attention_bwd_kv(qs, ks, vs, lse, dos, delta, lo, hi) -> (dks, dvs)  key rows [lo, hi)
   attention_bwd_q(qs, ks, vs, lse, dos, delta, lo, hi) -> dqs           query rows [lo, hi)
   pool_adjoint(dqs, dks, dvs, seq) -> (dq, dk, dv)
+The driver itself only moves rows (all-gathers, segment copies) and keeps the
+index bookkeeping; all arithmetic is in the backend.
 """
 
 from __future__ import annotations
+
+import ctypes
 
 from dataclasses import dataclass
 
@@ -202,11 +211,25 @@ def balanced_windows(S: int, world: int, kind: str = "query") -> list[tuple[int,
 
 # ---------------------------------------------------------------- exchanges
 
+def _all_gather(parts, x: torch.Tensor, group=None) -> None:
+    """dist.all_gather; CUDA tensors go through host copies when the group's
+    backend is gloo (which gathers host memory), e.g. ranks sharing one GPU in
+    a test."""
+    import torch.distributed as dist
+    if x.is_cuda and dist.get_backend(group) == "gloo":
+        host = [torch.empty(x.shape, dtype=x.dtype) for _ in parts]
+        dist.all_gather(host, x.cpu(), group=group)
+        for p, h in zip(parts, host):
+            p.copy_(h)
+    else:
+        dist.all_gather(parts, x, group=group)
+
+
 def allgather_cat(x: torch.Tensor, dim: int, group=None) -> torch.Tensor:
     """Equal-sized pieces, concatenated in rank order along `dim`."""
     import torch.distributed as dist
     parts = [torch.empty_like(x) for _ in range(dist.get_world_size(group))]
-    dist.all_gather(parts, x.contiguous(), group=group)
+    _all_gather(parts, x.contiguous(), group=group)
     return torch.cat(parts, dim=dim)
 
 
@@ -218,7 +241,7 @@ def allgather_rows(x: torch.Tensor, counts, group=None) -> torch.Tensor:
     pad = torch.zeros((x.shape[0], mx) + tuple(x.shape[2:]), dtype=x.dtype, device=x.device)
     pad[:, :x.shape[1]] = x
     parts = [torch.empty_like(pad) for _ in range(dist.get_world_size(group))]
-    dist.all_gather(parts, pad, group=group)
+    _all_gather(parts, pad, group=group)
     return torch.cat([p[:, :int(c)] for p, c in zip(parts, counts)], dim=1)
 
 
@@ -272,10 +295,8 @@ def cp_forward(backend, shard: Shard, q, k, v, selection: str = "parents", group
     win = [b - a for a, b in balanced_windows(S, W, "query")]
     os_f = allgather_rows(os_w, win, group)
     lse_f = allgather_rows(lse_w[..., None], win, group)[..., 0]
-    y = backend.scatter(_segment_rows(os_f, off, counts[r]), seq)
-    for h in range(BH):
-        for l, slot, rows in halo_in(kept[h], shard):
-            backend.halo_add_y(y, h, rows, os_f[h, slot])
+    halo = [halo_in(kept[h], shard) for h in range(BH)]
+    y = backend.scatter(_segment_rows(os_f, off, counts[r]), seq, os_f, halo)
     ctx = CpContext(seq=seq, kept=kept, counts=counts, off=off, qs=qs, ks=ks, vs=vs, os=os_f, lse=lse_f)
     return y, ctx
 
@@ -285,16 +306,11 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     BH = dy.shape[0]
     W, r, p, L = shard.world, shard.rank, shard.p, shard.L
     # halo: sums of dY over this shard's first p^l - 1 tokens, for the previous shard
-    heads = torch.stack([dy[:, :p ** l - 1].sum(dim=1) for l in range(1, L)], dim=1) if L > 1 else \
-        torch.zeros((BH, 0, dy.shape[2]), dtype=dy.dtype, device=dy.device)
-    heads_all = allgather_cat(heads[None], dim=0, group=group)  # [W, BH, L-1, d]
-    dos = backend.scatter_adjoint(dy, ctx.seq)
-    if r + 1 < W:
-        for h in range(BH):
-            lv, ix = ctx.seq[h]
-            for l, s in halo_out_entries(lv, ix, shard):
-                dos[h, s] += heads_all[r + 1, h, l - 1]
-    dos, delta = backend.finish_dos(dos, _segment_rows(ctx.os, ctx.off, ctx.counts[r]))
+    nxt = None
+    if L > 1:
+        heads_all = allgather_cat(backend.head_sums(dy)[None], dim=0, group=group)  # [W, BH, L-1, d]
+        nxt = heads_all[r + 1] if r + 1 < W else None
+    dos, delta = backend.scatter_adjoint(dy, ctx.seq, _segment_rows(ctx.os, ctx.off, ctx.counts[r]), nxt)
     dos_f = torch.stack([allgather_rows(dos[h:h + 1, :int(ctx.counts[r, h])], ctx.counts[:, h], group)[0]
                          for h in range(BH)])
     delta_f = torch.stack([allgather_rows(delta[h:h + 1, :int(ctx.counts[r, h]), None], ctx.counts[:, h],
@@ -310,3 +326,130 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     dvs = _segment_rows(allgather_rows(dvs_w, kwin, group), ctx.off, ctx.counts[r])
     dqs = _segment_rows(allgather_rows(dqs_w, qwin, group), ctx.off, ctx.counts[r])
     return backend.pool_adjoint(dqs, dks, dvs, ctx.seq)
+
+
+# ---------------------------------------------------------------- the CUDA backend
+
+class CudaBackend:
+    """The per-rank arithmetic in the library's kernels: the whole-layer stage
+    calls on the shard (pool, selection), the shard forms of the gather,
+    scatter-back, its adjoint and the pool adjoint (halo rows included), and
+    the row-window forms of the attention.  bf16 rows of 128 channels (the
+    scatter-back's halo path).  `layer` is the whole layer; tensors are CUDA."""
+
+    def __init__(self, layer, shard: Shard):
+        from . import api
+        if layer.dtype != "bf16" or layer.d != 128:
+            raise ValueError("the CUDA context-parallel backend takes bf16 rows of 128 channels")
+        self.api = api
+        self.layer = layer
+        self.shard = shard
+        self.local = api.Layer(layer.B, layer.H, shard.n, layer.d, layer.L, layer.p, layer.k, layer.chunk,
+                               layer.dtype, layer.scorer, layer.selection)
+        self.info = api.plan(layer)
+        self.local_info = api.plan(self.local)
+
+    def _shape4(self, x):
+        return x.reshape(self.layer.B, self.layer.H, *x.shape[1:])
+
+    def pool(self, q, k, v):
+        pq, pk, pv, norms = self.api.pyramid_pool(self.local, self._shape4(q.contiguous()),
+                                                  self._shape4(k.contiguous()), self._shape4(v.contiguous()))
+        return (pq, pk, pv), norms
+
+    def select(self, norms):
+        self.sel = self.api.score_topk(self.layer, norms.contiguous())
+        host = self.sel.cpu().numpy()
+        I, L, p = self.info, self.layer.L, self.layer.p
+        direct = self.layer.selection == "direct"
+        out = []
+        for h in range(host.shape[0]):
+            per = []
+            for l in range(L - 1):
+                n = int(I.kprime[l]) * (p if direct else 1)
+                per.append(host[h, int(I.sel_off[l]):int(I.sel_off[l]) + n].astype(np.int64))
+            out.append(per)
+        self.sel_lists = out
+        return out
+
+    def gather(self, q, k, v, levels, sel_local):
+        from . import _lib
+        sh, lay = self.shard, self.layer
+        kept = [kept_entries(self.sel_lists[h], lay.N, lay.p, lay.L, lay.selection) for h in range(lay.BH)]
+        counts = np.stack([segment_counts(kept[h], lay.N, lay.p, lay.L, sh.world) for h in range(lay.BH)], axis=1)
+        self.counts_r = counts[sh.rank]
+        self.seg_rows = max(1, int(self.counts_r.max()))
+        dev = q.device
+        seg_off = torch.from_numpy(counts[:sh.rank].sum(axis=0).astype(np.int64)).to(dev)
+        qs, ks, vs = (torch.zeros((lay.BH, self.seg_rows, lay.d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+        # rows past a head's segment hold an entry with an empty range
+        self.seq_map = torch.full((lay.BH, self.seg_rows), sh.n, dtype=torch.int32, device=dev)
+        self.slot_of = torch.empty((lay.BH, self.local_info.pyr_entries), dtype=torch.int32, device=dev)
+        pq, pk, pv = levels
+        p_ = self.api._p
+        _lib.call("lh_gather_shard", ctypes.byref(lay.cfg()), ctypes.c_int64(sh.t0), ctypes.c_int64(sh.t1),
+                  p_(seg_off), ctypes.c_int64(self.seg_rows), p_(q.contiguous()), p_(k.contiguous()),
+                  p_(v.contiguous()), p_(pq), p_(pk), p_(pv), p_(self.sel), p_(qs), p_(ks), p_(vs),
+                  p_(self.seq_map), p_(self.slot_of), self.api._stream())
+        sm = self.seq_map.cpu().numpy().astype(np.int64)
+        seq = [((sm[h, :c] >> 28), (sm[h, :c] & ((1 << 28) - 1))) for h, c in enumerate(self.counts_r)]
+        return seq, (qs, ks, vs)
+
+    def attention(self, qs, ks, vs, lo, hi):
+        os_, lse = self.api.attn_fwd_rows(self.layer, qs.contiguous(), ks.contiguous(), vs.contiguous(), lo, hi)
+        return os_[:, lo:hi], lse[:, lo:hi]
+
+    def scatter(self, os_seg, seq, os_all, halo):
+        from . import _lib
+        lay = self.layer
+        hal = torch.zeros((lay.BH, max(lay.L - 1, 1), lay.d), dtype=torch.float32, device=os_seg.device)
+        for h, ents in enumerate(halo):
+            for l, slot, rows in ents:
+                hal[h, l - 1] = os_all[h, slot]
+        y = torch.empty((lay.B, lay.H, self.shard.n, lay.d), dtype=torch.bfloat16, device=os_seg.device)
+        p_ = self.api._p
+        _lib.call("lh_scatter_back_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
+                  p_(os_seg.contiguous()), p_(self.slot_of), p_(hal), p_(y), self.api._stream())
+        return y.reshape(lay.BH, self.shard.n, lay.d)
+
+    def head_sums(self, dy):
+        from . import _lib
+        lay = self.layer
+        sums = torch.empty((lay.BH, lay.L - 1, lay.d), dtype=torch.float32, device=dy.device)
+        _lib.call("lh_head_sums", ctypes.byref(self.local.cfg()), self.api._p(dy.contiguous()), self.api._p(sums),
+                  self.api._stream())
+        return sums
+
+    def scatter_adjoint(self, dy, seq, os_seg, nxt):
+        from . import _lib
+        lay = self.layer
+        dos = torch.zeros((lay.BH, self.seg_rows, lay.d), dtype=torch.float16, device=dy.device)
+        delta = torch.zeros((lay.BH, self.seg_rows), dtype=torch.float32, device=dy.device)
+        p_ = self.api._p
+        _lib.call("lh_scatter_back_adjoint_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
+                  p_(dy.contiguous()), p_(self.seq_map), p_(os_seg.contiguous()),
+                  p_(nxt.contiguous()) if nxt is not None else None, p_(dos), p_(delta), self.api._stream())
+        return dos, delta
+
+    def _bwd(self, qs, ks, vs, lse, dos, delta, q_rows, k_rows):
+        return self.api.attn_bwd_rows(self.layer, qs.contiguous(), ks.contiguous(), vs.contiguous(),
+                                      lse.contiguous(), dos.contiguous(), delta.contiguous(), q_rows, k_rows)
+
+    def attention_bwd_kv(self, qs, ks, vs, lse, dos, delta, lo, hi):
+        _, dks, dvs = self._bwd(qs, ks, vs, lse, dos, delta, (0, 0), (lo, hi))
+        return dks[:, lo:hi], dvs[:, lo:hi]
+
+    def attention_bwd_q(self, qs, ks, vs, lse, dos, delta, lo, hi):
+        dqs, _, _ = self._bwd(qs, ks, vs, lse, dos, delta, (lo, hi), (0, 0))
+        return dqs[:, lo:hi]
+
+    def pool_adjoint(self, dqs, dks, dvs, seq):
+        from . import _lib
+        lay = self.layer
+        shp = (lay.B, lay.H, self.shard.n, lay.d)
+        dq, dk, dv = (torch.empty(shp, dtype=torch.bfloat16, device=dqs.device) for _ in range(3))
+        p_ = self.api._p
+        _lib.call("lh_pool_adjoint_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
+                  p_(dqs.contiguous()), p_(dks.contiguous()), p_(dvs.contiguous()), p_(self.slot_of), p_(dq),
+                  p_(dk), p_(dv), self.api._stream())
+        return tuple(t.reshape(lay.BH, self.shard.n, lay.d) for t in (dq, dk, dv))

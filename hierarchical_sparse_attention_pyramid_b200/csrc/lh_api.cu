@@ -322,6 +322,84 @@ lh_status lh_attn_bwd(const lh_config* cfg, int64_t S, const void* qs, const voi
   return LH_OK;
 }
 
+lh_status lh_gather_shard(const lh_config* cfg, int64_t t0, int64_t t1, const int64_t* seg_off, int64_t seg_rows,
+                         const void* q, const void* k, const void* v, const void* pyr_q, const void* pyr_k,
+                         const void* pyr_v, const int32_t* sel, void* qs, void* ks, void* vs, int32_t* seq_map,
+                         int32_t* slot_of, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  const int64_t ptop = (int64_t)1 << ((D.L - 1) * D.log2p);
+  if (t0 < 0 || t1 > D.N || t0 >= t1 || t0 % ptop != 0 || t1 % ptop != 0)
+    return fail(LH_ERR_INVALID_ARG, "lh_gather_shard: [t0, t1) must be a non-empty range of multiples of p^(L-1) in [0, N]");
+  if (seg_rows < 1 || seg_rows > D.S) return fail(LH_ERR_INVALID_ARG, "lh_gather_shard: seg_rows outside [1, S]");
+  // the shard's own plan: a layer of its t1 - t0 tokens
+  lh_config sc = *cfg;
+  sc.N = t1 - t0;
+  lh_plan_info sinfo;
+  Dims SD;
+  s = plan_impl(&sc, &sinfo, &SD);
+  if (s != LH_OK) return s;
+  if (!seg_off) return fail(LH_ERR_INVALID_ARG, "lh_gather_shard: NULL seg_off");
+  LH_CHECK_PTR(q); LH_CHECK_PTR(k); LH_CHECK_PTR(v);
+  if (D.L > 1) { LH_CHECK_PTR(pyr_q); LH_CHECK_PTR(pyr_k); LH_CHECK_PTR(pyr_v); LH_CHECK_PTR(sel); }
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(slot_of);
+  LH_CUDA(launch_gather(D, q, k, v, pyr_q, pyr_k, pyr_v, sel, qs, ks, vs, seq_map, slot_of, nullptr,
+                        (cudaStream_t)stream, 1, &SD, t0, seg_off, seg_rows),
+          "lh_gather_shard");
+  return LH_OK;
+}
+
+// a row window [lo, hi) of the sequence as 128-row tiles: lo a multiple of
+// 128, hi a multiple of 128 or S
+static bool tile_window(int64_t S, int64_t lo, int64_t hi, int64_t* t0, int64_t* t1) {
+  if (lo < 0 || hi > S || lo > hi || lo % 128 != 0 || (hi % 128 != 0 && hi != S)) return false;
+  *t0 = lo / 128;
+  *t1 = (hi + 127) / 128;
+  return true;
+}
+
+lh_status lh_attn_fwd_rows(const lh_config* cfg, int64_t S, int64_t row_lo, int64_t row_hi, const void* qs,
+                           const void* ks, const void* vs, float* os, float* lse, void* ws, lh_stream_t stream) {
+  if (!cfg) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd_rows: NULL cfg");
+  if (cfg->B < 1 || cfg->H < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd_rows: sizes must be positive");
+  if (cfg->d != 64 && cfg->d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd_rows: d must be 64 or 128");
+  if (cfg->H > 65535 || cfg->B * cfg->H > 65535)
+    return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd_rows: B*H must be <= 65535");
+  if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_attn_fwd_rows: S too large");
+  int64_t t0, t1;
+  if (!tile_window(S, row_lo, row_hi, &t0, &t1))
+    return fail(LH_ERR_INVALID_ARG, "lh_attn_fwd_rows: rows must be [lo, hi) with lo % 128 == 0 and hi % 128 == 0 or S");
+  if (t0 == t1) return LH_OK;
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(os); LH_CHECK_PTR(lse); LH_CHECK_PTR(ws);
+  LH_CUDA(launch_attn_fwd(cfg->B * cfg->H, S, cfg->d, qs, ks, vs, os, lse, err_word(ws), (cudaStream_t)stream,
+                          4000000000ll, 1, t0, t1),
+          "lh_attn_fwd_rows");
+  return LH_OK;
+}
+
+lh_status lh_attn_bwd_rows(const lh_config* cfg, int64_t S, int64_t q_lo, int64_t q_hi, int64_t k_lo, int64_t k_hi,
+                           const void* qs, const void* ks, const void* vs, const float* lse, const void* dos,
+                           const float* delta, float* dqs, float* dks, float* dvs, void* ws, lh_stream_t stream) {
+  if (!cfg) return fail(LH_ERR_INVALID_ARG, "lh_attn_bwd_rows: NULL cfg");
+  if (cfg->B < 1 || cfg->H < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "lh_attn_bwd_rows: sizes must be positive");
+  if (cfg->d != 64 && cfg->d != 128) return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd_rows: d must be 64 or 128");
+  if (cfg->H > 65535 || cfg->B * cfg->H > 65535)
+    return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd_rows: B*H must be <= 65535");
+  if (S >= ((int64_t)1 << 31)) return fail(LH_ERR_UNSUPPORTED, "lh_attn_bwd_rows: S too large");
+  int64_t qt0, qt1, kt0, kt1;
+  if (!tile_window(S, q_lo, q_hi, &qt0, &qt1) || !tile_window(S, k_lo, k_hi, &kt0, &kt1))
+    return fail(LH_ERR_INVALID_ARG, "lh_attn_bwd_rows: rows must be [lo, hi) with lo % 128 == 0 and hi % 128 == 0 or S");
+  if (qt0 == qt1 && kt0 == kt1) return LH_OK;
+  LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(lse); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
+  LH_CHECK_PTR(dqs); LH_CHECK_PTR(dks); LH_CHECK_PTR(dvs); LH_CHECK_PTR(ws);
+  LH_CUDA(launch_attn_bwd(cfg->B * cfg->H, S, cfg->d, qs, ks, vs, lse, dos, delta, dqs, dks, dvs, err_word(ws),
+                          (cudaStream_t)stream, qt0, qt1, kt0, kt1),
+          "lh_attn_bwd_rows");
+  return LH_OK;
+}
+
 lh_status lh_scatter_back(const lh_config* cfg, const float* os, const int32_t* slot_of, void* y,
                           lh_stream_t stream) {
   lh_plan_info info;
@@ -342,6 +420,68 @@ lh_status lh_scatter_back_adjoint(const lh_config* cfg, const void* dy, const in
   LH_CHECK_PTR(dy); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(os); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
   LH_CUDA(launch_scatter_adjoint(D, dy, seq_map, os, dos, delta, nullptr, (cudaStream_t)stream),
           "lh_scatter_back_adjoint");
+  return LH_OK;
+}
+
+// the plan of one shard's layer (cfg->N = the shard's tokens) with its
+// segment of seg_rows sequence rows per head in place of the plan's S
+static lh_status shard_dims(const lh_config* cfg, int64_t seg_rows, Dims* D, const char* who) {
+  lh_plan_info info;
+  lh_status s = plan_impl(cfg, &info, D);
+  if (s != LH_OK) return s;
+  if (seg_rows < 1 || seg_rows >= ((int64_t)1 << 31)) return fail(LH_ERR_INVALID_ARG, who);
+  D->S = seg_rows;
+  return LH_OK;
+}
+
+lh_status lh_scatter_back_shard(const lh_config* cfg, int64_t seg_rows, const float* os, const int32_t* slot_of,
+                                const float* halo, void* y, lh_stream_t stream) {
+  Dims D;
+  lh_status s = shard_dims(cfg, seg_rows, &D, "lh_scatter_back_shard: seg_rows outside [1, 2^31)");
+  if (s != LH_OK) return s;
+  if (D.dtype != LH_BF16 || D.d != 128)
+    return fail(LH_ERR_UNSUPPORTED, "lh_scatter_back_shard: bf16 rows of 128 channels only");
+  LH_CHECK_PTR(os); LH_CHECK_PTR(slot_of); LH_CHECK_PTR(y);
+  if (D.L > 1) LH_CHECK_PTR(halo);
+  LH_CUDA(launch_scatter_back(D, os, slot_of, y, (cudaStream_t)stream, D.L > 1 ? halo : nullptr),
+          "lh_scatter_back_shard");
+  return LH_OK;
+}
+
+lh_status lh_scatter_back_adjoint_shard(const lh_config* cfg, int64_t seg_rows, const void* dy,
+                                        const int32_t* seq_map, const float* os, const float* halo, void* dos,
+                                        float* delta, lh_stream_t stream) {
+  Dims D;
+  lh_status s = shard_dims(cfg, seg_rows, &D, "lh_scatter_back_adjoint_shard: seg_rows outside [1, 2^31)");
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(dy); LH_CHECK_PTR(seq_map); LH_CHECK_PTR(os); LH_CHECK_PTR(dos); LH_CHECK_PTR(delta);
+  if (halo) LH_CHECK_PTR(halo);
+  LH_CUDA(launch_scatter_adjoint(D, dy, seq_map, os, dos, delta, nullptr, (cudaStream_t)stream,
+                                 D.L > 1 ? halo : nullptr),
+          "lh_scatter_back_adjoint_shard");
+  return LH_OK;
+}
+
+lh_status lh_pool_adjoint_shard(const lh_config* cfg, int64_t seg_rows, const float* dqs, const float* dks,
+                                const float* dvs, const int32_t* slot_of, void* dq, void* dk, void* dv,
+                                lh_stream_t stream) {
+  Dims D;
+  lh_status s = shard_dims(cfg, seg_rows, &D, "lh_pool_adjoint_shard: seg_rows outside [1, 2^31)");
+  if (s != LH_OK) return s;
+  LH_CHECK_PTR(dqs); LH_CHECK_PTR(dks); LH_CHECK_PTR(dvs); LH_CHECK_PTR(slot_of);
+  LH_CHECK_PTR(dq); LH_CHECK_PTR(dk); LH_CHECK_PTR(dv);
+  LH_CUDA(launch_pool_adjoint(D, dqs, dks, dvs, slot_of, dq, dk, dv, (cudaStream_t)stream), "lh_pool_adjoint_shard");
+  return LH_OK;
+}
+
+lh_status lh_head_sums(const lh_config* cfg, const void* dy, float* sums, lh_stream_t stream) {
+  lh_plan_info info;
+  Dims D;
+  lh_status s = plan_impl(cfg, &info, &D);
+  if (s != LH_OK) return s;
+  if (D.L < 2) return LH_OK;
+  LH_CHECK_PTR(dy); LH_CHECK_PTR(sums);
+  LH_CUDA(launch_head_sums(D, dy, sums, (cudaStream_t)stream), "lh_head_sums");
   return LH_OK;
 }
 

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dK,
-                       float* __restrict__ dV, int* errw, int S, float scale_log2, float scale) {
+                       float* __restrict__ dV, int* errw, int S, float scale_log2, float scale, int kt0, int kt1) {
   using Lay = KvSmem<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (reinterpret_cast<uintptr_t>(smem_raw) & 1023) {  // the layout has no slack to align it
@@ -122,10 +122,11 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + 127) / 128;
-  // one CTA per (key tile, head), tile-major: small kt (most query tiles) of
-  // every head is started first, the short tiles fill the tail
-  const int BHn = (int)(gridDim.x / (unsigned)n_qt);
-  const int kt = (int)(blockIdx.x / (unsigned)BHn);
+  // one CTA per (key tile, head) of the key tiles [kt0, kt1), tile-major:
+  // small kt (most query tiles) of every head is started first, the short
+  // tiles fill the tail
+  const int BHn = (int)(gridDim.x / (unsigned)(kt1 - kt0));
+  const int kt = kt0 + (int)(blockIdx.x / (unsigned)BHn);
   const int bh = (int)(blockIdx.x % (unsigned)BHn);
   const int NJ = n_qt - kt;        // 128-query steps, from the diagonal tile on
 
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       const float* __restrict__ LSE, const float* __restrict__ Delta, float* __restrict__ dQ,
-                      int* errw, int S, float scale_log2, float scale) {
+                      int* errw, int S, float scale_log2, float scale, int qt0, int qt1) {
   using Lay = QSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -454,9 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (S + 127) / 128;
-  // one CTA per (query tile, head), tile-major with the longest rows first
-  const int BHn = (int)(gridDim.x / (unsigned)n_qt);
-  const int qt = n_qt - 1 - (int)(blockIdx.x / (unsigned)BHn);
+  // one CTA per (query tile, head) of the query tiles [qt0, qt1), tile-major
+  // with the longest rows first
+  const int BHn = (int)(gridDim.x / (unsigned)(qt1 - qt0));
+  const int qt = qt1 - 1 - (int)(blockIdx.x / (unsigned)BHn);
   const int bh = (int)(blockIdx.x % (unsigned)BHn);
   const int NJ = qt + 1;  // key tiles up to the diagonal
 
@@ -711,37 +713,53 @@ struct SeqMaps {
 
 template <int D>
 cudaError_t launch_bwd_d(int64_t BH, int64_t S, const SeqMaps& m, const float* lse, const float* delta, float* dqs,
-                         float* dks, float* dvs, int* errw, float scale_log2, float scale, cudaStream_t st) {
-  const unsigned n_qt = (unsigned)((S + 127) / 128);
-  if ((int64_t)n_qt * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
-  int smem = KvSmem<D>::kAlloc;
-  cudaError_t e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  attn_bwd_kv_kernel<D><<<dim3((unsigned)(n_qt * BH)), kThreadsKV, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dks, dvs,
-                                                                         errw, (int)S, scale_log2, scale);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  smem = QSmem<D>::kAlloc;
-  e = cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  attn_bwd_q_kernel<D><<<dim3((unsigned)(n_qt * BH)), kThreads, smem, st>>>(m.q, m.k, m.v, m.o, lse, delta, dqs, errw,
-                                                                        (int)S, scale_log2, scale);
-  return cudaGetLastError();
+                         float* dks, float* dvs, int* errw, float scale_log2, float scale, cudaStream_t st,
+                         int64_t qt0, int64_t qt1, int64_t kt0, int64_t kt1) {
+  // dK/dV of the key tiles [kt0, kt1), dQ of the query tiles [qt0, qt1); an
+  // empty window launches nothing
+  cudaError_t e;
+  if (kt1 > kt0) {
+    if ((kt1 - kt0) * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
+    const int smem = KvSmem<D>::kAlloc;
+    e = cudaFuncSetAttribute(attn_bwd_kv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_bwd_kv_kernel<D><<<dim3((unsigned)((kt1 - kt0) * BH)), kThreadsKV, smem, st>>>(
+        m.q, m.k, m.v, m.o, lse, delta, dks, dvs, errw, (int)S, scale_log2, scale, (int)kt0, (int)kt1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (qt1 > qt0) {
+    if ((qt1 - qt0) * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+    const int smem = QSmem<D>::kAlloc;
+    e = cudaFuncSetAttribute(attn_bwd_q_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attn_bwd_q_kernel<D><<<dim3((unsigned)((qt1 - qt0) * BH)), kThreads, smem, st>>>(
+        m.q, m.k, m.v, m.o, lse, delta, dqs, errw, (int)S, scale_log2, scale, (int)qt0, (int)qt1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
-                            float* dvs, int* errw, cudaStream_t st) {
+                            float* dvs, int* errw, cudaStream_t st, int64_t qt0, int64_t qt1, int64_t kt0,
+                            int64_t kt1) {
+  const int64_t n_qt = (S + 127) / 128;
+  if (qt1 < 0) qt1 = n_qt;
+  if (kt1 < 0) kt1 = n_qt;
+  if (qt0 < 0 || qt0 > qt1 || qt1 > n_qt || kt0 < 0 || kt0 > kt1 || kt1 > n_qt) return cudaErrorInvalidValue;
   SeqMaps m;
   if (!make_seq_map(&m.q, qs, BH, S, d, 128) || !make_seq_map(&m.k, ks, BH, S, d, 128) ||
       !make_seq_map(&m.v, vs, BH, S, d, 128) || !make_seq_map(&m.o, dos, BH, S, d, 128))
     return cudaErrorInvalidValue;
   const double scale = 1.0 / sqrt((double)d);
   const float scale_log2 = (float)(1.4426950408889634 * scale);
-  if (d == 128) return launch_bwd_d<128>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st);
-  return launch_bwd_d<64>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st);
+  if (d == 128)
+    return launch_bwd_d<128>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st, qt0, qt1, kt0, kt1);
+  return launch_bwd_d<64>(BH, S, m, lse, delta, dqs, dks, dvs, errw, scale_log2, (float)scale, st, qt0, qt1, kt0, kt1);
 }
 
 }  // namespace lh

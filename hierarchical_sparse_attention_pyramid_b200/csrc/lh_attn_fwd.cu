@@ -60,7 +60,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, float* __restrict__ O, float* __restrict__ LSE,
-                    int* errw, int S, float scale_log2, long long wait_cycles, int issue_loads) {
+                    int* errw, int S, float scale_log2, long long wait_cycles, int issue_loads, int qt0, int qt1) {
   using Lay = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -76,16 +76,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = (S + BM - 1) / BM;
-  const int n_pairs = (n_qt + 1) / 2;
+  // the query tiles [qt0, qt1) of the sequence (all of them, except for a
+  // row window of the sequence); key tiles run from 0 to each query tile
+  const int n_pairs = (qt1 - qt0 + 1) / 2;
   // one CTA per (tile pair, head), pair-major: the block scheduler starts
   // blocks in index order, so every head's longest pairs run first and the
   // short ones fill the tail
   const int BHn = (int)(gridDim.x / (unsigned)n_pairs);
   const int c = n_pairs - 1 - (int)(blockIdx.x / (unsigned)BHn);
   const int bh = (int)(blockIdx.x % (unsigned)BHn);
-  const int qtile[2] = {2 * c, 2 * c + 1};
-  const bool hasB = qtile[1] < n_qt;
+  const int qtile[2] = {qt0 + 2 * c, qt0 + 2 * c + 1};
+  const bool hasB = qtile[1] < qt1;
   const int last[2] = {qtile[0], hasB ? qtile[1] : -1};  // last key tile of each query tile
   const int n_kv = (hasB ? qtile[1] : qtile[0]) + 1;
 
@@ -381,27 +382,30 @@ bool make_f32_map(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, in
 }
 
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
-                            float* lse, int* errw, cudaStream_t st, long long wait_cycles, int issue_loads) {
+                            float* lse, int* errw, cudaStream_t st, long long wait_cycles, int issue_loads, int64_t qt0,
+                            int64_t qt1) {
   CUtensorMap mq, mk, mv;
   if (!make_seq_map(&mq, qs, BH, S, d, BM) || !make_seq_map(&mk, ks, BH, S, d, BN) ||
       !make_seq_map(&mv, vs, BH, S, d, BN))
     return cudaErrorInvalidValue;
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
   const int64_t n_qt = (S + BM - 1) / BM;
-  if (((n_qt + 1) / 2) * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
-  const dim3 grid((unsigned)(((n_qt + 1) / 2) * BH));
+  if (qt1 < 0) qt1 = n_qt;
+  if (qt0 < 0 || qt0 >= qt1 || qt1 > n_qt) return cudaErrorInvalidValue;
+  if (((qt1 - qt0 + 1) / 2) * BH > 0x7fffffffll) return cudaErrorInvalidConfiguration;  // one grid dimension
+  const dim3 grid((unsigned)(((qt1 - qt0 + 1) / 2) * BH));
   if (d == 128) {
     const int smem = FwdSmem<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attn_fwd_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2, wait_cycles,
-                                                               issue_loads);
+                                                               issue_loads, (int)qt0, (int)qt1);
   } else {
     const int smem = FwdSmem<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attn_fwd_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, os, lse, errw, (int)S, scale_log2, wait_cycles,
-                                                               issue_loads);
+                                                               issue_loads, (int)qt0, (int)qt1);
   }
   return cudaGetLastError();
 }

@@ -125,26 +125,42 @@ cudaError_t launch_score_topk(const Dims& D, const float* norms, float* spyr, in
                               cudaStream_t st);
 // kept entries of levels 1 .. first_level-1 are averaged from level 0 here
 // instead of being read from the pyramid
+// shard (optional): the plan of a layer of the shard's tokens [t0, t0 + shard->N);
+// only the entries whose key lies there are gathered, from the shard's rows,
+// into per-head segments of seg_rows rows starting at slot seg_off[bh]
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
                           const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
-                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level = 1);
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level = 1,
+                          const Dims* shard = nullptr, int64_t t0 = 0, const int64_t* seg_off = nullptr,
+                          int64_t seg_rows = 0);
 
 // first pyramid level lh_forward materialises: finer kept entries are cheaper
 // to average from level 0 in the gather than to write whole levels
 int materialized_level(const Dims& D);
-cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st);
+// halo (optional, context parallelism; [BH][L-1][d] fp32): the previous
+// shard's last entries' Os rows (scatter-back), the next shard's sums of dY
+// over its first p^l - 1 rows (adjoint)
+cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st,
+                                const float* halo = nullptr);
 cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
-                                   void* dos, float* delta, int* errw, cudaStream_t st);
+                                   void* dos, float* delta, int* errw, cudaStream_t st, const float* halo = nullptr);
+// sums[bh][l-1] = sum of dY rows [0, p^l - 1) of head bh, l = 1 .. L-1 (fp32)
+cudaError_t launch_head_sums(const Dims& D, const void* dy, float* sums, cudaStream_t st);
 cudaError_t launch_pool_adjoint(const Dims& D, const float* dqs, const float* dks, const float* dvs,
                                 const int32_t* slot_of, void* dq, void* dk, void* dv, cudaStream_t st);
 // wait_cycles bounds every barrier wait of the kernel (SM clocks);
 // issue_loads = 0 only for the timeout self-test (the producer loads nothing)
+// query tiles [qt0, qt1) of 128 rows (qt1 < 0: to the last tile); O and LSE
+// rows outside the window are not written
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs, float* os,
                             float* lse, int* errw, cudaStream_t st, long long wait_cycles = 4000000000ll,
-                            int issue_loads = 1);
+                            int issue_loads = 1, int64_t qt0 = 0, int64_t qt1 = -1);
+// dQ of the query tiles [qt0, qt1), dK and dV of the key tiles [kt0, kt1)
+// (a negative end: to the last tile)
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, const void* qs, const void* ks, const void* vs,
                             const float* lse, const void* dos, const float* delta, float* dqs, float* dks,
-                            float* dvs, int* errw, cudaStream_t st);
+                            float* dvs, int* errw, cudaStream_t st, int64_t qt0 = 0, int64_t qt1 = -1,
+                            int64_t kt0 = 0, int64_t kt1 = -1);
 
 // message of the last failure on this thread (set by the API layer)
 void set_error_message(const char* fmt, ...);

@@ -51,6 +51,16 @@ struct GatherArgs {
   // warp searches of the sorted lists: `rounds` rounds of 32 probes, the
   // first at stride stride0 = 32^(rounds-1) >= every list's length / 32
   int rounds, stride0;
+  // one shard of the tokens (context parallelism): only the entries whose key
+  // lies in [t0, t1) are gathered, from rows that hold that shard alone (x0:
+  // n_loc tokens per head, pyr: the shard's own pyramid), into a per-head
+  // segment of out_rows rows that starts at slot seg_off[bh]; seq_map and
+  // slot_of are the segment's and the shard's.  The whole layer is the shard
+  // [0, N) with seg_off null and out_rows = S.
+  int64_t t0, t1, out_rows, n_loc, upper_loc, pyr_loc;
+  const int64_t* seg_off;
+  int64_t upper_off_loc[LH_MAX_LEVELS];
+  int64_t level_off_loc[LH_MAX_LEVELS];
 };
 
 // Kept entries of every level whose key is below (e, -l), excluding level l
@@ -116,7 +126,9 @@ __device__ __forceinline__ int64_t kept_below_warp(const GatherArgs& a, const in
 
 // 16 blocks per SM (32 registers, a few spilled): 0.128 ms at 512K x 16 heads,
 // against 0.134 at the 48 registers the search takes unconstrained
-template <typename T, int D, int NL>
+// SHARD: one shard of the tokens (context parallelism; the whole layer is
+// compiled without its offsets)
+template <typename T, int D, int NL, bool SHARD>
 __global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
@@ -135,14 +147,18 @@ __global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArg
   const int64_t e = ((i + 1) << (l * a.log2p)) - 1;
   // the entry's slot: the kept entries whose key is below (e, -l), level l's
   // own j included
+  if (SHARD && (e < a.t0 || e >= a.t1)) return;  // another shard's entry
   const int64_t slot = j + kept_below_warp<NL>(a, sel_h, l, e, lane);
-  if (slot < 0 || slot >= a.S || i < 0 || i >= a.level_len[l]) {
+  // the row in this segment, and the entry's index in the shard's level l
+  const int64_t srow = SHARD ? slot - a.seg_off[bh] : slot;
+  const int64_t il = SHARD ? i - (a.t0 >> (l * a.log2p)) : i;
+  if (srow < 0 || srow >= a.out_rows || i < 0 || i >= a.level_len[l] || il < 0) {
     if (lane == 0) report_error(a.errw, ERRW_BOUNDS);
     return;
   }
   if (lane == 0) {
-    a.seq_map[bh * a.S + slot] = (int32_t)(((int64_t)l << 28) | i);
-    a.slot_of[bh * a.pyr_entries + a.level_off[l] + i] = (int32_t)slot;
+    a.seq_map[bh * a.out_rows + srow] = (int32_t)(((int64_t)l << 28) | il);
+    a.slot_of[bh * a.pyr_loc + a.level_off_loc[l] + il] = (int32_t)srow;
   }
   constexpr int CH = D / 8;
   if (l >= 1 && l < a.first_level) {
@@ -151,7 +167,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArg
     const float inv = __int_as_float((127 - l * a.log2p) << 23);  // 2^(-l log2p), exact
     for (int c = lane; c < 3 * CH; c += 32) {
       const int t = c / CH, off = (c % CH) * 8;
-      const T* src = static_cast<const T*>(a.x0[t]) + (bh * a.N + (i << (l * a.log2p))) * D + off;
+      const T* src = static_cast<const T*>(a.x0[t]) + (bh * a.n_loc + (il << (l * a.log2p))) * D + off;
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -170,9 +186,9 @@ __global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArg
       for (int e = 0; e < 8; ++e) acc[e] *= inv;
       if constexpr (sizeof(T) == 2) {
         // the materialised pyramid rounds the mean to bf16 once; do the same
-        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.S + slot) * D + off, acc);
+        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.out_rows + srow) * D + off, acc);
       } else {
-        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.S + slot) * D + off, acc);
+        store_vec<__nv_bfloat16, 8>(a.out[t] + (bh * a.out_rows + srow) * D + off, acc);
       }
     }
     return;
@@ -180,9 +196,9 @@ __global__ void __launch_bounds__(kGatherWarps * 32, 16) gather_kernel(GatherArg
   // copy the three rows, 8 elements per lane step, converting to bf16
   for (int c = lane; c < 3 * CH; c += 32) {
     const int t = c / CH, off = (c % CH) * 8;
-    const T* src = (l == 0) ? static_cast<const T*>(a.x0[t]) + (bh * a.N + i) * D
-                            : static_cast<const T*>(a.pyr[t]) + (bh * a.upper_entries + a.upper_off[l] + i) * D;
-    __nv_bfloat16* dst = a.out[t] + (bh * a.S + slot) * D + off;
+    const T* src = (l == 0) ? static_cast<const T*>(a.x0[t]) + (bh * a.n_loc + il) * D
+                            : static_cast<const T*>(a.pyr[t]) + (bh * a.upper_loc + a.upper_off_loc[l] + il) * D;
+    __nv_bfloat16* dst = a.out[t] + (bh * a.out_rows + srow) * D + off;
     if constexpr (sizeof(T) == 2) {
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src + off);
     } else {
@@ -210,6 +226,12 @@ struct ScatterArgs {
   int64_t tasks_per_head;
   int task_rows, log2p;
   int tbl_ints;  // slot indices of one task's entries of levels >= 1 (the streaming kernel's table)
+  // one shard of the tokens (context parallelism): the Os rows of the
+  // previous shard's last entry of each level l >= 1 ([BH][L-1][d], zeros
+  // where that entry is not kept), whose ranges reach this shard's first
+  // p^l - 1 rows; null for the whole layer
+  const float* halo;
+  int L;
 };
 
 template <typename T, int D>
@@ -312,7 +334,9 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_kernel(ScatterArgs a
 // their own boundaries: the top level's row once per top-level block, the
 // levels between it and level 1 summed at level-2 boundaries, level 1 at
 // level-1 boundaries.
-template <int NL>
+// HALO: one shard of the tokens with the previous shard's boundary rows (the
+// whole layer is compiled without them)
+template <int NL, bool HALO>
 __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(ScatterArgs a) {
   constexpr int D = 128;
   extern __shared__ int32_t sb_tbl[];
@@ -340,14 +364,16 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
       const int64_t i0 = (int64_t)(u0 >> (l * log2p)) - 1;
       for (int k = lane; k < n; k += 32) {
         const int64_t i = i0 + k;
-        tbl[off + k] = (i >= 0 && i < a.level_len[l]) ? so[a.level_off[l] + i] : -1;
+        // -1: no entry; -1 - l: the previous shard's entry of level l (halo)
+        tbl[off + k] = (i >= 0 && i < a.level_len[l]) ? so[a.level_off[l] + i] : ((HALO && i == -1) ? -1 - l : -1);
       }
       off += n;
     }
   }
   __syncwarp();
   auto add_row = [&](int slot, float (&acc)[8]) {
-    const float4* src = reinterpret_cast<const float4*>(os + (int64_t)slot * D);
+    const float4* src = reinterpret_cast<const float4*>(
+        (!HALO || slot >= 0) ? os + (int64_t)slot * D : a.halo + ((bh * (a.L - 1)) + (-2 - slot)) * D + cv * 8);
     const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
     acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
     acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
@@ -381,7 +407,7 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
 #pragma unroll
             for (int c = 0; c < 8; ++c) ctop[c] = 0.f;
             const int st = tbl[toff[NL - 1] + (r0 >> ((NL - 1) * log2p))];
-            if (st >= 0) add_row(st, ctop);
+            if (st != -1) add_row(st, ctop);
           }
           if constexpr (NL > 2) {
             if ((r0 & pm2) == 0) {
@@ -390,13 +416,13 @@ __global__ void __launch_bounds__(kWarps * 32) scatter_back_stream_kernel(Scatte
 #pragma unroll
               for (int l = 2; l < NL - 1; ++l) {
                 const int sl = tbl[toff[l] + (r0 >> (l * log2p))];
-                if (sl >= 0) add_row(sl, high);
+                if (sl != -1) add_row(sl, high);
               }
             }
 #pragma unroll
             for (int c = 0; c < 8; ++c) cs[c] = high[c];
             const int s1 = tbl[toff[1] + (r0 >> log2p)];
-            if (s1 >= 0) add_row(s1, cs);
+            if (s1 != -1) add_row(s1, cs);
           } else {
 #pragma unroll
             for (int c = 0; c < 8; ++c) cs[c] = ctop[c];
@@ -437,6 +463,10 @@ struct ScatterAdjArgs {
   int* errw;
   int64_t BH, N, S;
   int L, log2p;
+  // one shard of the tokens: the sums of dY over the next shard's first
+  // p^l - 1 rows ([BH][L-1][d] fp32), which the range of this shard's last
+  // entry of each level l >= 1 covers beyond its end; null for the whole layer
+  const float* halo;
 };
 
 template <typename T, int D>
@@ -484,6 +514,11 @@ __global__ void __launch_bounds__(kSadjWarps * 32) scatter_adjoint_kernel(Scatte
   for (int c = 0; c < VE; ++c)
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) acc[c] += __shfl_xor_sync(kFull, acc[c], o);
+  if (a.halo && l >= 1 && (i + 2) * b - 1 > a.N) {  // the range runs into the next shard
+    const float* hr = a.halo + (bh * (a.L - 1) + (l - 1)) * D + cv * VE;
+#pragma unroll
+    for (int c = 0; c < VE; ++c) acc[c] += hr[c];
+  }
   // round to bf16 once (stored as fp16, exact in range); Delta from the
   // rounded values and the fp32 Os
   __half h[VE];
@@ -508,6 +543,22 @@ __global__ void __launch_bounds__(kSadjWarps * 32) scatter_adjoint_kernel(Scatte
   }
 }
 
+// Sums of dY over the first p^l - 1 rows of every head, l = 1 .. L-1, in
+// fp32: under context parallelism, the part of the previous shard's last
+// level-l entry's range R(l, i) that lies in this shard.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) head_sums_kernel(const T* __restrict__ dy, float* __restrict__ sums, int64_t N,
+                                                      int L, int log2p) {
+  const int64_t bh = blockIdx.x;
+  const int l = (int)blockIdx.y + 1;
+  const int c = threadIdx.x;  // one channel per thread: each row read is one coalesced access
+  const int64_t rows = min(((int64_t)1 << (l * log2p)) - 1, N);
+  const T* src = dy + bh * N * D + c;
+  float acc = 0.f;
+  for (int64_t r = 0; r < rows; ++r) acc += Elem<T>::to_f(src[r * D]);
+  sums[(bh * (L - 1) + (l - 1)) * D + c] = acc;
+}
+
 template <typename T, int D>
 cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaStream_t st) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
@@ -516,7 +567,10 @@ cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaS
       const int64_t blocks = (tasks + kWarps - 1) / kWarps;
       switch (L) {
 #define LH_CASE(n) \
-  case n: scatter_back_stream_kernel<n><<<(unsigned)blocks, kWarps * 32, smem, st>>>(a); break;
+  case n:                                                                             \
+    if (a.halo) scatter_back_stream_kernel<n, true><<<(unsigned)blocks, kWarps * 32, smem, st>>>(a); \
+    else scatter_back_stream_kernel<n, false><<<(unsigned)blocks, kWarps * 32, smem, st>>>(a);       \
+    break;
         LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
 #undef LH_CASE
         default: return cudaErrorInvalidValue;
@@ -524,6 +578,7 @@ cudaError_t scatter_dispatch_L(int L, const ScatterArgs& a, int64_t tasks, cudaS
       return cudaGetLastError();
     }
   }
+  if (a.halo) return cudaErrorNotSupported;  // halo rows: the stream kernel's layouts only
   constexpr int R = RowLayout<T, D>::R;  // tasks per warp
   const int64_t blocks = ((tasks + R - 1) / R + kWarps - 1) / kWarps;
   switch (L) {
@@ -540,7 +595,10 @@ template <typename T, int D>
 cudaError_t gather_dispatch_L(int L, const GatherArgs& a, int64_t blocks, cudaStream_t st) {
   switch (L) {
 #define LH_CASE(n) \
-  case n: gather_kernel<T, D, n><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a); break;
+  case n:                                                                      \
+    if (a.seg_off) gather_kernel<T, D, n, true><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a); \
+    else gather_kernel<T, D, n, false><<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(a);         \
+    break;
     LH_CASE(1) LH_CASE(2) LH_CASE(3) LH_CASE(4) LH_CASE(5) LH_CASE(6) LH_CASE(7) LH_CASE(8)
 #undef LH_CASE
     default: return cudaErrorInvalidValue;
@@ -552,7 +610,8 @@ cudaError_t gather_dispatch_L(int L, const GatherArgs& a, int64_t blocks, cudaSt
 
 cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const void* v, const void* pq,
                           const void* pk, const void* pv, const int32_t* sel, void* qs, void* ks, void* vs,
-                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level) {
+                          int32_t* seq_map, int32_t* slot_of, int* errw, cudaStream_t st, int first_level,
+                          const Dims* shard, int64_t t0, const int64_t* seg_off, int64_t seg_rows) {
   GatherArgs a{};
   a.x0[0] = q; a.x0[1] = k; a.x0[2] = v;
   a.pyr[0] = pq; a.pyr[1] = pk; a.pyr[2] = pv;
@@ -589,7 +648,21 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
     ++a.rounds;
     a.stride0 *= 32;
   }
-  cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * D.pyr_entries * sizeof(int32_t), st);
+  // the shard (the whole layer unless one is given): its token range, row
+  // counts and table offsets
+  const Dims& Ls = shard ? *shard : D;
+  a.t0 = shard ? t0 : 0;
+  a.t1 = a.t0 + Ls.N;
+  a.seg_off = seg_off;
+  a.out_rows = shard ? seg_rows : D.S;
+  a.n_loc = Ls.N;
+  a.upper_loc = Ls.upper_entries;
+  a.pyr_loc = Ls.pyr_entries;
+  for (int l = 0; l < LH_MAX_LEVELS; ++l) {
+    a.upper_off_loc[l] = Ls.upper_off[l];
+    a.level_off_loc[l] = Ls.level_off[l];
+  }
+  cudaError_t e = cudaMemsetAsync(slot_of, 0xff, (size_t)D.BH * Ls.pyr_entries * sizeof(int32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (D.BH * D.S + kGatherWarps - 1) / kGatherWarps;
   if (D.dtype == LH_BF16) {
@@ -600,11 +673,14 @@ cudaError_t launch_gather(const Dims& D, const void* q, const void* k, const voi
                     : gather_dispatch_L<float, 64>(D.L, a, blocks, st);
 }
 
-cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st) {
+cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* slot_of, void* y, cudaStream_t st,
+                                const float* halo) {
   ScatterArgs a{};
   a.os = os;
   a.slot_of = slot_of;
   a.y = y;
+  a.halo = halo;
+  a.L = D.L;
   a.BH = D.BH; a.N = D.N; a.S = D.S; a.pyr_entries = D.pyr_entries;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) {
     a.level_off[l] = D.level_off[l];
@@ -627,8 +703,9 @@ cudaError_t launch_scatter_back(const Dims& D, const float* os, const int32_t* s
 }
 
 cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t* seq_map, const float* os,
-                                   void* dos, float* delta, int* errw, cudaStream_t st) {
+                                   void* dos, float* delta, int* errw, cudaStream_t st, const float* halo) {
   ScatterAdjArgs a{};
+  a.halo = halo;
   a.dy = dy;
   a.seq_map = seq_map;
   a.os = os;
@@ -645,6 +722,25 @@ cudaError_t launch_scatter_adjoint(const Dims& D, const void* dy, const int32_t*
   } else {
     if (D.d == 128) scatter_adjoint_kernel<float, 128><<<(unsigned)blocks, kSadjWarps * 32, 0, st>>>(a);
     else scatter_adjoint_kernel<float, 64><<<(unsigned)blocks, kSadjWarps * 32, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_sums(const Dims& D, const void* dy, float* sums, cudaStream_t st) {
+  if (D.L < 2) return cudaSuccess;
+  const dim3 grid((unsigned)D.BH, (unsigned)(D.L - 1));
+  if (D.dtype == LH_BF16) {
+    if (D.d == 128)
+      head_sums_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(dy), sums, D.N, D.L,
+                                                                   D.log2p);
+    else
+      head_sums_kernel<__nv_bfloat16, 64><<<grid, 64, 0, st>>>(static_cast<const __nv_bfloat16*>(dy), sums, D.N, D.L,
+                                                                 D.log2p);
+  } else {
+    if (D.d == 128)
+      head_sums_kernel<float, 128><<<grid, 128, 0, st>>>(static_cast<const float*>(dy), sums, D.N, D.L, D.log2p);
+    else
+      head_sums_kernel<float, 64><<<grid, 64, 0, st>>>(static_cast<const float*>(dy), sums, D.N, D.L, D.log2p);
   }
   return cudaGetLastError();
 }

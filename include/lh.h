@@ -245,6 +245,84 @@ lh_status lh_attn_bwd(const lh_config *cfg, int64_t S, const void *qs, const voi
                       const float *lse, const void *dos, const float *delta, float *dqs, float *dks, float *dvs,
                       void *ws, lh_stream_t stream);
 
+/* Stage 3 for one shard of the tokens (context parallelism: each GPU holds
+ * the tokens [t0, t1) of every head).  Cite: LH-post "How it works" (3) (the
+ * kept triples in causal order form one sequence); the entries whose key
+ * e = (i+1) p^l - 1 lies in [t0, t1) form one contiguous segment of that
+ * sequence, and their blocks lie inside the shard.
+ * In:  cfg and sel of the whole layer (the selection every shard shares);
+ *      t0 < t1 multiples of p^(L-1) in [0, N]; q, k, v [B][H][t1-t0][d] the
+ *      shard's tokens; pyr_q/k/v the shard's pyramid, as lh_pyramid_pool
+ *      writes it for a layer of the shard's t1 - t0 tokens (all levels);
+ *      seg_off [B*H] int64 on the device: the slot of each head's first
+ *      entry in the shard (the kept entries of the earlier shards).
+ * Out: qs, ks, vs [B*H][seg_rows][d] bf16 and seq_map [B*H][seg_rows]: row
+ *      r of head h is the entry at slot seg_off[h] + r (rows past the
+ *      head's segment are left as they are; seg_rows >= the longest
+ *      segment); seq_map holds (level << 28) | index within the shard's
+ *      level; slot_of [B*H][pyr_entries of the shard's layer]: the row of
+ *      each of the shard's entries in the segment, or -1.
+ * Errors: LH_ERR_INVALID_ARG for a bad range, seg_rows outside [1, S] or a
+ * NULL or misaligned pointer.  An entry whose segment row falls outside
+ * [0, seg_rows) (seg_off or seg_rows too small) is skipped without a report
+ * (the call takes no error word): size seg_rows from the selection. */
+lh_status lh_gather_shard(const lh_config *cfg, int64_t t0, int64_t t1, const int64_t *seg_off, int64_t seg_rows,
+                          const void *q, const void *k, const void *v, const void *pyr_q, const void *pyr_k,
+                          const void *pyr_v, const int32_t *sel, void *qs, void *ks, void *vs, int32_t *seq_map,
+                          int32_t *slot_of, lh_stream_t stream);
+
+/* Stages 5, 5 backward and 1 backward for one shard of the tokens (context
+ * parallelism), with cfg the layer of the shard's tokens (cfg->N = t1 - t0)
+ * and the shard's segment of seg_rows sequence rows per head in place of the
+ * plan's S (os, dos, delta, dqs/dks/dvs and seq_map as [B*H][seg_rows][...]).
+ * slot_of and seq_map are the shard's, as lh_gather_shard writes them; rows
+ * of seq_map past a head's segment must hold (0 << 28) | cfg->N (an empty
+ * range).  Each equals the whole-layer call on the shard's rows except where
+ * an entry's range R(l, i) crosses the shard's edge:
+ *  - lh_scatter_back_shard adds halo [B*H][L-1][d] fp32: for l >= 1 the Os row
+ *    of the previous shard's last level-l entry (zeros where it is not kept;
+ *    all zeros on the first shard), whose range covers this shard's first
+ *    p^l - 1 rows; the sum is rounded once.  bf16 rows of 128 channels only
+ *    (else LH_ERR_UNSUPPORTED).
+ *  - lh_scatter_back_adjoint_shard adds halo [B*H][L-1][d] fp32 (NULL on the
+ *    last shard): for l >= 1 the next shard's sum of dY over its first
+ *    p^l - 1 rows (lh_head_sums), to this shard's last level-l entry before
+ *    the rounding and delta.
+ *  - lh_pool_adjoint_shard: no halo (an entry's block lies in its shard).
+ * lh_head_sums writes sums [B*H][L-1][d] fp32: for l = 1 .. L-1 the sum of
+ * dY over the first p^l - 1 rows of each head (the part of the previous
+ * shard's last level-l range that lies in this shard).
+ * Errors as the whole-layer calls, and LH_ERR_INVALID_ARG for seg_rows
+ * outside [1, 2^31). */
+lh_status lh_scatter_back_shard(const lh_config *cfg, int64_t seg_rows, const float *os, const int32_t *slot_of,
+                                const float *halo, void *y, lh_stream_t stream);
+lh_status lh_scatter_back_adjoint_shard(const lh_config *cfg, int64_t seg_rows, const void *dy,
+                                        const int32_t *seq_map, const float *os, const float *halo, void *dos,
+                                        float *delta, lh_stream_t stream);
+lh_status lh_pool_adjoint_shard(const lh_config *cfg, int64_t seg_rows, const float *dqs, const float *dks,
+                                const float *dvs, const int32_t *slot_of, void *dq, void *dk, void *dv,
+                                lh_stream_t stream);
+lh_status lh_head_sums(const lh_config *cfg, const void *dy, float *sums, lh_stream_t stream);
+
+/* Stage 4 over a row window of the sequence: the rows [row_lo, row_hi) of
+ * lh_attn_fwd's os and lse (each query row still attends every key row up to
+ * itself), for running the attention of one sequence in pieces (one piece per
+ * GPU under context parallelism).  row_lo a multiple of 128; row_hi a
+ * multiple of 128 or S.  Rows outside the window are not written; an empty
+ * window queues nothing.  Other arguments and errors as lh_attn_fwd; the
+ * window's rows equal lh_attn_fwd's bit for bit. */
+lh_status lh_attn_fwd_rows(const lh_config *cfg, int64_t S, int64_t row_lo, int64_t row_hi, const void *qs,
+                           const void *ks, const void *vs, float *os, float *lse, void *ws, lh_stream_t stream);
+
+/* Stage 4 backward over row windows: dqs rows [q_lo, q_hi) and dks, dvs rows
+ * [k_lo, k_hi) of lh_attn_bwd (every query and key row of the sequence is
+ * read).  Each bound as for lh_attn_fwd_rows; either window may be empty.
+ * Rows outside the windows are not written; the windows' rows equal
+ * lh_attn_bwd's bit for bit. */
+lh_status lh_attn_bwd_rows(const lh_config *cfg, int64_t S, int64_t q_lo, int64_t q_hi, int64_t k_lo, int64_t k_hi,
+                           const void *qs, const void *ks, const void *vs, const float *lse, const void *dos,
+                           const float *delta, float *dqs, float *dks, float *dvs, void *ws, lh_stream_t stream);
+
 /* Stage 5 - scatter-back.  Cite: LH-summary "Technical details" (4) (outputs
  * return to the N positions and each position j sums over the ranges
  * R(l, i)); LH-post "How it works" (4) (shifted ranges keep causality).

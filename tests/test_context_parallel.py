@@ -172,21 +172,25 @@ class OracleBackend:
             lse.append(torch.from_numpy(ls[a:b]))
         return torch.stack(os_), torch.stack(lse)
 
-    def scatter(self, os_seg, seq):
-        return torch.stack([torch.from_numpy(lo.scatter_back(os_seg[h, :len(lv)].numpy(), lv, ix, self.n, self.p,
-                                                             self.L)) for h, (lv, ix) in enumerate(seq)])
+    def scatter(self, os_seg, seq, os_all, halo):
+        y = torch.stack([torch.from_numpy(lo.scatter_back(os_seg[h, :len(lv)].numpy(), lv, ix, self.n, self.p,
+                                                          self.L)) for h, (lv, ix) in enumerate(seq)])
+        for h, ents in enumerate(halo):
+            for l, slot, rows in ents:
+                y[h, :rows] += os_all[h, slot]
+        return y
 
-    def halo_add_y(self, y, h, rows, row):
-        y[h, :rows] += row
+    def head_sums(self, dy):
+        return torch.stack([dy[:, :self.p ** l - 1].sum(dim=1) for l in range(1, self.L)], dim=1)
 
-    def scatter_adjoint(self, dy, seq):
+    def scatter_adjoint(self, dy, seq, os_seg, nxt):
         mx = max(len(s[0]) for s in seq)
-        out = torch.zeros((dy.shape[0], mx, self.d), dtype=torch.float64)
+        dos = torch.zeros((dy.shape[0], mx, self.d), dtype=torch.float64)
         for h, (lv, ix) in enumerate(seq):
-            out[h, :len(lv)] = torch.from_numpy(lo.scatter_adjoint(dy[h].numpy(), lv, ix, self.n, self.p))
-        return out
-
-    def finish_dos(self, dos, os_seg):
+            dos[h, :len(lv)] = torch.from_numpy(lo.scatter_adjoint(dy[h].numpy(), lv, ix, self.n, self.p))
+            if nxt is not None:
+                for l, s in cp.halo_out_entries(lv, ix, self.shard):
+                    dos[h, s] += nxt[h, l - 1]
         return dos, (dos * os_seg).sum(-1)
 
     def _bwd(self, qs, ks, vs, dos):

@@ -250,3 +250,30 @@ def test_pool_adjoint(name):
             lv = lo.gather_adjoint(np.float32(o[src]).astype(np.float64), sv["seq_level"], sv["seq_index"], w.N, w.p, w.L)
             want = lo.pyramid_pool_adjoint(lv, w.p)
             pu.assert_close(got.reshape(w.B * w.H, w.N, w.d)[bh], want, f"{name} {t}")
+
+
+@pytest.mark.parametrize("BH,S,d,cuts", [(2, 1000, 128, (0, 384, 640, 1000)), (1, 300, 64, (0, 128, 300)),
+                                         (3, 777, 128, (0, 0, 256, 777))])
+def test_attn_row_windows(BH, S, d, cuts):
+    """The attention over row windows (the pieces context parallelism runs on
+    different GPUs) equals the whole-sequence kernels bit for bit, row by row,
+    whatever the cuts (empty windows included)."""
+    g = torch.Generator().manual_seed(S + d)
+    qs, ks, vs = (torch.randn(BH, S, d, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    L = lh.Layer(1, BH, 4096, d, 3, 2, 8)
+    os_full, lse_full = lh.attn_fwd(L, qs, ks, vs)
+    os_w = torch.full_like(os_full, float("nan"))
+    lse_w = torch.full_like(lse_full, float("nan"))
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        lh.attn_fwd_rows(L, qs, ks, vs, lo, hi, os_w, lse_w)
+    torch.cuda.synchronize()
+    assert torch.equal(os_w, os_full) and torch.equal(lse_w, lse_full)
+    dos = torch.randn(BH, S, d, generator=g).to(torch.bfloat16).to(torch.float16).cuda()
+    delta = (dos.float() * os_full).sum(-1).contiguous()
+    dq, dk, dv = lh.attn_bwd(L, qs, ks, vs, lse_full, dos, delta)
+    dq_w, dk_w, dv_w = (torch.full_like(dq, float("nan")) for _ in range(3))
+    # query windows in order, key windows in reverse order (independent pieces)
+    for (qlo, qhi), (klo, khi) in zip(zip(cuts[:-1], cuts[1:]), reversed(list(zip(cuts[:-1], cuts[1:])))):
+        lh.attn_bwd_rows(L, qs, ks, vs, lse_full, dos, delta, (qlo, qhi), (klo, khi), dq_w, dk_w, dv_w)
+    torch.cuda.synchronize()
+    assert torch.equal(dq_w, dq) and torch.equal(dk_w, dk) and torch.equal(dv_w, dv)
