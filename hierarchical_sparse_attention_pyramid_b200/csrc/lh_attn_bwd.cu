@@ -61,7 +61,6 @@ constexpr int kComputeKV = 512;  // dK/dV kernel: four compute warpgroups
 constexpr int kThreadsKV = kComputeKV + 64;
 constexpr int kRegion = 128 * 128;  // one [128 rows][64 bf16] SW128 region
 
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void compute_sync_kv() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
 // P^T / dS (hi, lo) of 32 columns c0..c0+31 of one row as bf16 pairs over the
@@ -316,7 +315,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       const int q0 = (kt + j) * 128;
       const bool diag = j == 0;  // the diagonal query tile
       // warp-uniform outcome for the collective TMEM accesses; after a failed
-      // wait the loop keeps its compute_sync count and skips the work
+      // wait the loop keeps its compute_sync_kv count and skips the work
       ok = __all_sync(0xffffffffu, ok && mbar_wait(bS, j & 1, abort_flag));
       if (!ok) continue;
       tc_fence_after();
@@ -454,7 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::oBar + 196);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = (S + 127) / 128;
   // one CTA per (query tile, head) of the query tiles [qt0, qt1), tile-major
   // with the longest rows first
   const int BHn = (int)(gridDim.x / (unsigned)(qt1 - qt0));
