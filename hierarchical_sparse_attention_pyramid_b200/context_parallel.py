@@ -245,6 +245,33 @@ def allgather_rows(x: torch.Tensor, counts, group=None) -> torch.Tensor:
     return torch.cat([p[:, :int(c)] for p, c in zip(parts, counts)], dim=1)
 
 
+def segment_index(counts: np.ndarray, mx: int) -> np.ndarray:
+    """Where each head's sequence rows sit once every rank's segments are
+    gathered as one [W, BH, mx] block of rows: for head h and sequence row s,
+    the flat row r*BH*mx + h*mx + j of segment row j of rank r.  [BH, S]."""
+    W, BH = counts.shape
+    return np.stack([np.concatenate([r * BH * mx + h * mx + np.arange(int(counts[r, h]), dtype=np.int64)
+                                     for r in range(W)]) for h in range(BH)])
+
+
+def allgather_segments(x: torch.Tensor, counts: np.ndarray, group=None) -> torch.Tensor:
+    """The whole sequence of every head from each rank's segments, in one
+    collective.  x on rank r: [BH, >= counts[r, h], ...], rows past a head's
+    count ignored; counts: [W, BH], every head's column summing to the same S.
+    Returns [BH, S, ...]."""
+    import torch.distributed as dist
+    W, BH = counts.shape
+    mx = max(1, int(counts.max()))
+    rest = tuple(x.shape[2:])
+    pad = torch.zeros((BH, mx) + rest, dtype=x.dtype, device=x.device)
+    m = min(mx, x.shape[1])
+    pad[:, :m] = x[:, :m]
+    parts = [torch.empty_like(pad) for _ in range(dist.get_world_size(group))]
+    _all_gather(parts, pad, group=group)
+    idx = torch.from_numpy(segment_index(counts, mx)).to(x.device)
+    return torch.stack(parts).reshape((W * BH * mx,) + rest)[idx.reshape(-1)].reshape((BH, idx.shape[1]) + rest)
+
+
 # ---------------------------------------------------------------- driver
 
 @dataclass
@@ -264,10 +291,14 @@ class CpContext:
 def _segment_rows(full: torch.Tensor, off, counts_r) -> torch.Tensor:
     """Rows [off_h, off_h + S_r,h) of every head (same count for every head is
     not assumed: heads are padded to the largest with zeros)."""
+    BH = full.shape[0]
     mx = int(max(counts_r))
-    out = torch.zeros((full.shape[0], mx) + tuple(full.shape[2:]), dtype=full.dtype, device=full.device)
-    for h in range(full.shape[0]):
-        out[h, :int(counts_r[h])] = full[h, int(off[h]):int(off[h]) + int(counts_r[h])]
+    j = np.arange(mx, dtype=np.int64)[None, :]
+    valid = j < np.asarray(counts_r, np.int64)[:, None]
+    src = np.where(valid, np.asarray(off, np.int64)[:, None] + j, 0)
+    dev = full.device
+    out = full[torch.arange(BH, device=dev)[:, None], torch.from_numpy(src).to(dev)]
+    out[torch.from_numpy(~valid).to(dev)] = 0
     return out
 
 
@@ -283,12 +314,9 @@ def cp_forward(backend, shard: Shard, q, k, v, selection: str = "parents", group
     off = counts[:r].sum(axis=0)
     sel_loc = [local_selection(sel[h], shard, selection) for h in range(BH)]
     seq, (qs_r, ks_r, vs_r) = backend.gather(q, k, v, levels, sel_loc)
-    # the whole sequence on every rank (heads differ in S_r: gathered per head)
-    full = []
-    for t in (qs_r, ks_r, vs_r):
-        full.append(torch.stack([allgather_rows(t[h:h + 1, :int(counts[r, h])], counts[:, h], group)[0]
-                                 for h in range(BH)]))
-    qs, ks, vs = full
+    # the whole sequence on every rank: one collective for Qs, Ks and Vs of all heads
+    qkv = allgather_segments(torch.stack((qs_r, ks_r, vs_r), dim=2), counts, group)
+    qs, ks, vs = (qkv[:, :, t].contiguous() for t in range(3))
     S = qs.shape[1]
     lo, hi = balanced_windows(S, W, "query")[r]
     os_w, lse_w = backend.attention(qs, ks, vs, lo, hi)
@@ -303,18 +331,15 @@ def cp_forward(backend, shard: Shard, q, k, v, selection: str = "parents", group
 
 def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     """Backward of this rank's shard.  dy: [BH, n, d].  Returns dq, dk, dv [BH, n, d]."""
-    BH = dy.shape[0]
-    W, r, p, L = shard.world, shard.rank, shard.p, shard.L
+    W, r, L = shard.world, shard.rank, shard.L
     # halo: sums of dY over this shard's first p^l - 1 tokens, for the previous shard
     nxt = None
     if L > 1:
         heads_all = allgather_cat(backend.head_sums(dy)[None], dim=0, group=group)  # [W, BH, L-1, d]
         nxt = heads_all[r + 1] if r + 1 < W else None
     dos, delta = backend.scatter_adjoint(dy, ctx.seq, _segment_rows(ctx.os, ctx.off, ctx.counts[r]), nxt)
-    dos_f = torch.stack([allgather_rows(dos[h:h + 1, :int(ctx.counts[r, h])], ctx.counts[:, h], group)[0]
-                         for h in range(BH)])
-    delta_f = torch.stack([allgather_rows(delta[h:h + 1, :int(ctx.counts[r, h]), None], ctx.counts[:, h],
-                                          group)[0, :, 0] for h in range(BH)])
+    dos_f = allgather_segments(dos, ctx.counts, group)
+    delta_f = allgather_segments(delta, ctx.counts, group)
     S = ctx.qs.shape[1]
     klo, khi = balanced_windows(S, W, "key")[r]
     qlo, qhi = balanced_windows(S, W, "query")[r]
@@ -322,8 +347,8 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     dqs_w = backend.attention_bwd_q(ctx.qs, ctx.ks, ctx.vs, ctx.lse, dos_f, delta_f, qlo, qhi)
     kwin = [b - a for a, b in balanced_windows(S, W, "key")]
     qwin = [b - a for a, b in balanced_windows(S, W, "query")]
-    dks = _segment_rows(allgather_rows(dks_w, kwin, group), ctx.off, ctx.counts[r])
-    dvs = _segment_rows(allgather_rows(dvs_w, kwin, group), ctx.off, ctx.counts[r])
+    dkv = _segment_rows(allgather_rows(torch.stack((dks_w, dvs_w), dim=2), kwin, group), ctx.off, ctx.counts[r])
+    dks, dvs = dkv[:, :, 0], dkv[:, :, 1]
     dqs = _segment_rows(allgather_rows(dqs_w, qwin, group), ctx.off, ctx.counts[r])
     return backend.pool_adjoint(dqs, dks, dvs, ctx.seq)
 

@@ -253,3 +253,43 @@ def test_sharded_layer_matches_unsharded_oracle(name, world):
         got = np.concatenate([out[r][t] for r in range(world)], axis=1)
         for h in range(H):
             np.testing.assert_allclose(got[h], want[h][t], rtol=1e-9, atol=1e-11, err_msg=f"{name} {nm} head {h}")
+
+
+def _count_main(rank, world, port, name, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    calls = []
+    real = cp._all_gather
+
+    def counting(parts, x, group=None):
+        calls.append(tuple(x.shape))
+        real(parts, x, group=group)
+
+    cp._all_gather = counting
+    try:
+        case = CASES[name]
+        N, d, L, p, kk, T, H, selection, scorer = case
+        q, k, v, dy = (torch.from_numpy(x) for x in _inputs(N, d, H, 3))
+        shard = cp.Shard(N, p, L, world, rank)
+        sl = slice(shard.t0, shard.t1)
+        be = OracleBackend(case, shard)
+        y, ctx = cp.cp_forward(be, shard, q[:, sl], k[:, sl], v[:, sl], selection)
+        n_fwd = len(calls)
+        cp.cp_backward(be, shard, dy[:, sl].contiguous(), ctx)
+        out[rank] = (n_fwd, len(calls) - n_fwd)
+    finally:
+        cp._all_gather = real
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", ["p2_L3", "direct_p2_L4"])
+def test_collectives_per_layer_do_not_grow_with_heads(name):
+    """One all-gather per exchanged quantity, whatever the number of heads:
+    forward norms, Qs|Ks|Vs, Os, LSE; backward head sums, dOs, Delta,
+    dKs|dVs, dQs."""
+    out = mp.Manager().dict()
+    mp.spawn(_count_main, args=(2, _free_port(), name, out), nprocs=2, join=True)
+    assert [out[r] for r in range(2)] == [(4, 5), (4, 5)]
