@@ -348,12 +348,20 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     kwin = [b - a for a, b in balanced_windows(S, W, "key")]
     qwin = [b - a for a, b in balanced_windows(S, W, "query")]
     dkv = _segment_rows(allgather_rows(torch.stack((dks_w, dvs_w), dim=2), kwin, group), ctx.off, ctx.counts[r])
-    dks, dvs = dkv[:, :, 0], dkv[:, :, 1]
+    dks, dvs = dkv[:, :, 0].contiguous(), dkv[:, :, 1].contiguous()
     dqs = _segment_rows(allgather_rows(dqs_w, qwin, group), ctx.off, ctx.counts[r])
     return backend.pool_adjoint(dqs, dks, dvs, ctx.seq)
 
 
 # ---------------------------------------------------------------- the CUDA backend
+
+def _contiguous(*ts):
+    """Contiguous forms of the tensors, held by the caller until its library
+    call has been issued: a pointer taken from a temporary `.contiguous()`
+    copy dangles once the copy is freed, and the allocator hands that memory
+    to the next copy."""
+    return tuple(t.contiguous() for t in ts)
+
 
 class CudaBackend:
     """The per-rank arithmetic in the library's kernels: the whole-layer stage
@@ -411,11 +419,11 @@ class CudaBackend:
         self.seq_map = torch.full((lay.BH, self.seg_rows), sh.n, dtype=torch.int32, device=dev)
         self.slot_of = torch.empty((lay.BH, self.local_info.pyr_entries), dtype=torch.int32, device=dev)
         pq, pk, pv = levels
+        q, k, v = _contiguous(q, k, v)
         p_ = self.api._p
         _lib.call("lh_gather_shard", ctypes.byref(lay.cfg()), ctypes.c_int64(sh.t0), ctypes.c_int64(sh.t1),
-                  p_(seg_off), ctypes.c_int64(self.seg_rows), p_(q.contiguous()), p_(k.contiguous()),
-                  p_(v.contiguous()), p_(pq), p_(pk), p_(pv), p_(self.sel), p_(qs), p_(ks), p_(vs),
-                  p_(self.seq_map), p_(self.slot_of), self.api._stream())
+                  p_(seg_off), ctypes.c_int64(self.seg_rows), p_(q), p_(k), p_(v), p_(pq), p_(pk), p_(pv),
+                  p_(self.sel), p_(qs), p_(ks), p_(vs), p_(self.seq_map), p_(self.slot_of), self.api._stream())
         sm = self.seq_map.cpu().numpy().astype(np.int64)
         seq = [((sm[h, :c] >> 28), (sm[h, :c] & ((1 << 28) - 1))) for h, c in enumerate(self.counts_r)]
         return seq, (qs, ks, vs)
@@ -432,16 +440,18 @@ class CudaBackend:
             for l, slot, rows in ents:
                 hal[h, l - 1] = os_all[h, slot]
         y = torch.empty((lay.B, lay.H, self.shard.n, lay.d), dtype=torch.bfloat16, device=os_seg.device)
+        (os_seg,) = _contiguous(os_seg)
         p_ = self.api._p
         _lib.call("lh_scatter_back_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
-                  p_(os_seg.contiguous()), p_(self.slot_of), p_(hal), p_(y), self.api._stream())
+                  p_(os_seg), p_(self.slot_of), p_(hal), p_(y), self.api._stream())
         return y.reshape(lay.BH, self.shard.n, lay.d)
 
     def head_sums(self, dy):
         from . import _lib
         lay = self.layer
         sums = torch.empty((lay.BH, lay.L - 1, lay.d), dtype=torch.float32, device=dy.device)
-        _lib.call("lh_head_sums", ctypes.byref(self.local.cfg()), self.api._p(dy.contiguous()), self.api._p(sums),
+        (dy,) = _contiguous(dy)
+        _lib.call("lh_head_sums", ctypes.byref(self.local.cfg()), self.api._p(dy), self.api._p(sums),
                   self.api._stream())
         return sums
 
@@ -450,10 +460,13 @@ class CudaBackend:
         lay = self.layer
         dos = torch.zeros((lay.BH, self.seg_rows, lay.d), dtype=torch.float16, device=dy.device)
         delta = torch.zeros((lay.BH, self.seg_rows), dtype=torch.float32, device=dy.device)
+        dy, os_seg = _contiguous(dy, os_seg)
+        if nxt is not None:
+            (nxt,) = _contiguous(nxt)
         p_ = self.api._p
         _lib.call("lh_scatter_back_adjoint_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
-                  p_(dy.contiguous()), p_(self.seq_map), p_(os_seg.contiguous()),
-                  p_(nxt.contiguous()) if nxt is not None else None, p_(dos), p_(delta), self.api._stream())
+                  p_(dy), p_(self.seq_map), p_(os_seg), p_(nxt) if nxt is not None else None, p_(dos), p_(delta),
+                  self.api._stream())
         return dos, delta
 
     def _bwd(self, qs, ks, vs, lse, dos, delta, q_rows, k_rows):
@@ -473,8 +486,8 @@ class CudaBackend:
         lay = self.layer
         shp = (lay.B, lay.H, self.shard.n, lay.d)
         dq, dk, dv = (torch.empty(shp, dtype=torch.bfloat16, device=dqs.device) for _ in range(3))
+        dqs, dks, dvs = _contiguous(dqs, dks, dvs)
         p_ = self.api._p
         _lib.call("lh_pool_adjoint_shard", ctypes.byref(self.local.cfg()), ctypes.c_int64(self.seg_rows),
-                  p_(dqs.contiguous()), p_(dks.contiguous()), p_(dvs.contiguous()), p_(self.slot_of), p_(dq),
-                  p_(dk), p_(dv), self.api._stream())
+                  p_(dqs), p_(dks), p_(dvs), p_(self.slot_of), p_(dq), p_(dk), p_(dv), self.api._stream())
         return tuple(t.reshape(lay.BH, self.shard.n, lay.d) for t in (dq, dk, dv))

@@ -198,3 +198,17 @@ def test_selftest_timeout_argument_checks(lib):
                                         None) == 1
     assert lib.lh_selftest_wait_timeout(None, ctypes.c_size_t(_lib.SELFTEST_WS_BYTES), ctypes.c_int64(1000),
                                         None) == 1
+
+
+def test_no_pointer_from_a_temporary():
+    """A pointer handed to the library must come from a tensor that outlives
+    the call's launch: `_p(x.contiguous())` frees the copy as soon as the
+    pointer is taken, and the allocator gives that memory to the next copy."""
+    pkg = os.path.join(ROOT, "hierarchical_sparse_attention_pyramid_b200")
+    bad = re.compile(r"\b_?p_?\([^()]*\.contiguous\(\)\)")
+    hits = []
+    for f in sorted(os.listdir(pkg)):
+        if f.endswith(".py"):
+            with open(os.path.join(pkg, f)) as fh:
+                hits += [f"{f}:{i + 1}" for i, line in enumerate(fh) if bad.search(line)]
+    assert not hits, hits
