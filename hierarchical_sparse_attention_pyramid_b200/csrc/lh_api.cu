@@ -351,6 +351,10 @@ lh_status lh_gather_shard(const lh_config* cfg, int64_t t0, int64_t t1, const in
   return LH_OK;
 }
 
+// the kernels' default bound on each of their waits, in SM clock cycles
+// (about 2 s at the B200's 1965 MHz maximum)
+constexpr long long kLaunchWaitCycles = 4000000000ll;
+
 // a row window [lo, hi) of the sequence as 128-row tiles: lo a multiple of
 // 128, hi a multiple of 128 or S
 static bool tile_window(int64_t S, int64_t lo, int64_t hi, int64_t* t0, int64_t* t1) {
@@ -374,7 +378,7 @@ lh_status lh_attn_fwd_rows(const lh_config* cfg, int64_t S, int64_t row_lo, int6
   if (t0 == t1) return LH_OK;
   LH_CHECK_PTR(qs); LH_CHECK_PTR(ks); LH_CHECK_PTR(vs); LH_CHECK_PTR(os); LH_CHECK_PTR(lse); LH_CHECK_PTR(ws);
   LH_CUDA(launch_attn_fwd(cfg->B * cfg->H, S, cfg->d, qs, ks, vs, os, lse, err_word(ws), (cudaStream_t)stream,
-                          4000000000ll, 1, t0, t1),
+                          kLaunchWaitCycles, 1, t0, t1),
           "lh_attn_fwd_rows");
   return LH_OK;
 }
@@ -569,7 +573,7 @@ lh_status lh_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t wait_cycle
   LH_CHECK_PTR(ws);
   if (ws_bytes < LH_SELFTEST_WS_BYTES)
     return fail(LH_ERR_WORKSPACE, "lh_selftest_wait_timeout: ws smaller than LH_SELFTEST_WS_BYTES");
-  if (wait_cycles < 1 || wait_cycles > 4000000000ll)
+  if (wait_cycles < 1 || wait_cycles > kLaunchWaitCycles)
     return fail(LH_ERR_INVALID_ARG, "lh_selftest_wait_timeout: wait_cycles outside [1, 4e9]");
   // one 128 x 64 tile each of Qs, Ks, Vs (bf16, 16 KB) after the error word,
   // then O (fp32, 32 KB) and LSE (512 B): 256 + 3 * 16384 + 32768 + 512 bytes
