@@ -121,6 +121,59 @@ def test_failure_paths_return_before_any_gpu_work(lib):
     assert lib.lh_attn_fwd(ctypes.byref(bad), 100, fake, fake, fake, fake, fake, fake, None) == 2
 
 
+def test_shard_and_window_calls_reject_bad_arguments_before_any_launch(lib):
+    """The context-parallel entry points refuse, on the host, token windows
+    that split a top-level block, row windows that are not tile-aligned,
+    segment sizes out of range, unsupported layouts and missing pointers; an
+    empty attention window is a successful no-op.  No case reaches a launch."""
+    cfg = _lib.LhConfig(1, 2, 4096, 128, 3, 2, 16, 0, 0, 0, 0)  # bf16, p^(L-1) = 4
+    info = _lib.LhPlanInfo()
+    assert lib.lh_plan(ctypes.byref(cfg), ctypes.byref(info)) == 0
+    S = info.S
+    fake = ctypes.c_void_p(1 << 40)  # never dereferenced
+    I64 = ctypes.c_int64
+
+    def gather(t0, t1, seg_off, seg_rows):
+        return lib.lh_gather_shard(ctypes.byref(cfg), I64(t0), I64(t1), seg_off, I64(seg_rows), *([fake] * 12), None)
+
+    assert gather(2, 2050, fake, 10) == 1       # t0 inside a top-level block
+    assert gather(0, 4100, fake, 10) == 1       # past N
+    assert gather(2048, 2048, fake, 10) == 1    # empty shard
+    assert gather(0, 2048, fake, 0) == 1        # no segment rows
+    assert gather(0, 2048, fake, S + 1) == 1    # more rows than the whole sequence
+    assert gather(0, 2048, None, 10) == 1       # no segment offsets
+    assert "lh_gather_shard" in lib.lh_last_error_message().decode()
+
+    def fwd(lo, hi):
+        return lib.lh_attn_fwd_rows(ctypes.byref(cfg), I64(S), I64(lo), I64(hi), *([fake] * 6), None)
+
+    assert fwd(64, 256) == 1       # lo not on a tile edge
+    assert fwd(0, S + 128) == 1    # past S
+    assert fwd(256, 128) == 1      # reversed
+    assert fwd(0, 1000) == 1       # hi neither on a tile edge nor S
+    assert fwd(256, 256) == 0      # empty: nothing to do
+
+    def bwd(qlo, qhi, klo, khi):
+        return lib.lh_attn_bwd_rows(ctypes.byref(cfg), I64(S), I64(qlo), I64(qhi), I64(klo), I64(khi),
+                                    *([fake] * 10), None)
+
+    assert bwd(64, 128, 0, 0) == 1
+    assert bwd(0, 0, 0, 1000) == 1
+    assert bwd(128, 128, 0, 0) == 0
+
+    shard = _lib.LhConfig(1, 2, 2048, 128, 3, 2, 16, 0, 0, 0, 0)  # one shard's layer
+    assert lib.lh_scatter_back_shard(ctypes.byref(shard), I64(0), fake, fake, fake, fake, None) == 1
+    assert lib.lh_scatter_back_shard(ctypes.byref(shard), I64(10), fake, fake, None, fake, None) == 1  # no halo
+    narrow = _lib.LhConfig(1, 2, 2048, 64, 3, 2, 16, 0, 0, 0, 0)
+    assert lib.lh_scatter_back_shard(ctypes.byref(narrow), I64(10), fake, fake, fake, fake, None) == 2
+    assert lib.lh_scatter_back_adjoint_shard(ctypes.byref(shard), I64(1 << 31), *([fake] * 6), None) == 1
+    assert lib.lh_scatter_back_adjoint_shard(ctypes.byref(shard), I64(10), None, *([fake] * 5), None) == 1
+    assert lib.lh_pool_adjoint_shard(ctypes.byref(shard), I64(-1), *([fake] * 7), None) == 1
+    assert lib.lh_pool_adjoint_shard(ctypes.byref(shard), I64(10), fake, fake, fake, None, fake, fake, fake,
+                                     None) == 1
+    assert lib.lh_head_sums(ctypes.byref(shard), None, fake, None) == 1
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.lh_status_string(s).decode()
