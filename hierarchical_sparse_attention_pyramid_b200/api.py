@@ -69,6 +69,40 @@ def _p(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(name: str, t, dtype=None, numel: int | None = None, min_numel: int | None = None, shape=None):
+    """Host check of a tensor argument before its pointer reaches the library,
+    which cannot see sizes: a wrong size would make a kernel read or write
+    outside the tensor."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected at least {min_numel}")
+
+
+def _need_qkv(layer: "Layer", **ts) -> None:
+    """Token-major tensors of the layer: B*H*N*d elements ([B, H, N, d] or [B*H, N, d]) in the layer's dtype."""
+    for name, t in ts.items():
+        _need(name, t, layer.torch_dtype, numel=layer.BH * layer.N * layer.d)
+
+
+def _need_seq(layer: "Layer", qs, **ts) -> int:
+    """Sequence tensors: qs [B*H, S, d] bf16 (S from qs), the others of the same
+    rows: name -> (tensor, dtype, trailing dims).  Returns S."""
+    if not isinstance(qs, torch.Tensor) or qs.dim() != 3 or qs.shape[0] != layer.BH or qs.shape[2] != layer.d:
+        raise ValueError(f"qs: shape {tuple(getattr(qs, 'shape', ()))}, expected ({layer.BH}, S, {layer.d})")
+    _need("qs", qs, torch.bfloat16)
+    S = qs.shape[1]
+    for name, (t, dtype, tail) in ts.items():
+        _need(name, t, dtype, shape=(layer.BH, S) + tail)
+    return S
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -86,6 +120,7 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 def pyramid_pool(layer: Layer, q, k, v, first_level: int | None = None):
     """-> pyr_q, pyr_k, pyr_v [BH, upper_entries, d] (levels >= 1), norms [2, BH, N] fp32.
     With first_level (lh_pyramid_pool_from), levels below it are not written (rows left zero here)."""
+    _need_qkv(layer, q=q, k=k, v=v)
     info = plan(layer)
     dev = q.device
     shp = (layer.BH, max(info.upper_entries, 1), layer.d)
@@ -103,7 +138,10 @@ def pyramid_pool(layer: Layer, q, k, v, first_level: int | None = None):
 
 def score_topk(layer: Layer, norms, ws=None):
     """-> sel [BH, sel_per_head] int32 (per level l at sel_off[l], ascending parents at level l+1)."""
+    _need("norms", norms, torch.float32, numel=2 * layer.BH * layer.N)
     info = plan(layer)
+    if ws is not None and ws.numel() * ws.element_size() < max(info.topk_ws_bytes, _lib.ERR_WORD_BYTES):
+        raise ValueError(f"ws: {ws.numel() * ws.element_size()} bytes, expected at least {info.topk_ws_bytes}")
     dev = norms.device
     sel = torch.zeros((layer.BH, max(info.sel_per_head, 1)), dtype=torch.int32, device=dev)
     ws = _ws(info.topk_ws_bytes, dev) if ws is None else ws
@@ -114,7 +152,11 @@ def score_topk(layer: Layer, norms, ws=None):
 def gather(layer: Layer, q, k, v, pq, pk, pv, sel, first_level: int | None = None):
     """-> qs, ks, vs [BH, S, d] bf16, seq_map [BH, S] int32, slot_of [BH, pyr_entries] int32.
     With first_level (lh_gather_from), kept entries of the levels below it are averaged from q, k, v."""
+    _need_qkv(layer, q=q, k=k, v=v)
     info = plan(layer)
+    for name, t in (("pq", pq), ("pk", pk), ("pv", pv)):
+        _need(name, t, layer.torch_dtype, min_numel=layer.BH * info.upper_entries * layer.d)
+    _need("sel", sel, torch.int32, min_numel=layer.BH * info.sel_per_head)
     dev = q.device
     S = info.S
     qs, ks, vs = (_empty((layer.BH, S, layer.d), torch.bfloat16, dev) for _ in range(3))
@@ -131,6 +173,7 @@ def gather(layer: Layer, q, k, v, pq, pk, pv, sel, first_level: int | None = Non
 
 def attn_fwd(layer: Layer, qs, ks, vs, ws=None):
     """Causal attention over the sequence -> os [BH, S, d] fp32, lse [BH, S] fp32."""
+    _need_seq(layer, qs, ks=(ks, torch.bfloat16, (layer.d,)), vs=(vs, torch.bfloat16, (layer.d,)))
     BH, S, d = qs.shape
     os_ = _empty((BH, S, d), torch.float32, qs.device)
     lse = _empty((BH, S), torch.float32, qs.device)
@@ -141,7 +184,9 @@ def attn_fwd(layer: Layer, qs, ks, vs, ws=None):
 
 
 def attn_bwd(layer: Layer, qs, ks, vs, lse, dos, delta, ws=None):
-    """-> dqs, dks, dvs [BH, S, d] fp32."""
+    """-> dqs, dks, dvs [BH, S, d] fp32.  dos: fp16 holding bf16 values."""
+    _need_seq(layer, qs, ks=(ks, torch.bfloat16, (layer.d,)), vs=(vs, torch.bfloat16, (layer.d,)),
+              lse=(lse, torch.float32, ()), dos=(dos, torch.float16, (layer.d,)), delta=(delta, torch.float32, ()))
     BH, S, d = qs.shape
     dqs, dks, dvs = (_empty((BH, S, d), torch.float32, qs.device) for _ in range(3))
     ws = _ws(0, qs.device) if ws is None else ws
@@ -153,6 +198,10 @@ def attn_bwd(layer: Layer, qs, ks, vs, lse, dos, delta, ws=None):
 def attn_fwd_rows(layer: Layer, qs, ks, vs, row_lo: int, row_hi: int, os_=None, lse=None, ws=None):
     """Rows [row_lo, row_hi) of attn_fwd's os and lse, written into os_ [BH, S, d]
     and lse [BH, S] (allocated when None; other rows left as they are)."""
+    out = {} if os_ is None else dict(os_=(os_, torch.float32, (layer.d,)))
+    if lse is not None:
+        out["lse"] = (lse, torch.float32, ())
+    _need_seq(layer, qs, ks=(ks, torch.bfloat16, (layer.d,)), vs=(vs, torch.bfloat16, (layer.d,)), **out)
     BH, S, d = qs.shape
     os_ = _empty((BH, S, d), torch.float32, qs.device) if os_ is None else os_
     lse = _empty((BH, S), torch.float32, qs.device) if lse is None else lse
@@ -165,6 +214,10 @@ def attn_fwd_rows(layer: Layer, qs, ks, vs, row_lo: int, row_hi: int, os_=None, 
 def attn_bwd_rows(layer: Layer, qs, ks, vs, lse, dos, delta, q_rows, k_rows, dqs=None, dks=None, dvs=None, ws=None):
     """dqs rows q_rows = (lo, hi) and dks, dvs rows k_rows of attn_bwd, written into
     [BH, S, d] fp32 buffers (allocated when None; other rows left as they are)."""
+    out = {n: (t, torch.float32, (layer.d,)) for n, t in (("dqs", dqs), ("dks", dks), ("dvs", dvs)) if t is not None}
+    _need_seq(layer, qs, ks=(ks, torch.bfloat16, (layer.d,)), vs=(vs, torch.bfloat16, (layer.d,)),
+              lse=(lse, torch.float32, ()), dos=(dos, torch.float16, (layer.d,)), delta=(delta, torch.float32, ()),
+              **out)
     BH, S, d = qs.shape
     dqs, dks, dvs = (_empty((BH, S, d), torch.float32, qs.device) if t is None else t for t in (dqs, dks, dvs))
     ws = _ws(0, qs.device) if ws is None else ws
@@ -175,12 +228,19 @@ def attn_bwd_rows(layer: Layer, qs, ks, vs, lse, dos, delta, q_rows, k_rows, dqs
 
 
 def scatter_back(layer: Layer, os_, slot_of):
+    info = plan(layer)
+    _need("os", os_, torch.float32, numel=layer.BH * info.S * layer.d)
+    _need("slot_of", slot_of, torch.int32, min_numel=layer.BH * info.pyr_entries)
     y = _empty((layer.B, layer.H, layer.N, layer.d), layer.torch_dtype, os_.device)
     call("lh_scatter_back", ctypes.byref(layer.cfg()), _p(os_), _p(slot_of), _p(y), _stream())
     return y
 
 
 def scatter_back_adjoint(layer: Layer, dy, seq_map, os_):
+    info = plan(layer)
+    _need_qkv(layer, dy=dy)
+    _need("os", os_, torch.float32, shape=(layer.BH, info.S, layer.d))
+    _need("seq_map", seq_map, torch.int32, min_numel=layer.BH * info.S)
     BH, S, d = os_.shape
     dos = _empty((BH, S, d), torch.float16, dy.device)  # bf16-rounded values, stored as fp16
     delta = _empty((BH, S), torch.float32, dy.device)
@@ -190,6 +250,10 @@ def scatter_back_adjoint(layer: Layer, dy, seq_map, os_):
 
 
 def pool_adjoint(layer: Layer, dqs, dks, dvs, slot_of):
+    info = plan(layer)
+    for name, t in (("dqs", dqs), ("dks", dks), ("dvs", dvs)):
+        _need(name, t, torch.float32, numel=layer.BH * info.S * layer.d)
+    _need("slot_of", slot_of, torch.int32, min_numel=layer.BH * info.pyr_entries)
     shp = (layer.B, layer.H, layer.N, layer.d)
     dq, dk, dv = (_empty(shp, layer.torch_dtype, dqs.device) for _ in range(3))
     call("lh_pool_adjoint", ctypes.byref(layer.cfg()), _p(dqs), _p(dks), _p(dvs), _p(slot_of), _p(dq), _p(dk),
@@ -244,6 +308,11 @@ class Buffers:
 
 def forward(layer: Layer, q, k, v, bufs: Buffers | None = None, y=None):
     """Whole forward -> (y, bufs).  bufs holds the saved context for backward."""
+    _need_qkv(layer, q=q, k=k, v=v)
+    if y is not None:
+        _need_qkv(layer, y=y)
+    if bufs is not None and bufs.layer != layer:
+        raise ValueError("bufs were planned for another layer")
     bufs = Buffers(layer, q.device) if bufs is None else bufs
     y = _empty((layer.B, layer.H, layer.N, layer.d), layer.torch_dtype, q.device) if y is None else y
     call("lh_forward", ctypes.byref(layer.cfg()), _p(q), _p(k), _p(v), _p(y), _p(bufs.ctx),
@@ -253,6 +322,11 @@ def forward(layer: Layer, q, k, v, bufs: Buffers | None = None, y=None):
 
 def backward(layer: Layer, dy, bufs: Buffers, grads=None):
     """Whole backward from the saved context -> (dq, dk, dv)."""
+    _need_qkv(layer, dy=dy)
+    if bufs.layer != layer:
+        raise ValueError("bufs were saved by a forward of another layer")
+    if grads is not None:
+        _need_qkv(layer, dq=grads[0], dk=grads[1], dv=grads[2])
     shp = (layer.B, layer.H, layer.N, layer.d)
     if grads is None:
         grads = tuple(_empty(shp, layer.torch_dtype, dy.device) for _ in range(3))
@@ -288,9 +362,16 @@ class LighthouseAttentionFn(torch.autograd.Function):
         return dq, dk, dv, None
 
 
-def lighthouse_attention(q, k, v, L: int, p: int, k_budget: int, chunk: int = 2048, scorer: str = "qk_sum"):
+def lighthouse_attention(q, k, v, L: int, p: int, k_budget: int, chunk: int = 2048, scorer: str = "qk_sum",
+                         selection: str = "parents"):
     """One Lighthouse attention layer over causal q, k, v of shape [B, H, N, d]."""
+    if q.dim() != 4:
+        raise ValueError(f"q: shape {tuple(q.shape)}, expected [B, H, N, d]")
     B, H, N, d = q.shape
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"q: dtype {q.dtype}, expected bfloat16 or float32")
+    for name, t in (("k", k), ("v", v)):
+        _need(name, t, q.dtype, shape=q.shape)
     dtype = {torch.bfloat16: "bf16", torch.float32: "fp32"}[q.dtype]
-    layer = Layer(B, H, N, d, L, p, k_budget, chunk, dtype, scorer)
+    layer = Layer(B, H, N, d, L, p, k_budget, chunk, dtype, scorer, selection)
     return LighthouseAttentionFn.apply(q, k, v, layer)

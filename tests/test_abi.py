@@ -265,3 +265,57 @@ def test_no_pointer_from_a_temporary():
             with open(os.path.join(pkg, f)) as fh:
                 hits += [f"{f}:{i + 1}" for i, line in enumerate(fh) if bad.search(line)]
     assert not hits, hits
+
+
+def test_binding_checks_tensor_sizes_and_dtypes_on_the_host():
+    """The library sees only pointers, so the binding refuses tensors whose
+    size or dtype does not match the layer before a pointer is passed (a
+    wrong size would make a kernel read or write outside the tensor).  CPU
+    tensors of the right size get past these checks and stop at the next one
+    (the library takes CUDA tensors)."""
+    import torch
+
+    import hierarchical_sparse_attention_pyramid_b200 as lh
+
+    layer = Layer(1, 2, 4096, 64, 3, 2, 16)
+    info = plan(layer)
+    S = info.S
+    shp = (1, 2, 4096, 64)
+    q, k, v, dy = (torch.zeros(shp, dtype=torch.bfloat16) for _ in range(4))
+    short = torch.zeros((1, 2, 4095, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="^k: "):
+        lh.forward(layer, q, short, v)
+    with pytest.raises(ValueError, match="^q: dtype"):
+        lh.forward(layer, q.float(), k, v)
+    with pytest.raises(ValueError, match="liblh takes CUDA tensors"):
+        lh.forward(layer, q, k, v)
+    other = lh.Buffers(Layer(1, 2, 4096, 64, 3, 2, 8), "cpu")
+    with pytest.raises(ValueError, match="another layer"):
+        lh.backward(layer, dy, other)
+    with pytest.raises(ValueError, match="^dy: "):
+        lh.backward(layer, short, lh.Buffers(layer, "cpu"))
+    with pytest.raises(ValueError, match="^norms: "):
+        lh.score_topk(layer, torch.zeros((2, 2, 4095), dtype=torch.float32))
+    with pytest.raises(ValueError, match="^sel: "):
+        lh.gather(layer, q, k, v, *(torch.zeros((2, info.upper_entries, 64), dtype=torch.bfloat16)
+                                    for _ in range(3)), torch.zeros(1, dtype=torch.int32))
+    qs = torch.zeros((2, S, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="^qs: shape"):
+        lh.attn_fwd(layer, torch.zeros((3, S, 64), dtype=torch.bfloat16), qs, qs)
+    with pytest.raises(ValueError, match="^vs: shape"):
+        lh.attn_fwd(layer, qs, qs, qs[:, :-1])
+    lse = torch.zeros((2, S), dtype=torch.float32)
+    with pytest.raises(ValueError, match="^dos: dtype"):
+        lh.attn_bwd(layer, qs, qs, qs, lse, qs, lse)  # dOs must be fp16
+    with pytest.raises(ValueError, match="^os_: shape"):
+        lh.attn_fwd_rows(layer, qs, qs, qs, 0, 128, torch.zeros((2, S, 32), dtype=torch.float32))
+    os_short = torch.zeros((2, S - 1, 64), dtype=torch.float32)
+    seq_map = torch.zeros((2, S), dtype=torch.int32)
+    with pytest.raises(ValueError, match="^os: shape"):
+        lh.scatter_back_adjoint(layer, dy, seq_map, os_short)
+    with pytest.raises(ValueError, match="^os: "):
+        lh.scatter_back(layer, os_short, torch.zeros((2, info.pyr_entries), dtype=torch.int32))
+    with pytest.raises(ValueError, match="^slot_of: "):
+        lh.pool_adjoint(layer, *(torch.zeros((2, S, 64)) for _ in range(3)), torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="^v: shape"):
+        lh.lighthouse_attention(q, k, short, L=3, p=2, k_budget=16)

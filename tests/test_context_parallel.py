@@ -245,7 +245,7 @@ def _rank_main(rank, world, port, name, out):
 def test_sharded_layer_matches_unsharded_oracle(name, world):
     case = CASES[name]
     N, d, L, p, kk, T, H, selection, scorer = case
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), name, out), nprocs=world, join=True)
     q, k, v, dy = _inputs(N, d, H, 3)
     want = _oracle(case, q, k, v, dy)
@@ -290,6 +290,6 @@ def test_collectives_per_layer_do_not_grow_with_heads(name):
     """One all-gather per exchanged quantity, whatever the number of heads:
     forward norms, Qs|Ks|Vs, Os, LSE; backward head sums, dOs, Delta,
     dKs|dVs, dQs."""
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_count_main, args=(2, _free_port(), name, out), nprocs=2, join=True)
     assert [out[r] for r in range(2)] == [(4, 5), (4, 5)]

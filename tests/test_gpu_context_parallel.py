@@ -60,7 +60,7 @@ def _rank_main(rank, world, port, name, out):
 def test_sharded_layer_matches_unsharded(name):
     w = CASES[name]
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), name, out), nprocs=world, join=True)
     x = pu.all_heads_case(w)
     L = lh.Layer.of(w)

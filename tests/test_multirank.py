@@ -34,7 +34,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_the_max_step_time():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     assert dict(out) == {0: 15.0, 1: 15.0}
     # whole-job tokens/s: both ranks' tokens over the slowest rank's time
