@@ -50,6 +50,18 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(name: str, t, dtype, numel: int | None = None, min_numel: int | None = None):
+    """Host check before a pointer reaches the library, which cannot see sizes."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected at least {min_numel}")
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -57,6 +69,9 @@ def _stream():
 def pool_keys(sel: Pisa, k, kpyr=None):
     """-> the key pyramid [BH, upper_entries, d] bf16 (levels >= 1)."""
     info = plan(sel)
+    _need("k", k, torch.bfloat16, numel=sel.BH * sel.N * sel.d)
+    if kpyr is not None:
+        _need("kpyr", kpyr, torch.bfloat16, min_numel=sel.BH * info.upper_entries * sel.d)
     if kpyr is None:
         kpyr = torch.empty((sel.BH, max(info.upper_entries, 1), sel.d), dtype=torch.bfloat16, device=k.device)
     call("lh_pisa_pool_keys", ctypes.byref(sel.cfg()), _p(k), _p(kpyr), _stream())
@@ -66,6 +81,15 @@ def pool_keys(sel: Pisa, k, kpyr=None):
 def select(sel: Pisa, q, k, kpyr, out=None, ws=None):
     """-> kept_idx [BH, n_groups, L, topk] int32, kept_score (same, fp32); level 0 is the selection."""
     info = plan(sel)
+    for name, t in (("q", q), ("k", k)):
+        _need(name, t, torch.bfloat16, numel=sel.BH * sel.N * sel.d)
+    _need("kpyr", kpyr, torch.bfloat16, min_numel=sel.BH * info.upper_entries * sel.d)
+    n_out = sel.BH * info.n_groups * sel.L * sel.topk
+    if out is not None:
+        _need("kept_idx", out[0], torch.int32, numel=n_out)
+        _need("kept_score", out[1], torch.float32, numel=n_out)
+    if ws is not None and ws.numel() * ws.element_size() < _lib.ERR_WORD_BYTES:
+        raise ValueError(f"ws: {ws.numel() * ws.element_size()} bytes, expected at least {_lib.ERR_WORD_BYTES}")
     dev = q.device
     if out is None:
         shp = (sel.BH, info.n_groups, sel.L, sel.topk)

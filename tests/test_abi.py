@@ -319,3 +319,27 @@ def test_binding_checks_tensor_sizes_and_dtypes_on_the_host():
         lh.pool_adjoint(layer, *(torch.zeros((2, S, 64)) for _ in range(3)), torch.zeros(1, dtype=torch.int32))
     with pytest.raises(ValueError, match="^v: shape"):
         lh.lighthouse_attention(q, k, short, L=3, p=2, k_budget=16)
+
+
+def test_pisa_binding_checks_sizes_and_dtypes_on_the_host():
+    import torch
+
+    from hierarchical_sparse_attention_pyramid_b200 import pisa
+
+    s = pisa.Pisa(1, 2, 8192, 128, 4, 3)
+    info = pisa.plan(s)
+    k = torch.zeros((1, 2, 8192, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="^k: dtype"):
+        pisa.pool_keys(s, k.float())
+    with pytest.raises(ValueError, match="^k: "):
+        pisa.pool_keys(s, k[:, :1])
+    with pytest.raises(ValueError, match="liblh takes"):
+        pisa.pool_keys(s, k)
+    kp = torch.zeros((2, info.upper_entries, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="^kpyr: "):
+        pisa.select(s, k, k, kp[:1])
+    out = (torch.zeros((2, info.n_groups, 3, 8), dtype=torch.int32), torch.zeros((2, info.n_groups, 3, 7)))
+    with pytest.raises(ValueError, match="^kept_score: "):
+        pisa.select(s, k, k, kp, out)
+    with pytest.raises(ValueError, match="^ws: "):
+        pisa.select(s, k, k, kp, ws=torch.zeros(16, dtype=torch.uint8))
