@@ -18,11 +18,13 @@ Partition (each rank r owns tokens [t0, t1) = [r N/W, (r+1) N/W)):
     contiguous segment [off_r, off_r + S_r) of the gathered sequence.  Each
     rank gathers its own segment.
   * The causal attention over S needs every earlier key: the segments of Qs,
-    Ks, Vs (and for the backward dOs, LSE, Delta) are all-gathered, and each
+    Ks, Vs (and for the backward dOs, Delta) are all-gathered, and each
     rank computes a window of rows chosen so the causal work is balanced
     (query tile t costs t+1 key tiles; key tile t costs n_tiles - t query
-    tiles).  The windows' outputs are all-gathered back so each rank reads the
-    rows of its own segment.
+    tiles).  The windows' outputs go back point to point: each rank receives
+    only the rows of its own segment (and, for Os, its halo rows) from the
+    ranks whose windows hold them; LSE, which every window's backward reads,
+    is all-gathered.
   * Halo.  R(l, i) = [e, e + p^l) starts in the entry's own shard and can run
     into the next one: for l >= 1 exactly the entry (l, t1/p^l - 1), whose
     e = t1 - 1, covers the next shard's first p^l - 1 tokens.  Forward: each
@@ -39,9 +41,9 @@ Backend interface (one object per rank; tensors are [BH, ...] per shard):
                                                 seq: per head (level, index) of the shard's
                                                 segment in causal order (local indices)
   attention(qs, ks, vs, lo, hi) -> (os, lse)    rows [lo, hi) of the causal attention
-  scatter(os_seg, seq, os_all, halo) -> y       the shard's Y; halo: per head the previous
-                                                shard's kept boundary entries (level, slot in
-                                                os_all, rows), summed into the first rows
+  scatter(os_seg, seq, halo) -> y              the shard's Y; halo: per head the previous
+                                                shard's kept boundary entries (level, Os row
+                                                [d], rows), summed into the first rows
   head_sums(dy) -> [BH, L-1, d]                 sums of dY over the shard's first p^l - 1 rows
   scatter_adjoint(dy, seq, os_seg, nxt) -> (dos, delta)
                                                 dOs over each entry's range inside the shard,
@@ -211,11 +213,67 @@ def balanced_windows(S: int, world: int, kind: str = "query") -> list[tuple[int,
 
 # ---------------------------------------------------------------- exchanges
 
+# the exchanges of one layer, in the order the driver issues them: all-gathers
+# (norms, qkv, lse, head_sums, dos, delta) and point-to-point row moves from
+# the attention windows to the segments (os, dkv, dq)
+EXCHANGES = ("norms", "qkv", "os", "lse", "head_sums", "dos", "delta", "dkv", "dq")
+# element sizes under the CUDA backend: fp32 norms, bf16 Qs|Ks|Vs, fp32 Os,
+# LSE, head sums and Delta, fp16 dOs (bf16 values), fp32 gradients
+CUDA_ELEMENT_BYTES = dict(norms=4, qkv=2, os=4, lse=4, head_sums=4, dos=2, delta=4, dkv=4, dq=4)
+# when a list, every exchange appends the elements this rank received
+EXCHANGE_LOG: list | None = None
+
+
+def _log(n: int) -> None:
+    if EXCHANGE_LOG is not None:
+        EXCHANGE_LOG.append(int(n))
+
+
+def segment_rows(counts: np.ndarray, rank: int) -> list[np.ndarray]:
+    """Per head, the sequence rows of a rank's segment."""
+    off = counts[:rank].sum(axis=0)
+    return [np.arange(off[h], off[h] + counts[rank, h], dtype=np.int64) for h in range(counts.shape[1])]
+
+
+def os_rows_needed(kept, counts: np.ndarray, shard: "Shard") -> list[np.ndarray]:
+    """Per head, the Os rows a rank reads: its segment, then the previous
+    shard's kept boundary entries (halo_in order)."""
+    seg = segment_rows(counts, shard.rank)
+    return [np.concatenate([seg[h], np.array([slot for _, slot, _ in halo_in(kept[h], shard)], np.int64)])
+            for h in range(counts.shape[1])]
+
+
+def exchange_elements(BH: int, N: int, d: int, L: int, S: int, world: int, rank: int, counts: np.ndarray,
+                      os_need) -> dict:
+    """Elements one rank receives in each exchange of a layer (forward and
+    backward).  counts: [world, BH] segment lengths; os_need: this rank's
+    os_rows_needed.  An all-gather brings world - 1 pieces padded to the
+    longest piece; a row move brings the needed rows that lie outside this
+    rank's own window."""
+    seg_rows = max(1, int(counts.max()))
+    qwin, kwin = balanced_windows(S, world, "query"), balanced_windows(S, world, "key")
+
+    def outside(rows, win):
+        lo, hi = win[rank]
+        return sum(int(((r < lo) | (r >= hi)).sum()) for r in rows)
+
+    seg = segment_rows(counts, rank)
+    wq = max(b - a for a, b in qwin)
+    out = dict(norms=(world - 1) * 2 * BH * (N // world), qkv=(world - 1) * BH * seg_rows * 3 * d,
+               os=outside(os_need, qwin) * d, lse=(world - 1) * BH * wq)
+    if L > 1:
+        out["head_sums"] = (world - 1) * BH * (L - 1) * d
+    out.update(dos=(world - 1) * BH * seg_rows * d, delta=(world - 1) * BH * seg_rows,
+               dkv=outside(seg, kwin) * 2 * d, dq=outside(seg, qwin) * d)
+    return out
+
+
 def _all_gather(parts, x: torch.Tensor, group=None) -> None:
     """dist.all_gather; CUDA tensors go through host copies when the group's
     backend is gloo (which gathers host memory), e.g. ranks sharing one GPU in
     a test."""
     import torch.distributed as dist
+    _log((len(parts) - 1) * x.numel())
     if x.is_cuda and dist.get_backend(group) == "gloo":
         host = [torch.empty(x.shape, dtype=x.dtype) for _ in parts]
         dist.all_gather(host, x.cpu(), group=group)
@@ -284,22 +342,66 @@ class CpContext:
     qs: torch.Tensor         # all-gathered sequence tensors [BH, S, d]
     ks: torch.Tensor
     vs: torch.Tensor
-    os: torch.Tensor         # [BH, S, d]
+    os: torch.Tensor         # [BH, max segment, d]: Os rows of this rank's segment
     lse: torch.Tensor        # [BH, S]
 
 
-def _segment_rows(full: torch.Tensor, off, counts_r) -> torch.Tensor:
-    """Rows [off_h, off_h + S_r,h) of every head (same count for every head is
-    not assumed: heads are padded to the largest with zeros)."""
-    BH = full.shape[0]
-    mx = int(max(counts_r))
-    j = np.arange(mx, dtype=np.int64)[None, :]
-    valid = j < np.asarray(counts_r, np.int64)[:, None]
-    src = np.where(valid, np.asarray(off, np.int64)[:, None] + j, 0)
-    dev = full.device
-    out = full[torch.arange(BH, device=dev)[:, None], torch.from_numpy(src).to(dev)]
-    out[torch.from_numpy(~valid).to(dev)] = 0
-    return out
+def redistribute_rows(x_w: torch.Tensor, windows, need, group=None) -> torch.Tensor:
+    """Move the rows of window-distributed tensors to the ranks that read them.
+    x_w: this rank's rows [lo, hi) of its window, every head: [BH, hi - lo, ...]
+    (windows[rank] = (lo, hi)); need[q][h]: the sequence rows rank q reads of
+    head h (every rank passes the same windows and need).  Each rank sends
+    each other rank, in one batch of point-to-point transfers, the rows it
+    needs from this window, packed head by head, and copies its own.  Returns
+    [BH, max_h len(need[rank][h]), ...]: row j of head h holds sequence row
+    need[rank][h][j] (zeros past a head's rows)."""
+    import torch.distributed as dist
+    W, r = dist.get_world_size(group), dist.get_rank(group)
+    lo, hi = windows[r]
+    BH, rest, dev = x_w.shape[0], tuple(x_w.shape[2:]), x_w.device
+    mx = max(1, max(len(n) for n in need[r]))
+    out = torch.zeros((BH * mx,) + rest, dtype=x_w.dtype, device=dev)
+    src = x_w.contiguous().reshape((BH * (hi - lo),) + rest)
+
+    def inside(rows_of_heads, a, b):  # per head: (positions in the list, rows) inside [a, b)
+        return [(np.nonzero((rows >= a) & (rows < b))[0], rows[(rows >= a) & (rows < b)]) for rows in rows_of_heads]
+
+    def index(parts, row_of):  # flat indices, head by head
+        return torch.from_numpy(np.concatenate([row_of(h, j, rows) for h, (j, rows) in enumerate(parts)]
+                                               + [np.zeros(0, np.int64)]).astype(np.int64)).to(dev)
+
+    def src_index(parts):  # rows of this window
+        return index(parts, lambda h, j, rows: h * (hi - lo) + (rows - lo))
+
+    def dst_index(parts):  # positions in this rank's list
+        return index(parts, lambda h, j, rows: h * mx + j)
+
+    own = inside(need[r], lo, hi)
+    if sum(len(j) for j, _ in own):
+        out[dst_index(own)] = src[src_index(own)]
+    # gloo moves host memory: stage through it (ranks sharing a GPU in a test)
+    stage = torch.device("cpu") if dist.get_backend(group) == "gloo" else dev
+    ops, recvs = [], []
+    for q in range(W):
+        if q == r:
+            continue
+        peer = q if group is None else dist.get_global_rank(group, q)
+        send = inside(need[q], lo, hi)
+        if sum(len(j) for j, _ in send):
+            ops.append(dist.P2POp(dist.isend, src[src_index(send)].to(stage), peer, group))
+        recv = inside(need[r], *windows[q])
+        n = sum(len(j) for j, _ in recv)
+        if n:
+            buf = torch.empty((n,) + rest, dtype=x_w.dtype, device=stage)
+            ops.append(dist.P2POp(dist.irecv, buf, peer, group))
+            recvs.append((buf, dst_index(recv)))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+    _log(sum(b.numel() for b, _ in recvs))
+    for buf, idx in recvs:
+        out[idx] = buf.to(dev)
+    return out.reshape((BH, mx) + rest)
 
 
 def cp_forward(backend, shard: Shard, q, k, v, selection: str = "parents", group=None):
@@ -318,14 +420,21 @@ def cp_forward(backend, shard: Shard, q, k, v, selection: str = "parents", group
     qkv = allgather_segments(torch.stack((qs_r, ks_r, vs_r), dim=2), counts, group)
     qs, ks, vs = (qkv[:, :, t].contiguous() for t in range(3))
     S = qs.shape[1]
-    lo, hi = balanced_windows(S, W, "query")[r]
+    qwin = balanced_windows(S, W, "query")
+    lo, hi = qwin[r]
     os_w, lse_w = backend.attention(qs, ks, vs, lo, hi)
-    win = [b - a for a, b in balanced_windows(S, W, "query")]
-    os_f = allgather_rows(os_w, win, group)
-    lse_f = allgather_rows(lse_w[..., None], win, group)[..., 0]
-    halo = [halo_in(kept[h], shard) for h in range(BH)]
-    y = backend.scatter(_segment_rows(os_f, off, counts[r]), seq, os_f, halo)
-    ctx = CpContext(seq=seq, kept=kept, counts=counts, off=off, qs=qs, ks=ks, vs=vs, os=os_f, lse=lse_f)
+    # Os rows go to the ranks that read them (their segments and halo rows);
+    # LSE, read by every window of the backward, to every rank
+    need = [os_rows_needed(kept, counts, Shard(N, p, L, W, q_)) for q_ in range(W)]
+    os_need = redistribute_rows(os_w, qwin, need, group)
+    lse_f = allgather_rows(lse_w[..., None], [b - a for a, b in qwin], group)[..., 0]
+    mxs = int(counts[r].max())
+    os_seg = os_need[:, :mxs].clone()
+    os_seg[torch.from_numpy(np.arange(mxs)[None, :] >= counts[r][:, None]).to(os_seg.device)] = 0
+    halo = [[(l, os_need[h, int(counts[r, h]) + i], rows) for i, (l, _, rows) in enumerate(halo_in(kept[h], shard))]
+            for h in range(BH)]
+    y = backend.scatter(os_seg, seq, halo)
+    ctx = CpContext(seq=seq, kept=kept, counts=counts, off=off, qs=qs, ks=ks, vs=vs, os=os_seg, lse=lse_f)
     return y, ctx
 
 
@@ -337,7 +446,7 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     if L > 1:
         heads_all = allgather_cat(backend.head_sums(dy)[None], dim=0, group=group)  # [W, BH, L-1, d]
         nxt = heads_all[r + 1] if r + 1 < W else None
-    dos, delta = backend.scatter_adjoint(dy, ctx.seq, _segment_rows(ctx.os, ctx.off, ctx.counts[r]), nxt)
+    dos, delta = backend.scatter_adjoint(dy, ctx.seq, ctx.os, nxt)
     dos_f = allgather_segments(dos, ctx.counts, group)
     delta_f = allgather_segments(delta, ctx.counts, group)
     S = ctx.qs.shape[1]
@@ -345,11 +454,11 @@ def cp_backward(backend, shard: Shard, dy, ctx: CpContext, group=None):
     qlo, qhi = balanced_windows(S, W, "query")[r]
     dks_w, dvs_w = backend.attention_bwd_kv(ctx.qs, ctx.ks, ctx.vs, ctx.lse, dos_f, delta_f, klo, khi)
     dqs_w = backend.attention_bwd_q(ctx.qs, ctx.ks, ctx.vs, ctx.lse, dos_f, delta_f, qlo, qhi)
-    kwin = [b - a for a, b in balanced_windows(S, W, "key")]
-    qwin = [b - a for a, b in balanced_windows(S, W, "query")]
-    dkv = _segment_rows(allgather_rows(torch.stack((dks_w, dvs_w), dim=2), kwin, group), ctx.off, ctx.counts[r])
+    # each gradient row goes to the rank whose segment holds it
+    seg = [segment_rows(ctx.counts, q_) for q_ in range(W)]
+    dkv = redistribute_rows(torch.stack((dks_w, dvs_w), dim=2), balanced_windows(S, W, "key"), seg, group)
     dks, dvs = dkv[:, :, 0].contiguous(), dkv[:, :, 1].contiguous()
-    dqs = _segment_rows(allgather_rows(dqs_w, qwin, group), ctx.off, ctx.counts[r])
+    dqs = redistribute_rows(dqs_w, balanced_windows(S, W, "query"), seg, group)
     return backend.pool_adjoint(dqs, dks, dvs, ctx.seq)
 
 
@@ -432,13 +541,13 @@ class CudaBackend:
         os_, lse = self.api.attn_fwd_rows(self.layer, qs.contiguous(), ks.contiguous(), vs.contiguous(), lo, hi)
         return os_[:, lo:hi], lse[:, lo:hi]
 
-    def scatter(self, os_seg, seq, os_all, halo):
+    def scatter(self, os_seg, seq, halo):
         from . import _lib
         lay = self.layer
         hal = torch.zeros((lay.BH, max(lay.L - 1, 1), lay.d), dtype=torch.float32, device=os_seg.device)
         for h, ents in enumerate(halo):
-            for l, slot, rows in ents:
-                hal[h, l - 1] = os_all[h, slot]
+            for l, row, rows in ents:
+                hal[h, l - 1] = row
         y = torch.empty((lay.B, lay.H, self.shard.n, lay.d), dtype=torch.bfloat16, device=os_seg.device)
         (os_seg,) = _contiguous(os_seg)
         p_ = self.api._p

@@ -172,12 +172,12 @@ class OracleBackend:
             lse.append(torch.from_numpy(ls[a:b]))
         return torch.stack(os_), torch.stack(lse)
 
-    def scatter(self, os_seg, seq, os_all, halo):
+    def scatter(self, os_seg, seq, halo):
         y = torch.stack([torch.from_numpy(lo.scatter_back(os_seg[h, :len(lv)].numpy(), lv, ix, self.n, self.p,
                                                           self.L)) for h, (lv, ix) in enumerate(seq)])
         for h, ents in enumerate(halo):
-            for l, slot, rows in ents:
-                y[h, :rows] += os_all[h, slot]
+            for l, row, rows in ents:
+                y[h, :rows] += row
         return y
 
     def head_sums(self, dy):
@@ -261,14 +261,7 @@ def _count_main(rank, world, port, name, out):
 
     import torch.distributed as dist
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
-    calls = []
-    real = cp._all_gather
-
-    def counting(parts, x, group=None):
-        calls.append(tuple(x.shape))
-        real(parts, x, group=group)
-
-    cp._all_gather = counting
+    calls = cp.EXCHANGE_LOG = []
     try:
         case = CASES[name]
         N, d, L, p, kk, T, H, selection, scorer = case
@@ -279,17 +272,20 @@ def _count_main(rank, world, port, name, out):
         y, ctx = cp.cp_forward(be, shard, q[:, sl], k[:, sl], v[:, sl], selection)
         n_fwd = len(calls)
         cp.cp_backward(be, shard, dy[:, sl].contiguous(), ctx)
-        out[rank] = (n_fwd, len(calls) - n_fwd)
+        need = cp.os_rows_needed(ctx.kept, ctx.counts, shard)
+        want = cp.exchange_elements(H, N, d, L, ctx.qs.shape[1], world, rank, ctx.counts, need)
+        out[rank] = (n_fwd, len(calls) - n_fwd, calls == [want[n] for n in cp.EXCHANGES if n in want])
     finally:
-        cp._all_gather = real
+        cp.EXCHANGE_LOG = None
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("name", ["p2_L3", "direct_p2_L4"])
 def test_collectives_per_layer_do_not_grow_with_heads(name):
-    """One all-gather per exchanged quantity, whatever the number of heads:
-    forward norms, Qs|Ks|Vs, Os, LSE; backward head sums, dOs, Delta,
-    dKs|dVs, dQs."""
+    """One exchange per quantity, whatever the number of heads: forward norms,
+    Qs|Ks|Vs (all-gathers), Os (rows to the ranks that read them), LSE;
+    backward head sums, dOs, Delta (all-gathers), dKs|dVs, dQs (rows to the
+    segments' ranks); each rank receiving what exchange_elements predicts."""
     out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_count_main, args=(2, _free_port(), name, out), nprocs=2, join=True)
-    assert [out[r] for r in range(2)] == [(4, 5), (4, 5)]
+    assert [out[r] for r in range(2)] == [(4, 5, True), (4, 5, True)]
