@@ -240,8 +240,7 @@ def _rank_main(rank, world, port, name, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("name", sorted(CASES))
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("name,world", [(n, w) for n in sorted(CASES) for w in (2, 4)] + [("p4_L4", 8)])
 def test_sharded_layer_matches_unsharded_oracle(name, world):
     case = CASES[name]
     N, d, L, p, kk, T, H, selection, scorer = case
