@@ -288,3 +288,43 @@ def test_collectives_per_layer_do_not_grow_with_heads(name):
     out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_count_main, args=(2, _free_port(), name, out), nprocs=2, join=True)
     assert [out[r] for r in range(2)] == [(4, 5, True), (4, 5, True)]
+
+
+def _redistribute_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        g = np.random.default_rng(11)  # the same draws on every rank
+        ok = []
+        for dtype in (torch.float32, torch.bfloat16, torch.float16):
+            BH, S = 3, 700
+            X = torch.from_numpy(g.standard_normal((BH, S, 2, 5))).to(dtype)
+            # windows tile [0, S), one of them empty
+            cuts = np.sort(g.choice(np.arange(1, S), world - 2, replace=False))
+            cuts = [0, 0] + list(cuts) + [S] if world > 2 else [0, 0, S]
+            windows = list(zip(cuts[:-1], cuts[1:]))[:world]
+            windows[-1] = (windows[-1][0], S)
+            # every rank reads an arbitrary, unsorted set of rows per head (some none)
+            need = [[g.permutation(S)[:g.integers(0, 200)] for _ in range(BH)] for _ in range(world)]
+            lo, hi = windows[rank]
+            got = cp.redistribute_rows(X[:, lo:hi], windows, need, None)
+            mx = max(1, max(len(n) for n in need[rank]))
+            want = torch.zeros((BH, mx, 2, 5), dtype=dtype)
+            for h in range(BH):
+                want[h, :len(need[rank][h])] = X[h, torch.from_numpy(need[rank][h])]
+            ok.append(got.dtype == dtype and torch.equal(got, want))
+        out[rank] = all(ok)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_redistribute_rows_delivers_every_needed_row():
+    """Each rank gets exactly the rows it asks for, in its own order, from
+    whichever rank's window holds them (an empty window included), for the
+    dtypes the CUDA backend exchanges; rows past a head's list are zero."""
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_redistribute_main, args=(3, _free_port(), out), nprocs=3, join=True)
+    assert [out[r] for r in range(3)] == [True] * 3
